@@ -1,0 +1,540 @@
+#!/usr/bin/env python3
+"""Benchmark of MoE token dispatch + combine on B200 (libepx, sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl epx|reference]
+
+A step is one pass of the hot path over one batch: routing layout ->
+dispatch/expand -> combine reduce (the stand-in expert output that combine
+reads is produced once before timing; the stand-in is not part of the
+metric).  Prints ONE JSON line on rank 0.
+
+N > 1 (launched by torch.distributed.run): every rank runs an independent
+replica on its own GPU with its own seeded batch (weak scaling, no
+collective on the data path); a barrier brackets the timed region and the
+elapsed time is the max over ranks.
+
+--impl reference times the CPU oracle (single-threaded C) on the host on a
+bounded sample of the same workload, for the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine tokens/s at 7168×top8; achieved HBM GB/s vs B200 roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+DESCRIBE = {
+    "tiny": "tiny T=128 H=256 E=16 R=4 top-4 uniform",
+    "decode": "decode T=128 H=7168 E=256 R=16 top-8 uniform",
+    "prefill": "prefill-skew T=4096 H=7168 E=256 R=16 top-8 zipf(1.2)",
+    "lowbatch1": "low-batch T=1 H=3584 E=896 R=32 top-16 (1 real row)",
+    "lowbatch2": "low-batch T=2 H=3584 E=896 R=32 top-16 (1 real row)",
+    "lowbatch4": "low-batch T=4 H=3584 E=896 R=32 top-16 (1 real row)",
+    "lowbatch8": "low-batch T=8 H=3584 E=896 R=32 top-16 (1 real row)",
+    "dp_compact": "dp-batch [120,1x7] compact 127 rows H=7168 E=256 R=16 top-8",
+    "dp_padded": "dp-batch [120,1x7] padded to 960 rows H=7168 E=256 R=16 top-8",
+}
+
+# sources whose hash keys the committed ncu DRAM traffic figure
+KERNEL_SOURCES = {
+    "dispatch_expand": ["combine_ep_layout_07_b200/csrc/dispatch.cu",
+                        "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "combine_reduce": ["combine_ep_layout_07_b200/csrc/combine.cu",
+                       "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "layout": ["combine_ep_layout_07_b200/csrc/layout.cu",
+               "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+
+
+# ------------------------------------------------------------------ helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["epx", "reference"], default="epx")
+    ap.add_argument("--workload", choices=sorted(DESCRIBE), default="prefill")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--dispatch-variant", type=int, default=0)
+    ap.add_argument("--combine-variant", type=int, default=0)
+    ap.add_argument("--idx-bits", type=int, choices=[32, 64], default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--flush", choices=["auto", "always", "never"], default="auto")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes):
+    """Algorithmic HBM bytes per step of each kernel (each byte the definition
+    must move once; no re-reads)."""
+    row = H * 2
+    layout = T * k * idx_bytes + T * k * 4 + T * R * 4
+    dispatch = T_real * row + (N_recv + N_route) * row + T * k * 4 + T * R * 4
+    combine = N_route * row + T * row + T * k * (4 + 4)
+    return dict(layout=layout, dispatch_expand=dispatch, combine_reduce=combine,
+                total=layout + dispatch + combine)
+
+
+def sources_hash(kernel):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; otherwise None."""
+    try:
+        lines = open(TRAFFIC_FILE).read().splitlines()
+    except OSError:
+        return None
+    want = sources_hash(kernel)
+    for ln in lines:
+        if ln.startswith("#") or not ln.strip():
+            continue
+        kv = dict(x.split("=", 1) for x in ln.split() if "=" in x)
+        if (kv.get("kernel") == kernel and kv.get("workload") == workload
+                and kv.get("source") == want):
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+        self.error = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", self.gpu_id],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception as e:  # nvidia-smi missing
+            self.error = str(e)
+            return
+        t0 = time.time()
+        while time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t_lo, t_hi):
+        if self.error or not self.path:
+            return {"error": self.error or "not started"}
+        rows = []
+        for ln in open(self.path).read().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append(dict(ts=ts, sm=float(parts[2]), smax=float(parts[3]),
+                                 power=parts[4], active=parts[5], hw=parts[6],
+                                 hwt=parts[7], swt=parts[8], pcap=parts[9]))
+            except (ValueError, IndexError):
+                continue
+        os.unlink(self.path)
+        inwin = [r for r in rows if t_lo - 0.25 <= r["ts"] <= t_hi + 0.25]
+        window = "timed"
+        if len(inwin) < 3:
+            inwin, window = rows, "whole run (timed region shorter than the sampling period)"
+        if not inwin:
+            return {"error": "no samples"}
+        reasons = set()
+        for r in inwin:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in inwin),
+                "sm_max_mhz": max(r["smax"] for r in inwin),
+                "reasons": sorted(reasons), "samples": len(inwin), "window": window}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = torch.cuda.get_device_properties(dev).uuid
+        s = str(u)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    except Exception:
+        return str(dev)
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_pass(oracle, wl, y_bits, idx):
+    """One oracle pass of the timed path (layout, dispatch/expand, combine)."""
+    lay = oracle.layout(idx, wl["E"], wl["R"])
+    oracle.dispatch_expand(wl["x"], lay)
+    return oracle.combine(y_bits, wl["topk_weights"], lay), lay
+
+
+def slice_workload(wl, n):
+    out = dict(wl)
+    for key in ("x", "topk_idx", "topk_weights"):
+        out[key] = np.ascontiguousarray(wl[key][:n])
+    out["T"] = n
+    return out
+
+
+def cpu_baseline(wl, budget_s, idx_bits):
+    """Oracle, as it stands, over the full workload repeated for ~budget_s."""
+    import oracle
+    oracle.build()
+    idx = wl["topk_idx"].astype(np.int64 if idx_bits == 64 else np.int32)
+    lay = oracle.layout(idx, wl["E"], wl["R"])
+    _, expanded = oracle.dispatch_expand(wl["x"], lay)
+    y = oracle.standin(expanded, lay)
+    passes, t0 = 0, time.perf_counter()
+    out = None
+    while True:
+        out, _ = oracle_pass(oracle, wl, y, idx)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    value = lay["T_real"] * passes / el
+    return dict(value=value, unit=UNIT, cores=1, kind="oracle",
+                sample=f"{passes} full pass(es) of the {wl['name']} workload "
+                       f"({lay['T_real']} effective tokens each) in {el:.1f} s, "
+                       f"single-threaded C, layout+dispatch/expand+combine"), \
+        dict(layout=lay, expanded=expanded, y=y, out=out)
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0            # rank 0 alone runs the CPU oracle
+    import oracle
+    from combine_ep_layout_07_b200 import workloads as wlmod
+    oracle.build()
+    wl = wlmod.make(args.workload, seed=args.seed)
+    idx_full = wl["topk_idx"].astype(np.int64 if args.idx_bits == 64 else np.int32)
+    # calibrate the per-token oracle cost, then size the sample so the whole
+    # run (warm-up + timed) takes about two minutes at most
+    n_cal = min(wl["T"], 64)
+    sub = slice_workload(wl, n_cal)
+    sidx = idx_full[:n_cal]
+    slay = oracle.layout(sidx, wl["E"], wl["R"])
+    _, sex = oracle.dispatch_expand(sub["x"], slay)
+    sy = oracle.standin(sex, slay)
+    t0 = time.perf_counter()
+    oracle_pass(oracle, sub, sy, sidx)
+    per_tok = (time.perf_counter() - t0) / n_cal
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(wl["T"], budget / max(per_tok, 1e-9))))
+    sub = slice_workload(wl, n)
+    sidx = np.ascontiguousarray(idx_full[:n])
+    slay = oracle.layout(sidx, wl["E"], wl["R"])
+    _, sex = oracle.dispatch_expand(sub["x"], slay)
+    sy = oracle.standin(sex, slay)
+    for _ in range(args.warmup):
+        oracle_pass(oracle, sub, sy, sidx)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(oracle, sub, sy, sidx)
+    el = time.perf_counter() - t0
+    units = slay["T_real"] * args.steps
+    value = units / el
+    sample = (f"first {n} of {wl['T']} rows of the {wl['name']} workload "
+              f"({slay['T_real']} effective tokens) per step, single-threaded C oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate / bf16 data",
+        "data": "synthetic", "config": workload_config(wl, args, slay),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(wl, args, lay_totals, flush_desc=None):
+    cfg = {"workload": DESCRIBE[args.workload], "T": wl["T"], "H": wl["H"], "E": wl["E"],
+           "R": wl["R"], "k": wl["k"], "seed": args.seed, "idx_bits": args.idx_bits,
+           "T_real": int(lay_totals["T_real"]), "N_recv": int(lay_totals["N_recv"]),
+           "N_route": int(lay_totals["N_route"]),
+           "timed": "layout + dispatch_expand + combine_reduce",
+           "parallelism": f"replicas x{dist_env()[1]}"}
+    if flush_desc:
+        cfg["l2"] = flush_desc
+    return cfg
+
+
+# ---------------------------------------------------------------- epx arm
+
+def run_epx(args):
+    import torch
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl epx needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    from combine_ep_layout_07_b200 import epx
+    from combine_ep_layout_07_b200 import workloads as wlmod
+
+    wl = wlmod.make(args.workload, seed=args.seed + rank)
+    T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
+    itype = torch.int64 if args.idx_bits == 64 else torch.int32
+    x = torch.from_numpy(wl["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+    idx = torch.from_numpy(wl["topk_idx"]).to(itype).to(dev)
+    w = torch.from_numpy(wl["topk_weights"]).to(dev)
+    stream = torch.cuda.Stream(device=dev)
+    lay = epx.Layout(T, k, E, R, args.idx_bits, device=dev)
+    recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=dev)
+    expanded = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16, device=dev)
+    y = torch.empty_like(expanded)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+
+    def step_kernels(events=None):
+        if events is not None:
+            events[0].record(stream)
+        epx.layout(idx, E, R, out=lay, stream=stream)
+        if events is not None:
+            events[1].record(stream)
+        epx.dispatch_expand(x, lay, recv=recv, expanded=expanded,
+                            variant=args.dispatch_variant, stream=stream)
+        if events is not None:
+            events[2].record(stream)
+        epx.combine_reduce(y, w, lay, out=out, variant=args.combine_variant, stream=stream)
+        if events is not None:
+            events[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        epx.layout(idx, E, R, out=lay, stream=stream)
+        epx.dispatch_expand(x, lay, recv=recv, expanded=expanded, stream=stream)
+        epx.standin_expert(expanded, lay, y=y, stream=stream)
+    tot = epx.read_totals(lay, stream=stream)
+
+    bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
+                       args.idx_bits // 8)
+    working = bytes_["total"]
+    flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
+    flush_desc = ("L2 flushed between steps (256 MiB write, outside the timed events)" if flush
+                  else f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)")
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            if flush:
+                flush_buf.add_(1)
+            step_kernels()
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+
+    sampler = ClockSampler(gpu_uuid(torch, local)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    t_lo = time.time()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            if flush:
+                flush_buf.add_(1)
+            step_kernels(evs[i])
+    torch.cuda.synchronize(dev)
+    t_hi = time.time()
+    if pg:
+        pg.barrier()
+    if sampler:
+        sampler.stop()
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    k_ms = {"layout": [e[0].elapsed_time(e[1]) for e in evs],
+            "dispatch_expand": [e[1].elapsed_time(e[2]) for e in evs],
+            "combine_reduce": [e[2].elapsed_time(e[3]) for e in evs]}
+    total_ms = sum(step_ms)
+    if pg:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    units = tot["T_real"] * args.steps * world
+    value = units / (total_ms / 1e3)
+
+    # ---- e2e through the host-buffer C-ABI call
+    e2e = run_e2e(torch, epx, wl, args, dev, stream, pg, world, tot["T_real"])
+
+    if rank != 0:
+        finish(pg)
+        return 0
+
+    peak, peak_kind = load_peaks()
+    kernels = {}
+    for name, ms in k_ms.items():
+        avg_s = statistics.fmean(ms) / 1e3
+        gbs = bytes_[name] / avg_s / 1e9
+        kernels[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
+                         "alg_bytes": bytes_[name], "gbs": gbs, "frac": gbs / peak}
+    dom = max(kernels, key=lambda n: kernels[n]["us"])
+    traffic = committed_traffic(dom, args.workload)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
+                "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind ==
+                "measured" else "fallback 6.65 TB/s",
+                "traffic": traffic}
+    step_gbs = bytes_["total"] / (total_ms / args.steps / 1e3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(wl, args, tot, flush_desc),
+        "roofline": roofline,
+        "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
+        "kernels": kernels,
+        "gpu_launches": 3 * args.steps,
+        "e2e": e2e,
+    }
+    if sampler:
+        line["clocks"] = sampler.summary(t_lo, t_hi)
+    if world == 1 and not args.no_cpu_baseline:
+        cb, ores = cpu_baseline(wl, args.cpu_budget, args.idx_bits)
+        line["cpu_baseline"] = cb
+        line["parity"] = parity_summary(torch, lay, expanded, out, ores)
+    print(json.dumps(line), flush=True)
+    finish(pg)
+    return 0
+
+
+def parity_summary(torch, lay, expanded, out, ores):
+    """Whole-output comparison with the oracle on the benchmarked workload."""
+    from combine_ep_layout_07_b200 import workloads as wlmod
+    o = ores["layout"]
+    pos_ok = bool(np.array_equal(lay.pos.cpu().numpy(), o["pos"]))
+    ne = o["N_route"]
+    ex = expanded[:ne].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    ex_ok = bool(np.array_equal(ex, ores["expanded"]))
+    g = wlmod.bf16_bits_to_f32(out.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+    r = wlmod.bf16_bits_to_f32(ores["out"])
+    ok = bool(np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-3))
+    return {"layout_pos_bit_exact": pos_ok, "expanded_bit_exact": ex_ok,
+            "combine_within_tol": ok}
+
+
+def run_e2e(torch, epx, wl, args, dev, stream, pg, world, T_real):
+    T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
+    itype = torch.int64 if args.idx_bits == 64 else torch.int32
+    x_h = torch.from_numpy(wl["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    i_h = torch.from_numpy(wl["topk_idx"]).to(itype).pin_memory()
+    w_h = torch.from_numpy(wl["topk_weights"]).pin_memory()
+    out_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    nbytes = epx.roundtrip_device_bytes(T, H, k, E, R, args.idx_bits)
+    dmem = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    n = max(1, args.e2e_steps)
+    for _ in range(3):
+        epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem, out_h, stream=stream)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem, out_h, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = x_h.numel() * 2 + i_h.numel() * i_h.element_size() + w_h.numel() * 4
+    d2h = out_h.numel() * 2
+    return {"value": T_real * n * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n,
+            "path": "ep_roundtrip_host: pinned host -> device, layout, dispatch/expand, "
+                    "stand-in expert, combine, device -> host"}
+
+
+def finish(pg):
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_epx(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,8 @@
+"""epx: B200-native (sm_100a) MoE token dispatch and combine.
+
+The compute path is libepx.so (hand-written CUDA, C ABI in include/epx.h);
+``combine_ep_layout_07_b200.epx`` is its argument-marshalling binding.
+``combine_ep_layout_07_b200.workloads`` draws the seeded synthetic inputs.
+"""
+from .epx import (EpxError, Layout, combine_reduce, dispatch_expand, layout,  # noqa: F401
+                  read_totals, roundtrip_device_bytes, roundtrip_host, standin_expert)

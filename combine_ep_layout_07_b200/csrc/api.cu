@@ -1,0 +1,318 @@
+// C ABI of libepx: argument validation, layout carving and launches.
+// The operations themselves are documented in include/epx.h.
+#include <string.h>
+
+#include "epx_internal.cuh"
+
+using namespace epx;
+
+namespace {
+
+inline cudaStream_t as_stream(void *s) { return static_cast<cudaStream_t>(s); }
+
+inline bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool sizes_ok(int32_t T, int32_t k, int32_t E, int32_t R)
+{
+    if (T < 0 || k < 1 || E < 1 || R < 1) return false;
+    if (k > EPX_MAX_TOPK || R > EPX_MAX_RANKS || E > EPX_MAX_EXPERTS) return false;
+    if (E % R != 0) return false;
+    if ((int64_t)T * k > INT32_MAX || (int64_t)T * R > INT32_MAX) return false;
+    return true;
+}
+
+bool layout_ok(const ep_layout_t *L)
+{
+    if (!L) return false;
+    if (!sizes_ok(L->T, L->k, L->E, L->R)) return false;
+    if (L->idx_bits != 32 && L->idx_bits != 64) return false;
+    return L->cnt_e && L->off_e && L->cnt_r && L->off_r && L->pos && L->recv_pos && L->totals;
+}
+
+ep_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t ep_abi_version(void) { return EPX_ABI_VERSION; }
+
+const char *ep_status_str(ep_status_t s)
+{
+    switch (s) {
+    case EP_OK: return "EP_OK";
+    case EP_ERR_INVALID_ARG: return "EP_ERR_INVALID_ARG: invalid argument";
+    case EP_ERR_MISALIGNED: return "EP_ERR_MISALIGNED: buffer not 16-byte aligned";
+    case EP_ERR_CAPACITY: return "EP_ERR_CAPACITY: a destination row exceeded a capacity";
+    case EP_ERR_BAD_INDEX: return "EP_ERR_BAD_INDEX: a topk index < -1 or >= E was dropped";
+    case EP_ERR_CUDA: return "EP_ERR_CUDA: CUDA runtime error";
+    case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED: size beyond a library limit";
+    }
+    return "EP_ERR_UNKNOWN";
+}
+
+size_t ep_layout_bytes(int32_t T, int32_t k, int32_t E, int32_t R)
+{
+    if (!sizes_ok(T, k, E, R)) return 0;
+    size_t n = 0;
+    n += round_up(sizeof(int32_t) * (size_t)E, 16);
+    n += round_up(sizeof(int32_t) * ((size_t)E + 1), 16);
+    n += round_up(sizeof(int32_t) * (size_t)R, 16);
+    n += round_up(sizeof(int32_t) * ((size_t)R + 1), 16);
+    n += round_up(sizeof(int32_t) * (size_t)T * k, 16);
+    n += round_up(sizeof(int32_t) * (size_t)T * R, 16);
+    n += round_up(sizeof(int32_t) * 4, 16);
+    return n;
+}
+
+ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E, int32_t R,
+                           int32_t idx_bits, void *dev_mem, size_t bytes)
+{
+    if (!L || !dev_mem) return EP_ERR_INVALID_ARG;
+    if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return EP_ERR_INVALID_ARG;
+    if (k > EPX_MAX_TOPK || R > EPX_MAX_RANKS || E > EPX_MAX_EXPERTS) return EP_ERR_UNSUPPORTED;
+    if (!sizes_ok(T, k, E, R)) return EP_ERR_INVALID_ARG;
+    if (idx_bits != 32 && idx_bits != 64) return EP_ERR_INVALID_ARG;
+    if (!aligned(dev_mem, 16)) return EP_ERR_MISALIGNED;
+    if (bytes < ep_layout_bytes(T, k, E, R)) return EP_ERR_INVALID_ARG;
+    char *p = static_cast<char *>(dev_mem);
+    auto take = [&](size_t n) {
+        int32_t *r = reinterpret_cast<int32_t *>(p);
+        p += round_up(sizeof(int32_t) * n, 16);
+        return r;
+    };
+    ep_layout_t l;
+    memset(&l, 0, sizeof l);
+    l.T = T;
+    l.k = k;
+    l.E = E;
+    l.R = R;
+    l.idx_bits = idx_bits;
+    l.cnt_e = take((size_t)E);
+    l.off_e = take((size_t)E + 1);
+    l.cnt_r = take((size_t)R);
+    l.off_r = take((size_t)R + 1);
+    l.pos = take((size_t)T * k);
+    l.recv_pos = take((size_t)T * R);
+    l.totals = take(4);
+    *L = l;
+    return EP_OK;
+}
+
+ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (L->T > 0 && !topk_idx) return EP_ERR_INVALID_ARG;
+    if (topk_idx && !aligned(topk_idx, (size_t)L->idx_bits / 8)) return EP_ERR_MISALIGNED;
+    LayoutParams p;
+    memset(&p, 0, sizeof p);
+    p.idx = topk_idx;
+    p.T = L->T;
+    p.k = L->k;
+    p.E = L->E;
+    p.R = L->R;
+    p.epr = L->E / L->R;
+    p.cnt_e = L->cnt_e;
+    p.off_e = L->off_e;
+    p.cnt_r = L->cnt_r;
+    p.off_r = L->off_r;
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.totals = L->totals;
+    return from_cuda(launch_layout(p, L->idx_bits, as_stream(stream)));
+}
+
+ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout_t *L,
+                                       void *recv, int64_t recv_cap, void *expanded,
+                                       int64_t exp_cap, int32_t variant, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || recv_cap < 0 || exp_cap < 0) return EP_ERR_INVALID_ARG;
+    if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!x || !recv || !expanded) return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(recv, 16) || !aligned(expanded, 16)) return EP_ERR_MISALIGNED;
+    DispatchParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint4 *>(x);
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.T = L->T;
+    p.k = L->k;
+    p.R = L->R;
+    p.V = H / 8;
+    p.recv = static_cast<uint4 *>(recv);
+    p.recv_cap = recv_cap;
+    p.expanded = static_cast<uint4 *>(expanded);
+    p.exp_cap = exp_cap;
+    p.err = L->totals + 3;
+    return from_cuda(launch_dispatch(p, variant, as_stream(stream)));
+}
+
+ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L, void *recv,
+                               int64_t recv_cap, void *expanded, int64_t exp_cap, void *stream)
+{
+    return ep_dispatch_expand_variant(x, H, L, recv, recv_cap, expanded, exp_cap, 0, stream);
+}
+
+ep_status_t ep_standin_expert(const void *expanded, int32_t H, const ep_layout_t *L, void *y,
+                              int64_t rows, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || rows < 0) return EP_ERR_INVALID_ARG;
+    if (rows == 0 || L->T == 0) return EP_OK;
+    if (!expanded || !y) return EP_ERR_INVALID_ARG;
+    if (!aligned(expanded, 16) || !aligned(y, 16)) return EP_ERR_MISALIGNED;
+    StandinParams p;
+    memset(&p, 0, sizeof p);
+    p.ex = static_cast<const uint4 *>(expanded);
+    p.off_e = L->off_e;
+    p.totals = L->totals;
+    p.E = L->E;
+    p.V = H / 8;
+    const int64_t cap = (int64_t)L->T * L->k;
+    p.rows = rows < cap ? rows : cap;
+    p.y = static_cast<uint4 *>(y);
+    return from_cuda(launch_standin(p, as_stream(stream)));
+}
+
+ep_status_t ep_combine_reduce_variant(const void *expert_out, const float *topk_weights,
+                                      int32_t H, const ep_layout_t *L, void *out,
+                                      int64_t y_rows, int32_t variant, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || y_rows < 0) return EP_ERR_INVALID_ARG;
+    if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!expert_out || !topk_weights || !out) return EP_ERR_INVALID_ARG;
+    if (!aligned(expert_out, 16) || !aligned(out, 16)) return EP_ERR_MISALIGNED;
+    if (!aligned(topk_weights, 4)) return EP_ERR_MISALIGNED;
+    CombineParams p;
+    memset(&p, 0, sizeof p);
+    p.y = static_cast<const uint4 *>(expert_out);
+    p.w = topk_weights;
+    p.pos = L->pos;
+    p.T = L->T;
+    p.k = L->k;
+    p.V = H / 8;
+    p.y_rows = y_rows;
+    p.out = static_cast<uint4 *>(out);
+    p.err = L->totals + 3;
+    return from_cuda(launch_combine(p, variant, as_stream(stream)));
+}
+
+ep_status_t ep_combine_reduce(const void *expert_out, const float *topk_weights, int32_t H,
+                              const ep_layout_t *L, void *out, int64_t y_rows, void *stream)
+{
+    return ep_combine_reduce_variant(expert_out, topk_weights, H, L, out, y_rows, 0, stream);
+}
+
+ep_status_t ep_layout_read_totals(const ep_layout_t *L, int64_t *n_route, int64_t *n_recv,
+                                  int64_t *t_real, int32_t *dev_err, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    int32_t h[4] = {0, 0, 0, 0};
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = cudaMemcpyAsync(h, L->totals, sizeof h, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return EP_ERR_CUDA;
+    if (n_route) *n_route = h[0];
+    if (n_recv) *n_recv = h[1];
+    if (t_real) *t_real = h[2];
+    if (dev_err) *dev_err = h[3];
+    if (h[3] & (int32_t)EP_DEVERR_BAD_INDEX) return EP_ERR_BAD_INDEX;
+    if (h[3] & (int32_t)(EP_DEVERR_RECV_CAP | EP_DEVERR_EXP_CAP | EP_DEVERR_Y_ROWS))
+        return EP_ERR_CAPACITY;
+    if (h[3] & (int32_t)EP_DEVERR_TIMEOUT) return EP_ERR_CUDA;
+    return EP_OK;
+}
+
+// ------------------------------------------------------- host round trip
+
+namespace {
+
+struct RoundtripCarve {
+    size_t x, idx, w, lay, recv, exp, y, out, total;
+};
+
+bool roundtrip_carve(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R, int32_t idx_bits,
+                     RoundtripCarve *c)
+{
+    if (!sizes_ok(T, k, E, R) || H <= 0 || H % 8 != 0) return false;
+    if (idx_bits != 32 && idx_bits != 64) return false;
+    const size_t row = (size_t)H * 2;
+    const size_t cap_recv = (size_t)T * (k < R ? k : R);
+    const size_t cap_exp = (size_t)T * k;
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        size_t r = off;
+        off += round_up(n ? n : 1, 256);
+        return r;
+    };
+    c->x = take((size_t)T * row);
+    c->idx = take((size_t)T * k * (idx_bits / 8));
+    c->w = take((size_t)T * k * 4);
+    c->lay = take(ep_layout_bytes(T, k, E, R));
+    c->recv = take(cap_recv * row);
+    c->exp = take(cap_exp * row);
+    c->y = take(cap_exp * row);
+    c->out = take((size_t)T * row);
+    c->total = off;
+    return true;
+}
+
+}  // namespace
+
+size_t ep_roundtrip_device_bytes(int32_t T, int32_t H, int32_t k, int32_t E, int32_t R,
+                                 int32_t idx_bits)
+{
+    RoundtripCarve c;
+    return roundtrip_carve(T, H, k, E, R, idx_bits, &c) ? c.total : 0;
+}
+
+ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
+                              const float *topk_weights_host, int32_t T, int32_t H, int32_t k,
+                              int32_t E, int32_t R, int32_t idx_bits, void *dev_mem, size_t bytes,
+                              void *out_host, void *stream)
+{
+    RoundtripCarve c;
+    if (!roundtrip_carve(T, H, k, E, R, idx_bits, &c)) return EP_ERR_INVALID_ARG;
+    if (!dev_mem || bytes < c.total) return EP_ERR_INVALID_ARG;
+    if (!aligned(dev_mem, 256)) return EP_ERR_MISALIGNED;
+    if (T > 0 && (!x_host || !topk_idx_host || !topk_weights_host || !out_host))
+        return EP_ERR_INVALID_ARG;
+    char *d = static_cast<char *>(dev_mem);
+    cudaStream_t s = as_stream(stream);
+    const size_t row = (size_t)H * 2;
+    const int64_t cap_recv = (int64_t)T * (k < R ? k : R);
+    const int64_t cap_exp = (int64_t)T * k;
+    ep_layout_t L;
+    ep_status_t st = ep_layout_init(&L, T, k, E, R, idx_bits, d + c.lay, ep_layout_bytes(T, k, E, R));
+    if (st != EP_OK) return st;
+    if (T > 0) {
+        cudaError_t e;
+        e = cudaMemcpyAsync(d + c.x, x_host, (size_t)T * row, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return EP_ERR_CUDA;
+        e = cudaMemcpyAsync(d + c.idx, topk_idx_host, (size_t)T * k * (idx_bits / 8),
+                            cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return EP_ERR_CUDA;
+        e = cudaMemcpyAsync(d + c.w, topk_weights_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return EP_ERR_CUDA;
+    }
+    st = ep_layout(d + c.idx, &L, stream);
+    if (st != EP_OK) return st;
+    if (T == 0) return EP_OK;
+    st = ep_dispatch_expand(d + c.x, H, &L, d + c.recv, cap_recv, d + c.exp, cap_exp, stream);
+    if (st != EP_OK) return st;
+    st = ep_standin_expert(d + c.exp, H, &L, d + c.y, cap_exp, stream);
+    if (st != EP_OK) return st;
+    st = ep_combine_reduce(d + c.y, reinterpret_cast<const float *>(d + c.w), H, &L, d + c.out,
+                           cap_exp, stream);
+    if (st != EP_OK) return st;
+    cudaError_t e = cudaMemcpyAsync(out_host, d + c.out, (size_t)T * row, cudaMemcpyDeviceToHost, s);
+    return from_cuda(e);
+}
+
+}  // extern "C"

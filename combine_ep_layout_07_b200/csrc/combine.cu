@@ -1,0 +1,166 @@
+// Combine reduce: out[t] = bf16_rn( sum over valid j, in k order, of
+// w[t, j] * expert_out[pos[t, j]] ), accumulated in fp32; +0 rows for tokens
+// with no valid route.
+//
+// The pages: the per-expert outputs of a token are reduced back into one row
+// (DeepEP issue #48, answer on the reduction before the combine all2all),
+// and the combine epilogue that gives each output token one warp starves the
+// GPU when only a handful of tokens exist per rank (DeepEP issue #760, the
+// report and its first proposed fix: several warps per output token).
+//
+// Schedules (same arithmetic, same result):
+//  * split: CTA (chunk c, token t) owns vectors [c*vpc, (c+1)*vpc) of row t;
+//    each thread keeps all valid routes' 16-byte loads of one vector in
+//    flight, then accumulates them in k order.  At low T the host picks many
+//    small chunks so the hidden dimension is spread over many SMs.
+//  * warp-per-token: one warp walks a whole output row (the DeepEP V2
+//    epilogue's schedule), kept as a measured baseline.
+#include <cuda_bf16.h>
+
+#include "epx_internal.cuh"
+
+namespace epx {
+namespace {
+
+__device__ __forceinline__ void fma8(float (&acc)[8], const uint4 &q, float w)
+{
+    const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float lo = __uint_as_float(u[i] << 16);
+        const float hi = __uint_as_float(u[i] & 0xffff0000u);
+        acc[2 * i] = fmaf(w, lo, acc[2 * i]);
+        acc[2 * i + 1] = fmaf(w, hi, acc[2 * i + 1]);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&acc)[8])
+{
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        u[i] = *reinterpret_cast<uint32_t *>(&b);
+    }
+    return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
+// Warp-collective: compact token t's valid routes (k order) into
+// s_pos/s_w; returns the count on every lane.
+__device__ __forceinline__ int build_routes(const CombineParams &p, int t, int *s_pos,
+                                            float *s_w)
+{
+    const int lane = threadIdx.x & 31;
+    int q = -1;
+    float w = 0.f;
+    if (lane < p.k) {
+        q = p.pos[(size_t)t * p.k + lane];
+        w = p.w[(size_t)t * p.k + lane];
+    }
+    const bool over = q >= 0 && (int64_t)q >= p.y_rows;
+    const bool ok = q >= 0 && !over;
+    if (over) atomicOr(p.err, (int)EP_DEVERR_Y_ROWS);
+    const unsigned m = __ballot_sync(kFull, ok);
+    if (ok) {
+        const int slot = __popc(m & lanemask_lt());
+        s_pos[slot] = q;
+        s_w[slot] = w;
+    }
+    __syncwarp();
+    return __popc(m);
+}
+
+// Accumulate vector v of the n routes; G loads are kept in flight at once.
+template <int G>
+__device__ __forceinline__ uint4 reduce_vector(const CombineParams &p, const int *s_pos,
+                                               const float *s_w, int n, int v)
+{
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i0 = 0; i0 < n; i0 += G) {
+        uint4 q[G];
+#pragma unroll
+        for (int u = 0; u < G; ++u)
+            if (i0 + u < n) q[u] = ld_v4(p.y + (size_t)s_pos[i0 + u] * p.V + v);
+#pragma unroll
+        for (int u = 0; u < G; ++u)
+            if (i0 + u < n) fma8(acc, q[u], s_w[i0 + u]);
+    }
+    return pack8(acc);
+}
+
+template <int G>
+__global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
+{
+    __shared__ int s_pos[EPX_MAX_TOPK];
+    __shared__ float s_w[EPX_MAX_TOPK];
+    __shared__ int s_n;
+    for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
+        if (threadIdx.x < 32) {
+            int n = build_routes(p, t, s_pos, s_w);
+            if (threadIdx.x == 0) s_n = n;
+        }
+        __syncthreads();
+        const int n = s_n;
+        const int v0 = blockIdx.x * p.vpc;
+        const int v1 = min(p.V, v0 + p.vpc);
+        for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x)
+            st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos, s_w, n, v));
+        __syncthreads();
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(128) combine_warp_per_token_kernel(CombineParams p)
+{
+    __shared__ int s_pos[4][EPX_MAX_TOPK];
+    __shared__ float s_w[4][EPX_MAX_TOPK];
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int t = blockIdx.x * 4 + wid; t < p.T; t += gridDim.x * 4) {
+        const int n = build_routes(p, t, s_pos[wid], s_w[wid]);
+        for (int v = lane; v < p.V; v += 32)
+            st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos[wid], s_w[wid], n, v));
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
+{
+    CombineParams p = p0;
+    if (p.T == 0) return cudaSuccess;
+    int nsm = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const bool big_k = p.k > 8;
+    if (variant == 1) {
+        int blocks = (p.T + 3) / 4;
+        if (blocks > 65535 * 16) blocks = 65535 * 16;
+        if (big_k)
+            combine_warp_per_token_kernel<16><<<blocks, 128, 0, s>>>(p);
+        else
+            combine_warp_per_token_kernel<8><<<blocks, 128, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    // split: enough CTAs for ~4 per SM, at least 32 vectors per CTA
+    int chunks = (4 * nsm + p.T - 1) / p.T;
+    const int max_chunks = (p.V + 31) / 32;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    p.vpc = (p.V + chunks - 1) / chunks;
+    chunks = (p.V + p.vpc - 1) / p.vpc;
+    int threads = p.vpc < 128 ? ((p.vpc + 31) / 32) * 32 : 128;
+    const int gy = p.T < 65535 ? p.T : 65535;
+    if (big_k)
+        combine_split_kernel<16><<<dim3(chunks, gy), threads, 0, s>>>(p);
+    else
+        combine_split_kernel<8><<<dim3(chunks, gy), threads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace epx

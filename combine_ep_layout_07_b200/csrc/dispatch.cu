@@ -1,0 +1,251 @@
+// Dispatch + expand: every token with at least one valid route is read from
+// x once and written to one `recv` row per destination rank and one
+// `expanded` row per valid route.
+//
+// The pages' structure: a token is received once per destination rank
+// together with its top-k indices, and a grouped-GEMM consumer then needs it
+// duplicated once per local expert (DeepEP issue #48, question and the
+// answers on DeepGEMM and on the VRAM / performance tradeoff).  On one GPU
+// both copies are made straight from the single read of x[t].
+//
+// Two copy engines, same result:
+//  * vector: 16-byte loads into registers, then 16-byte stores to every
+//    destination row (coalesced: a warp moves 512 contiguous bytes per row);
+//  * bulk: the row (or a chunk of it) is staged in shared memory by one TMA
+//    bulk load (cp.async.bulk, completion on an mbarrier) and written out by
+//    one TMA bulk store per destination row, issued by the warp's lanes in
+//    parallel.  No multicast: every copy is a plain global<->shared::cta
+//    bulk copy on this GPU.
+#include "epx_internal.cuh"
+
+namespace epx {
+namespace {
+
+constexpr int kMaxDst = EPX_MAX_TOPK + EPX_MAX_RANKS;
+
+// Warp-collective: compact the destination rows of token t into dst[0..n).
+// Expanded rows first (k order), then recv rows (rank order).  Rows beyond a
+// capacity are dropped and flagged.  Returns n on every lane.
+__device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
+                                              uint4 **dst)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = lanemask_lt();
+    unsigned flag = 0;
+    int n = 0;
+    {
+        int q = lane < p.k ? p.pos[(size_t)t * p.k + lane] : -1;
+        bool over = q >= 0 && (int64_t)q >= p.exp_cap;
+        bool ok = q >= 0 && !over;
+        flag |= over ? EP_DEVERR_EXP_CAP : 0u;
+        unsigned m = __ballot_sync(kFull, ok);
+        if (ok) dst[__popc(m & lt)] = p.expanded + (size_t)q * p.V;
+        n = __popc(m);
+    }
+    for (int r0 = 0; r0 < p.R; r0 += 32) {
+        const int r = r0 + lane;
+        int q = r < p.R ? p.recv_pos[(size_t)t * p.R + r] : -1;
+        bool over = q >= 0 && (int64_t)q >= p.recv_cap;
+        bool ok = q >= 0 && !over;
+        flag |= over ? EP_DEVERR_RECV_CAP : 0u;
+        unsigned m = __ballot_sync(kFull, ok);
+        if (ok) dst[n + __popc(m & lt)] = p.recv + (size_t)q * p.V;
+        n += __popc(m);
+    }
+    if (flag) atomicOr(p.err, (int)flag);
+    __syncwarp();
+    return n;
+}
+
+// ---------------------------------------------------------------- vector
+
+template <int VPT, bool STREAM>
+__global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
+{
+    __shared__ uint4 *s_dst[kMaxDst];
+    __shared__ int s_n;
+    for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
+        if (threadIdx.x < 32) {
+            int n = build_dst_list(p, t, s_dst);
+            if (threadIdx.x == 0) s_n = n;
+        }
+        __syncthreads();
+        const int n = s_n;
+        if (n > 0) {
+            const int v0 = blockIdx.x * p.vpc;
+            const int v1 = min(p.V, v0 + p.vpc);
+            const uint4 *src = p.x + (size_t)t * p.V;
+            for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x * VPT) {
+                uint4 val[VPT];
+#pragma unroll
+                for (int u = 0; u < VPT; ++u) {
+                    const int vv = v + u * blockDim.x;
+                    if (vv < v1) val[u] = ld_nc_v4(src + vv);
+                }
+                for (int i = 0; i < n; ++i) {
+                    uint4 *d = s_dst[i];
+#pragma unroll
+                    for (int u = 0; u < VPT; ++u) {
+                        const int vv = v + u * blockDim.x;
+                        if (vv < v1) {
+                            if (STREAM)
+                                st_cs_v4(d + vv, val[u]);
+                            else
+                                st_v4(d + vv, val[u]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ bulk
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// bounded wait for phase `parity` of the barrier; false if the limit ran out
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, long long limit)
+{
+    const uint32_t a = smem_addr(bar);
+    for (long long i = 0; i < limit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred P;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, P;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void bulk_g2s(void *sdst, const void *gsrc, unsigned bytes,
+                                         uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(sdst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_s2g(void *gdst, const void *ssrc, unsigned bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(smem_addr(ssrc)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_and_wait_read()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// try_wait polls; each poll may suspend for a hardware-defined time, so this
+// bound is far above any real completion time while still ending.
+constexpr long long kWaitLimit = 1ll << 22;
+
+// One warp per CTA; the CTA handles chunk blockIdx.x (vpc vectors) of token t.
+__global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
+{
+    extern __shared__ __align__(128) uint4 sbuf[];
+    __shared__ uint4 *s_dst[kMaxDst];
+    __shared__ __align__(8) uint64_t bar;
+    const int lane = threadIdx.x;
+    if (lane == 0) mbar_init(&bar, 1);
+    __syncwarp();
+    unsigned phase = 0;
+    const int v0 = blockIdx.x * p.vpc;
+    const int nv = min(p.V, v0 + p.vpc) - v0;
+    if (nv <= 0) return;
+    const unsigned bytes = (unsigned)nv * 16u;
+    for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
+        const int n = build_dst_list(p, t, s_dst);
+        if (n == 0) continue;
+        if (lane == 0) {
+            mbar_expect_tx(&bar, bytes);
+            bulk_g2s(sbuf, p.x + (size_t)t * p.V + v0, bytes, &bar);
+        }
+        if (!mbar_wait(&bar, phase, kWaitLimit)) {
+            if (lane == 0) atomicOr(p.err, (int)EP_DEVERR_TIMEOUT);
+            // give the copy in flight a second bounded chance before leaving
+            mbar_wait(&bar, phase, kWaitLimit);
+            return;
+        }
+        phase ^= 1u;
+        for (int i = lane; i < n; i += 32) bulk_s2g(s_dst[i] + v0, sbuf, bytes);
+        bulk_commit_and_wait_read();  // sbuf and s_dst are reused next token
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t s)
+{
+    DispatchParams p = p0;
+    if (p.T == 0) return cudaSuccess;
+    int nsm = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int gy = p.T < 65535 ? p.T : 65535;
+    if (variant == 0) variant = 1;
+    if (variant == 2) {
+        // chunks so that at least ~2 CTAs per SM exist; chunk <= 32 KB
+        int chunks = (2 * nsm + p.T - 1) / p.T;
+        const int max_chunks = (p.V + 63) / 64;  // >= 1 KB per chunk
+        if (chunks > max_chunks) chunks = max_chunks;
+        int vpc = (p.V + chunks - 1) / chunks;
+        if (vpc > 2048) vpc = 2048;
+        chunks = (p.V + vpc - 1) / vpc;
+        p.vpc = vpc;
+        const size_t smem = (size_t)vpc * 16;
+        static int attr_set_mask = 0;
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 32 && !(attr_set_mask & (1 << dev))) {
+            cudaError_t e = cudaFuncSetAttribute(
+                dispatch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            if (e != cudaSuccess) return e;
+            attr_set_mask |= 1 << dev;
+        }
+        dispatch_bulk_kernel<<<dim3(chunks, gy), 32, smem, s>>>(p);
+        return cudaGetLastError();
+    }
+    // vector engine: 128 threads x 2 vectors per pass
+    int chunks = (4 * nsm + p.T - 1) / p.T;
+    const int max_chunks = (p.V + 255) / 256;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    p.vpc = (p.V + chunks - 1) / chunks;
+    chunks = (p.V + p.vpc - 1) / p.vpc;
+    dispatch_vec_kernel<2, false><<<dim3(chunks, gy), 128, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace epx

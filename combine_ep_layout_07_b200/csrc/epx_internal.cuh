@@ -1,0 +1,116 @@
+// Internal declarations shared by the CUDA translation units of libepx.
+// Not part of the public ABI (that is include/epx.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "epx.h"
+
+namespace epx {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ------------------------------------------------------------ parameters
+
+struct LayoutParams {
+    const void *idx;
+    int T, k, E, R, epr;
+    int tpc;  // tokens per CTA of the cluster
+    int tpw;  // tokens per warp (a multiple of 32 / k)
+    int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
+};
+
+struct DispatchParams {
+    const uint4 *x;
+    const int32_t *pos;
+    const int32_t *recv_pos;
+    int T, k, R;
+    int V;    // 16-byte vectors per row (H / 8)
+    int vpc;  // vectors per CTA chunk
+    uint4 *recv;
+    int64_t recv_cap;
+    uint4 *expanded;
+    int64_t exp_cap;
+    int32_t *err;
+};
+
+struct CombineParams {
+    const uint4 *y;
+    const float *w;
+    const int32_t *pos;
+    int T, k;
+    int V;
+    int vpc;
+    int64_t y_rows;
+    uint4 *out;
+    int32_t *err;
+};
+
+struct StandinParams {
+    const uint4 *ex;
+    const int32_t *off_e;
+    const int32_t *totals;
+    int E, V, vpc;
+    int64_t rows;
+    uint4 *y;
+};
+
+// ------------------------------------------------------------- launchers
+// Each returns cudaSuccess or the launch error; arguments are already
+// validated by the C-ABI layer.
+
+cudaError_t launch_layout(const LayoutParams &p, int idx_bits, cudaStream_t s);
+cudaError_t launch_dispatch(const DispatchParams &p, int variant, cudaStream_t s);
+cudaError_t launch_standin(const StandinParams &p, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
+
+// maximum dynamic shared memory per block that the layout kernel may use
+constexpr int kMaxDynSmem = 227 * 1024;
+
+// ----------------------------------------------------- device utilities
+
+__device__ __forceinline__ unsigned lanemask_lt()
+{
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// 16-byte read-only load that does not allocate in L1 (each source vector is
+// read by exactly one thread).
+__device__ __forceinline__ uint4 ld_nc_v4(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte load of data written by an earlier kernel (plain global load).
+__device__ __forceinline__ uint4 ld_v4(const uint4 *p)
+{
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v4(uint4 *p, const uint4 &v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// streaming (evict-first) store for write-once outputs
+__device__ __forceinline__ void st_cs_v4(uint4 *p, const uint4 &v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+}  // namespace epx

@@ -1,0 +1,246 @@
+"""Thin ctypes binding of libepx.so (the C ABI declared in include/epx.h).
+
+Argument marshalling only: torch provides device memory and the current CUDA
+stream, every step of the path runs in the library's CUDA kernels.  There is
+no CPU fallback: if libepx.so is missing or no CUDA device is present, every
+call raises.
+
+Functions mirror the C entry points:
+
+    lay = layout(topk_idx, num_experts, num_ranks)
+    recv, expanded = dispatch_expand(x, lay)
+    y = standin_expert(expanded, lay)                 # test / bench helper
+    out = combine_reduce(y, topk_weights, lay)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
+    "combine_reduce", "read_totals", "roundtrip_host", "roundtrip_device_bytes",
+    "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libepx.so")
+MAX_TOPK, MAX_RANKS, MAX_EXPERTS = 32, 64, 4096
+
+EP_OK = 0
+_STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_MISALIGNED", 3: "EP_ERR_CAPACITY",
+           4: "EP_ERR_BAD_INDEX", 5: "EP_ERR_CUDA", 6: "EP_ERR_UNSUPPORTED"}
+
+
+class EpxError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        msg = lib().ep_status_str(int(status)).decode() if _lib is not None else _STATUS.get(status)
+        super().__init__(f"{what}: {msg}")
+
+
+class _LayoutC(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("k", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("R", ctypes.c_int32), ("idx_bits", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("cnt_e", ctypes.c_void_p), ("off_e", ctypes.c_void_p),
+                ("cnt_r", ctypes.c_void_p), ("off_r", ctypes.c_void_p),
+                ("pos", ctypes.c_void_p), ("recv_pos", ctypes.c_void_p),
+                ("totals", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libepx.so once; raise if it is missing (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libepx.so not built ({LIB_PATH}); run `python -m combine_ep_layout_07_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    LP = ctypes.POINTER(_LayoutC)
+    sig = {
+        "ep_abi_version": ([], I32),
+        "ep_status_str": ([I32], ctypes.c_char_p),
+        "ep_layout_bytes": ([I32, I32, I32, I32], SZ),
+        "ep_layout_init": ([LP, I32, I32, I32, I32, I32, P, SZ], I32),
+        "ep_layout": ([P, LP, P], I32),
+        "ep_dispatch_expand": ([P, I32, LP, P, I64, P, I64, P], I32),
+        "ep_dispatch_expand_variant": ([P, I32, LP, P, I64, P, I64, I32, P], I32),
+        "ep_standin_expert": ([P, I32, LP, P, I64, P], I32),
+        "ep_combine_reduce": ([P, P, I32, LP, P, I64, P], I32),
+        "ep_combine_reduce_variant": ([P, P, I32, LP, P, I64, I32, P], I32),
+        "ep_layout_read_totals": ([LP, ctypes.POINTER(I64), ctypes.POINTER(I64),
+                                   ctypes.POINTER(I64), ctypes.POINTER(I32), P], I32),
+        "ep_roundtrip_device_bytes": ([I32, I32, I32, I32, I32, I32], SZ),
+        "ep_roundtrip_host": ([P, P, P, I32, I32, I32, I32, I32, I32, P, SZ, P, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != EP_OK:
+        raise EpxError(status, what)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}")
+    return t.data_ptr() if t.numel() else None
+
+
+class Layout:
+    """Routing layout ("handle"): owns one device block holding every array."""
+
+    def __init__(self, T: int, k: int, E: int, R: int, idx_bits: int = 64, device=None):
+        device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+        nbytes = lib().ep_layout_bytes(T, k, E, R)
+        if nbytes == 0:
+            raise EpxError(6 if (k > MAX_TOPK or R > MAX_RANKS or E > MAX_EXPERTS) else 1,
+                           f"ep_layout_bytes(T={T}, k={k}, E={E}, R={R})")
+        self.mem = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.c = _LayoutC()
+        _check(lib().ep_layout_init(ctypes.byref(self.c), T, k, E, R, idx_bits,
+                                    self.mem.data_ptr(), nbytes), "ep_layout_init")
+        self.T, self.k, self.E, self.R, self.idx_bits = T, k, E, R, idx_bits
+        base = self.mem.data_ptr()
+
+        def view(ptr, n):
+            off = ptr - base
+            return self.mem[off:off + 4 * n].view(torch.int32)
+
+        self.cnt_e = view(self.c.cnt_e, E)
+        self.off_e = view(self.c.off_e, E + 1)
+        self.cnt_r = view(self.c.cnt_r, R)
+        self.off_r = view(self.c.off_r, R + 1)
+        self.pos = view(self.c.pos, T * k).view(T, k)
+        self.recv_pos = view(self.c.recv_pos, T * R).view(T, R)
+        self.totals = view(self.c.totals, 4)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+    @property
+    def recv_cap(self) -> int:
+        return self.T * min(self.k, self.R)
+
+    @property
+    def exp_cap(self) -> int:
+        return self.T * self.k
+
+
+def layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, out: Layout = None,
+           stream=None) -> Layout:
+    """ep_layout: routing layout of topk_idx (int32 or int64 [T, k], -1 = none)."""
+    if topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be [T, k]")
+    T, k = topk_idx.shape
+    bits = {torch.int64: 64, torch.int32: 32}.get(topk_idx.dtype)
+    if bits is None:
+        raise TypeError("topk_idx must be int32 or int64")
+    ptr = _dev(topk_idx, "topk_idx")
+    lay = out if out is not None else Layout(T, k, num_experts, num_ranks, bits,
+                                             device=topk_idx.device)
+    if (lay.T, lay.k, lay.E, lay.R, lay.idx_bits) != (T, k, num_experts, num_ranks, bits):
+        raise ValueError("layout buffer does not match the sizes")
+    _check(lib().ep_layout(ptr, lay.ref, _stream(stream)), "ep_layout")
+    return lay
+
+
+def dispatch_expand(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None,
+                    expanded: torch.Tensor = None, variant: int = 0, stream=None):
+    """ep_dispatch_expand: returns (recv [T*min(k,R), H], expanded [T*k, H]) bf16;
+    rows past N_recv / N_route are left as allocated."""
+    if x.dim() != 2 or x.shape[0] != lay.T:
+        raise ValueError("x must be [T, H]")
+    H = x.shape[1]
+    xp = _dev(x, "x", torch.bfloat16)
+    if recv is None:
+        recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=x.device)
+    if expanded is None:
+        expanded = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16, device=x.device)
+    for name, t in (("recv", recv), ("expanded", expanded)):
+        if t.dim() != 2 or t.shape[1] != H:
+            raise ValueError(f"{name} must be [rows, {H}]")
+    _check(lib().ep_dispatch_expand_variant(
+        xp, H, lay.ref, _dev(recv, "recv", torch.bfloat16), recv.shape[0],
+        _dev(expanded, "expanded", torch.bfloat16), expanded.shape[0], variant,
+        _stream(stream)), "ep_dispatch_expand")
+    return recv, expanded
+
+
+def standin_expert(expanded: torch.Tensor, lay: Layout, y: torch.Tensor = None, stream=None):
+    """ep_standin_expert: y[p] = bf16(float(expanded[p]) * (1 + e/E)) for p < N_route."""
+    H = expanded.shape[1]
+    if y is None:
+        y = torch.empty_like(expanded)
+    _check(lib().ep_standin_expert(_dev(expanded, "expanded", torch.bfloat16), H, lay.ref,
+                                   _dev(y, "y", torch.bfloat16),
+                                   min(expanded.shape[0], y.shape[0]), _stream(stream)),
+           "ep_standin_expert")
+    return y
+
+
+def combine_reduce(expert_out: torch.Tensor, topk_weights: torch.Tensor, lay: Layout,
+                   out: torch.Tensor = None, variant: int = 0, stream=None):
+    """ep_combine_reduce: out[t] = bf16(sum_j w[t,j] * expert_out[pos[t,j]])."""
+    H = expert_out.shape[1]
+    if topk_weights.shape != (lay.T, lay.k):
+        raise ValueError("topk_weights must be [T, k]")
+    if out is None:
+        out = torch.empty((lay.T, H), dtype=torch.bfloat16, device=expert_out.device)
+    _check(lib().ep_combine_reduce_variant(
+        _dev(expert_out, "expert_out", torch.bfloat16), _dev(topk_weights, "topk_weights",
+                                                              torch.float32),
+        H, lay.ref, _dev(out, "out", torch.bfloat16), expert_out.shape[0], variant,
+        _stream(stream)), "ep_combine_reduce")
+    return out
+
+
+def read_totals(lay: Layout, stream=None, raise_on_error: bool = True) -> dict:
+    """ep_layout_read_totals (synchronises the stream)."""
+    a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    e = ctypes.c_int32()
+    st = lib().ep_layout_read_totals(lay.ref, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c),
+                                     ctypes.byref(e), _stream(stream))
+    if raise_on_error:
+        _check(st, "ep_layout_read_totals")
+    return dict(N_route=a.value, N_recv=b.value, T_real=c.value, dev_err=e.value, status=st)
+
+
+def roundtrip_device_bytes(T, H, k, E, R, idx_bits=64) -> int:
+    return int(lib().ep_roundtrip_device_bytes(T, H, k, E, R, idx_bits))
+
+
+def roundtrip_host(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.Tensor,
+                   E: int, R: int, dev_mem: torch.Tensor, out_host: torch.Tensor, stream=None):
+    """ep_roundtrip_host: host buffers in, host buffer out (asynchronous)."""
+    T, H = x_host.shape
+    k = idx_host.shape[1]
+    bits = {torch.int64: 64, torch.int32: 32}[idx_host.dtype]
+    for t in (x_host, idx_host, w_host, out_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host buffers must be contiguous CPU tensors")
+    _check(lib().ep_roundtrip_host(x_host.data_ptr(), idx_host.data_ptr(), w_host.data_ptr(),
+                                   T, H, k, E, R, bits, dev_mem.data_ptr(), dev_mem.numel(),
+                                   out_host.data_ptr(), _stream(stream)), "ep_roundtrip_host")
+    return out_host

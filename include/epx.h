@@ -1,0 +1,215 @@
+/*
+ * epx -- MoE token dispatch and combine on one B200 (sm_100a).
+ *
+ * C ABI of libepx.so.  Every pointer documented as "device" is caller-owned
+ * device memory; the library never allocates or frees memory.  Every call is
+ * asynchronous on the given CUDA stream (`stream` is a cudaStream_t passed as
+ * void*, NULL = the legacy default stream) except ep_layout_read_totals,
+ * which synchronises that stream.
+ *
+ * Pipeline, as the pages state the problem (DeepEP issue #48 "How to apply
+ * Moe MLP to recv_x returned by dispatch when num_expert_per_rank > 1";
+ * DeepEP issue #760 "[Performance] DeepEP V2 combine epilogue low batch
+ * performance", section "Reproduction"):
+ *
+ *   ep_layout          topk_idx            -> routing layout ("handle")
+ *   ep_dispatch_expand x, layout           -> recv (one row per token and
+ *                                             destination rank), expanded
+ *                                             (one row per valid route,
+ *                                             expert-contiguous)
+ *   (expert FFN on expanded rows; ep_standin_expert is a deterministic
+ *    stand-in for tests and benchmarks)
+ *   ep_combine_reduce  expert_out, topk_weights, layout -> out
+ *
+ * Logical ranks: experts live on ranks in contiguous blocks of E/R
+ * (expert e on rank e / (E/R)), as in the issue #760 reproduction's
+ * local_experts.  All ranks are partitions of buffers on this one GPU.
+ *
+ * Ordering: inside an expert's segment of `expanded` and inside a rank's
+ * segment of `recv`, rows are ordered by token, then by top-k slot.  The
+ * result is deterministic and identical from run to run.
+ *
+ * Errors: arguments are validated on the host before anything is launched
+ * (EP_ERR_INVALID_ARG / EP_ERR_MISALIGNED; nothing is written).  Problems only
+ * the device can see -- an index < -1 or >= E, a destination row beyond a
+ * caller's capacity -- never trap: the offending route or row is skipped, a
+ * bit is set in the layout's device error word (totals[3]) and
+ * ep_layout_read_totals reports it.  A failed launch returns EP_ERR_CUDA.
+ */
+#ifndef EPX_H
+#define EPX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EPX_ABI_VERSION 1
+
+#define EPX_MAX_TOPK 32      /* k <= 32: one warp holds a token's routes      */
+#define EPX_MAX_RANKS 64     /* R <= 64: a token's rank set fits in 64 bits   */
+#define EPX_MAX_EXPERTS 4096 /* E <= 4096: per-warp expert histograms in smem */
+
+typedef enum ep_status {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1, /* bad size / null pointer / E % R != 0 ...       */
+    EP_ERR_MISALIGNED = 2,  /* a row buffer is not 16-byte aligned            */
+    EP_ERR_CAPACITY = 3,    /* device: a destination row exceeded a capacity  */
+    EP_ERR_BAD_INDEX = 4,   /* device: a topk index < -1 or >= E was skipped  */
+    EP_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed           */
+    EP_ERR_UNSUPPORTED = 6  /* size beyond a documented EPX_MAX_* limit       */
+} ep_status_t;
+
+/* bits of the device error word, totals[3] */
+#define EP_DEVERR_BAD_INDEX 0x1u
+#define EP_DEVERR_RECV_CAP 0x2u
+#define EP_DEVERR_EXP_CAP 0x4u
+#define EP_DEVERR_Y_ROWS 0x8u
+#define EP_DEVERR_TIMEOUT 0x10u /* a bounded wait on an async copy gave up */
+
+/*
+ * Routing layout ("handle" in the pages' dispatch/combine API).  Plain data;
+ * every array is device memory inside one caller-owned block carved by
+ * ep_layout_init.  All int32.
+ *   cnt_e[E]      valid routes per expert
+ *   off_e[E+1]    exclusive scan of cnt_e (expert e's rows in `expanded`
+ *                 are [off_e[e], off_e[e+1]))
+ *   cnt_r[R]      tokens received by rank r (a token counts once per rank)
+ *   off_r[R+1]    exclusive scan of cnt_r (rank r's rows in `recv`)
+ *   pos[T*k]      row of route (t, j) in `expanded`, -1 for no route
+ *   recv_pos[T*R] row of token t in `recv` for rank r, -1 if not sent
+ *   totals[4]     N_route = off_e[E], N_recv = off_r[R],
+ *                 T_real = rows with >= 1 valid route, device error word
+ */
+typedef struct ep_layout {
+    int32_t T, k, E, R;
+    int32_t idx_bits; /* 32 or 64: width of the topk_idx elements */
+    int32_t reserved;
+    int32_t *cnt_e;
+    int32_t *off_e;
+    int32_t *cnt_r;
+    int32_t *off_r;
+    int32_t *pos;
+    int32_t *recv_pos;
+    int32_t *totals;
+} ep_layout_t;
+
+/* ABI version of the loaded library (EPX_ABI_VERSION at build time). */
+int32_t ep_abi_version(void);
+
+/* Human-readable name of a status code; never NULL. */
+const char *ep_status_str(ep_status_t status);
+
+/* Device bytes ep_layout_init needs for a layout of these sizes; 0 if the
+ * sizes are invalid or unsupported. */
+size_t ep_layout_bytes(int32_t T, int32_t k, int32_t E, int32_t R);
+
+/*
+ * Fill *L by carving `dev_mem` (device, >= ep_layout_bytes(...) bytes,
+ * 16-byte aligned).  Host-only: launches nothing, touches no device memory.
+ * Requires T >= 0, 1 <= k <= EPX_MAX_TOPK, 1 <= R <= EPX_MAX_RANKS,
+ * 1 <= E <= EPX_MAX_EXPERTS, E % R == 0, idx_bits in {32, 64}.
+ */
+ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E,
+                           int32_t R, int32_t idx_bits, void *dev_mem,
+                           size_t bytes);
+
+/*
+ * Routing layout from topk_idx (device, [T, k] row-major, int32 or int64 as
+ * L->idx_bits says; -1 = no route).  Overwrites every array of *L, including
+ * totals[3] (the error word is reset here).  Indices < -1 or >= E are
+ * dropped and flagged EP_DEVERR_BAD_INDEX.  One launch (a thread-block
+ * cluster whose CTAs share histograms through distributed shared memory).
+ */
+ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream);
+
+/*
+ * Dispatch + expand.  x: device bf16 [T, H] row-major (16-byte aligned,
+ * H % 8 == 0).  Each token with >= 1 valid route is read once and written
+ *   recv[recv_pos[t, r]]  = x[t] for every rank r it reaches, and
+ *   expanded[pos[t, j]]   = x[t] for every valid route j.
+ * recv: device bf16 [recv_cap, H]; expanded: device bf16 [exp_cap, H].
+ * Worst-case capacities T*min(k, R) and T*k never overflow; a smaller
+ * capacity is allowed, and rows beyond it are skipped and flagged.
+ * Rows past N_recv / N_route are left untouched.
+ */
+ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L,
+                               void *recv, int64_t recv_cap, void *expanded,
+                               int64_t exp_cap, void *stream);
+
+/* Same, choosing the copy engine: 0 = automatic, 1 = 16-byte vector
+ * loads/stores through registers, 2 = TMA bulk copies staged in shared
+ * memory.  Results are identical. */
+ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H,
+                                       const ep_layout_t *L, void *recv,
+                                       int64_t recv_cap, void *expanded,
+                                       int64_t exp_cap, int32_t variant,
+                                       void *stream);
+
+/*
+ * Deterministic stand-in for the expert FFN (test and benchmark helper):
+ * y[p] = bf16_rn(float(expanded[p]) * (1 + e/E)) in IEEE fp32 for every row
+ * p < N_route of expert e's segment.  expanded, y: device bf16 [rows, H],
+ * rows >= N_route (rows beyond N_route are untouched).
+ */
+ep_status_t ep_standin_expert(const void *expanded, int32_t H,
+                              const ep_layout_t *L, void *y, int64_t rows,
+                              void *stream);
+
+/*
+ * Combine reduce.  expert_out: device bf16 [y_rows, H], row pos[t, j] holds
+ * expert idx[t, j]'s output for token t.  topk_weights: device fp32 [T, k].
+ *   out[t, h] = bf16_rn( sum over valid j in k order of
+ *                        topk_weights[t, j] * expert_out[pos[t, j], h] )
+ * accumulated in fp32; weights are used as given (no renormalisation);
+ * a token with no valid route gives a row of +0.  out: device bf16 [T, H].
+ * Work is split over the hidden dimension across CTAs when T is small, so
+ * that a handful of tokens still spreads over all SMs.
+ */
+ep_status_t ep_combine_reduce(const void *expert_out, const float *topk_weights,
+                              int32_t H, const ep_layout_t *L, void *out,
+                              int64_t y_rows, void *stream);
+
+/* Same, choosing the schedule: 0 = automatic, 1 = one warp per output token
+ * (the DeepEP V2 epilogue's schedule, kept as a baseline), 2 = hidden
+ * dimension split across CTAs.  Results are identical. */
+ep_status_t ep_combine_reduce_variant(const void *expert_out,
+                                      const float *topk_weights, int32_t H,
+                                      const ep_layout_t *L, void *out,
+                                      int64_t y_rows, int32_t variant,
+                                      void *stream);
+
+/*
+ * Copy the layout's totals to the host and synchronise `stream`.  Any
+ * pointer may be NULL.  Returns EP_ERR_BAD_INDEX or EP_ERR_CAPACITY when
+ * the device error word has the matching bit set (the totals are still
+ * written), EP_ERR_CUDA if the copy or an earlier launch failed.
+ */
+ep_status_t ep_layout_read_totals(const ep_layout_t *L, int64_t *n_route,
+                                  int64_t *n_recv, int64_t *t_real,
+                                  int32_t *dev_err, void *stream);
+
+/*
+ * End-to-end pass from host buffers: copies x (bf16 [T, H]), topk_idx
+ * ([T, k], idx_bits wide) and topk_weights (fp32 [T, k]) from host memory
+ * (pinned for asynchronous copies), runs layout, dispatch/expand, the
+ * stand-in expert and combine on the device, and copies out (bf16 [T, H])
+ * back to host memory.  dev_mem: caller-owned device scratch of at least
+ * ep_roundtrip_device_bytes(...) bytes, 256-byte aligned.  Asynchronous:
+ * the caller synchronises `stream` before reading out_host.
+ */
+size_t ep_roundtrip_device_bytes(int32_t T, int32_t H, int32_t k, int32_t E,
+                                 int32_t R, int32_t idx_bits);
+ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
+                              const float *topk_weights_host, int32_t T,
+                              int32_t H, int32_t k, int32_t E, int32_t R,
+                              int32_t idx_bits, void *dev_mem, size_t bytes,
+                              void *out_host, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EPX_H */

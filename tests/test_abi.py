@@ -1,0 +1,106 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports
+every function include/epx.h declares, and validates arguments on the host
+(no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from combine_ep_layout_07_b200 import build as epx_build
+from combine_ep_layout_07_b200 import epx
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "epx.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    epx_build.build()
+    return epx.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(ep_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for must in ("ep_layout", "ep_dispatch_expand", "ep_combine_reduce", "ep_layout_init",
+                 "ep_layout_bytes", "ep_layout_read_totals", "ep_standin_expert",
+                 "ep_status_str", "ep_roundtrip_host"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.ep_abi_version() == 1
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.ep_status_str(code).decode()
+        assert s.startswith("EP_")
+    assert lib.ep_status_str(99).decode() == "EP_ERR_UNKNOWN"
+
+
+def test_layout_bytes_and_init_validate_on_host(lib):
+    assert lib.ep_layout_bytes(128, 8, 256, 16) > 0
+    assert lib.ep_layout_bytes(128, 8, 250, 16) == 0      # E % R != 0
+    assert lib.ep_layout_bytes(128, 33, 256, 16) == 0     # k > 32
+    assert lib.ep_layout_bytes(128, 8, 256, 128) == 0     # R > 64
+    assert lib.ep_layout_bytes(128, 8, 8192, 16) == 0     # E > 4096
+    assert lib.ep_layout_bytes(-1, 8, 256, 16) == 0
+    c = epx._LayoutC()
+    fake = 0x10000  # never dereferenced: init only carves pointers
+    n = lib.ep_layout_bytes(128, 8, 256, 16)
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 8, 256, 16, 64, fake, n) == 0
+    assert c.T == 128 and c.k == 8 and c.E == 256 and c.R == 16 and c.idx_bits == 64
+    ptrs = [c.cnt_e, c.off_e, c.cnt_r, c.off_r, c.pos, c.recv_pos, c.totals]
+    assert all(p % 16 == 0 for p in ptrs)
+    assert ptrs == sorted(ptrs) and ptrs[-1] + 16 <= fake + n
+    assert c.pos - c.off_r >= 4 * 17 and c.recv_pos - c.pos >= 4 * 128 * 8
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 8, 256, 16, 64, fake, n - 1) == 1
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 8, 256, 16, 16, fake, n) == 1
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 8, 250, 16, 64, fake, n) == 1
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 40, 256, 16, 64, fake, 1 << 30) == 6
+    assert lib.ep_layout_init(ctypes.byref(c), 128, 8, 256, 16, 64, fake + 4, n) == 2
+    assert lib.ep_layout_init(None, 128, 8, 256, 16, 64, fake, n) == 1
+
+
+def test_calls_reject_bad_arguments_before_launching(lib):
+    # a NULL layout or an invalid one returns before any CUDA call
+    assert lib.ep_layout(None, None, None) == 1
+    bad = epx._LayoutC()
+    assert lib.ep_layout(None, ctypes.byref(bad), None) == 1
+    assert lib.ep_dispatch_expand(None, 64, ctypes.byref(bad), None, 0, None, 0, None) == 1
+    assert lib.ep_combine_reduce(None, None, 64, ctypes.byref(bad), None, 0, None) == 1
+    c = epx._LayoutC()
+    fake = 0x10000
+    n = lib.ep_layout_bytes(4, 2, 4, 2)
+    assert lib.ep_layout_init(ctypes.byref(c), 4, 2, 4, 2, 64, fake, n) == 0
+    # H % 8 != 0, negative capacity, unknown variant
+    assert lib.ep_dispatch_expand(fake, 12, ctypes.byref(c), fake, 8, fake, 8, None) == 1
+    assert lib.ep_dispatch_expand(fake, 16, ctypes.byref(c), fake, -1, fake, 8, None) == 1
+    assert lib.ep_dispatch_expand_variant(fake, 16, ctypes.byref(c), fake, 8, fake, 8, 7,
+                                          None) == 1
+    # 16-byte alignment of row buffers
+    assert lib.ep_dispatch_expand(fake + 2, 16, ctypes.byref(c), fake, 8, fake, 8, None) == 2
+    assert lib.ep_combine_reduce(fake + 8, fake, 16, ctypes.byref(c), fake, 8, None) == 2
+    assert lib.ep_combine_reduce(fake, fake + 2, 16, ctypes.byref(c), fake, 8, None) == 2
+    assert lib.ep_standin_expert(fake, 16, ctypes.byref(c), fake + 4, 8, None) == 2
+    # misaligned 64-bit indices
+    assert lib.ep_layout(fake + 4, ctypes.byref(c), None) == 2
+
+
+def test_roundtrip_sizes(lib):
+    n = lib.ep_roundtrip_device_bytes(128, 7168, 8, 256, 16, 64)
+    row = 7168 * 2
+    assert n >= 128 * row * (1 + 8 + 8 + 1) + 128 * 8 * row
+    assert lib.ep_roundtrip_device_bytes(128, 7167, 8, 256, 16, 64) == 0
+    assert lib.ep_roundtrip_host(None, None, None, 128, 7168, 8, 256, 16, 64, None, 0, None,
+                                 None) == 1
