@@ -82,6 +82,10 @@ def parse_args(argv=None):
                     help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--flush", choices=["auto", "always", "never"], default="auto")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the three calls from Python each step instead of replaying "
+                         "one captured CUDA graph per step")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args(argv)
 
 
@@ -304,7 +308,8 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * el / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate / bf16 data",
-        "data": "synthetic", "config": workload_config(wl, args, slay),
+        "data": "synthetic", "config": dict(workload_config(wl, args, slay),
+                                            launch="host CPU, single thread"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -322,6 +327,7 @@ def workload_config(wl, args, lay_totals, flush_desc=None):
            "parallelism": f"replicas x{dist_env()[1]}"}
     if flush_desc:
         cfg["l2"] = flush_desc
+    cfg["launch"] = "eager" if getattr(args, "eager", True) else "cuda graph per step"
     return cfg
 
 
@@ -358,19 +364,20 @@ def run_epx(args):
     y = torch.empty_like(expanded)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
 
-    def step_kernels(events=None):
+    def step_kernels(events=None, st=None):
+        st = stream if st is None else st
         if events is not None:
-            events[0].record(stream)
-        epx.layout(idx, E, R, out=lay, stream=stream)
+            events[0].record(st)
+        epx.layout(idx, E, R, out=lay, stream=st)
         if events is not None:
-            events[1].record(stream)
+            events[1].record(st)
         epx.dispatch_expand(x, lay, recv=recv, expanded=expanded,
-                            variant=args.dispatch_variant, stream=stream)
+                            variant=args.dispatch_variant, stream=st)
         if events is not None:
-            events[2].record(stream)
-        epx.combine_reduce(y, w, lay, out=out, variant=args.combine_variant, stream=stream)
+            events[2].record(st)
+        epx.combine_reduce(y, w, lay, out=out, variant=args.combine_variant, stream=st)
         if events is not None:
-            events[3].record(stream)
+            events[3].record(st)
 
     with torch.cuda.stream(stream):
         epx.layout(idx, E, R, out=lay, stream=stream)
@@ -386,12 +393,40 @@ def run_epx(args):
     flush_desc = ("L2 flushed between steps (256 MiB write, outside the timed events)" if flush
                   else f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)")
 
+    graph = None
+    gev = None
+    if not args.eager:
+        # one step captured as a CUDA graph with timing events inside it, so
+        # the three kernels run back to back with no host launch gaps
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            step_kernels()          # launchers set their function attributes here
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(graph, stream=stream):
+            step_kernels(gev, st=torch.cuda.current_stream())
+        torch.cuda.synchronize(dev)
+
+    def run_step(events_out=None):
+        if flush:
+            flush_buf.add_(1)
+        if graph is not None:
+            graph.replay()
+            if events_out is not None:
+                torch.cuda.current_stream().synchronize()
+                events_out.append([gev[0].elapsed_time(gev[j]) for j in (1, 2, 3)])
+        else:
+            if events_out is not None:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                step_kernels(ev)
+                events_out.append(ev)
+            else:
+                step_kernels()
+
     # warm-up
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            if flush:
-                flush_buf.add_(1)
-            step_kernels()
+            run_step()
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
@@ -399,16 +434,14 @@ def run_epx(args):
     sampler = ClockSampler(gpu_uuid(torch, local)) if rank == 0 else None
     if sampler:
         sampler.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    rec = []
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     t_lo = time.time()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            if flush:
-                flush_buf.add_(1)
-            step_kernels(evs[i])
+            run_step(rec)
     torch.cuda.synchronize(dev)
     t_hi = time.time()
     if pg:
@@ -416,10 +449,12 @@ def run_epx(args):
     if sampler:
         sampler.stop()
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    k_ms = {"layout": [e[0].elapsed_time(e[1]) for e in evs],
-            "dispatch_expand": [e[1].elapsed_time(e[2]) for e in evs],
-            "combine_reduce": [e[2].elapsed_time(e[3]) for e in evs]}
+    if graph is None:   # cumulative times from each step's first event
+        rec = [[e[0].elapsed_time(e[j]) for j in (1, 2, 3)] for e in rec]
+    step_ms = [r[2] for r in rec]
+    k_ms = {"layout": [r[0] for r in rec],
+            "dispatch_expand": [r[1] - r[0] for r in rec],
+            "combine_reduce": [r[2] - r[1] for r in rec]}
     total_ms = sum(step_ms)
     if pg:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
@@ -429,7 +464,10 @@ def run_epx(args):
     value = units / (total_ms / 1e3)
 
     # ---- e2e through the host-buffer C-ABI call
-    e2e = run_e2e(torch, epx, wl, args, dev, stream, pg, world, tot["T_real"])
+    e2e = None if args.no_e2e else run_e2e(torch, epx, wl, args, dev, stream, pg, world,
+                                           tot["T_real"])
+    if graph is not None:
+        del graph
 
     if rank != 0:
         finish(pg)

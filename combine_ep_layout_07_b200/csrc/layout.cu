@@ -10,17 +10,21 @@
 //
 // Design (one launch, one thread-block cluster of up to 8 CTAs):
 //  * tokens are split into contiguous ranges: CTA c of the cluster, then
-//    warp w of the CTA, then steps of floor(32/k) whole tokens, one route per
-//    lane, so lane order inside a step is (token, slot) order;
-//  * pass 1: warp-aggregated counting -- __match_any_sync groups the lanes of
-//    a step by expert (and by (token, rank) to deduplicate ranks) and the
-//    group leader adds the group size to the warp's private histogram row in
-//    shared memory, so no atomics are needed;
+//    warp w of the CTA; each warp walks its range in steps of floor(32/k)
+//    whole tokens, one route per lane, so lane order inside a step is
+//    (token, slot) order;
+//  * staging: the CTA loads its routes with coalesced loads into shared
+//    memory (one DRAM round trip instead of one per step), then one thread
+//    per token validates the indices, computes each route's rank e / (E/R)
+//    and marks the first route of every (token, rank) pair;
+//  * pass 1: per-warp histograms of experts and of first routes per rank,
+//    counted with shared-memory atomics (order does not matter for counts);
 //  * scans: per expert, an exclusive scan over the CTA's warps; the CTA
 //    totals are exchanged through distributed shared memory, giving each CTA
-//    its base and every CTA the global exclusive scan over experts;
-//  * pass 2: the same walk again, each lane taking its expert's warp cursor
-//    plus its rank among equal experts in the step (popc of the lower peers).
+//    its base and every CTA the global exclusive scan over experts / ranks;
+//  * pass 2: the ordered walk -- __match_any_sync groups a step's lanes by
+//    expert (and first-routes by rank); each lane takes the warp cursor plus
+//    the number of lower lanes in its group, the group leader advances it.
 // Rows therefore come out ordered by token, then slot, inside every expert
 // segment and every rank segment, independent of scheduling.
 #include <cooperative_groups.h>
@@ -31,6 +35,10 @@ namespace cg = cooperative_groups;
 
 namespace epx {
 namespace {
+
+// staged route code: -2 = no token here, -1 = no route (or a dropped bad
+// index), else expert | rank << 16 | (first route of its rank) << 30
+constexpr int kAbsent = -2;
 
 // Exclusive scan of one int per thread across the CTA.  `sm` has >= 34 ints.
 __device__ int block_exclusive_scan(int v, int *sm, int *total)
@@ -63,44 +71,65 @@ __device__ int block_exclusive_scan(int v, int *sm, int *total)
     return res;
 }
 
-// One step of a warp's walk: lane = route (t0 + lane / k, lane % k).
-struct Step {
-    bool act;     // lane holds a route of a token in range
-    bool valid;   // ... and its expert index is in [0, E)
-    bool bad;     // ... or its index is < -1 or >= E
-    bool first;   // first valid lane of its (token, rank) pair
-    int e, r;     // expert and rank (valid lanes)
-    unsigned pe;  // lanes with the same expert
-    unsigned pr;  // first-lanes with the same rank
-    int nreal;    // tokens of the step with >= 1 valid route (same on all lanes)
+struct Ranges {
+    int c0, c1;  // this CTA's tokens
+    int tpw;     // tokens per warp
+    __device__ int w0(int w) const { return min(c1, c0 + w * tpw); }
+    __device__ int w1(int w) const { return min(c1, c0 + (w + 1) * tpw); }
 };
 
+// Stage chunk c (tokens [w0 + c*S, w0 + c*S + S) of every warp w) into
+// codes[w][s*k + j].  first_pass also fills recv_pos with -1 for the staged
+// tokens and counts bad indices / real tokens into misc[0] / misc[1].
 template <typename IdxT>
-__device__ __forceinline__ Step make_step(const IdxT *__restrict__ idx, int t0,
-                                          int tend, int k, int E, int epr,
-                                          int tps, int lane)
+__device__ void stage_chunk(const LayoutParams &p, const IdxT *__restrict__ idx,
+                            const Ranges &rg, int c, int NW, int32_t *codes,
+                            int32_t *misc, bool first_pass)
 {
-    Step s;
-    const int tl = lane / k;
-    const int j = lane - tl * k;
-    const int t = t0 + tl;
-    s.act = tl < tps && t < tend;
-    long long e = s.act ? (long long)idx[(size_t)t * k + j] : -1;
-    s.bad = s.act && (e < -1 || e >= E);
-    s.valid = s.act && e >= 0 && e < E;
-    s.e = s.valid ? (int)e : -1;
-    s.pe = __match_any_sync(kFull, s.e);
-    s.r = s.valid ? s.e / epr : 0;
-    // (token slot, rank) key: tl < 32 and r < 64
-    const unsigned ptr = __match_any_sync(kFull, s.valid ? (tl << 6) | s.r : -1);
-    s.first = s.valid && lane == __ffs(ptr) - 1;
-    s.pr = __match_any_sync(kFull, s.first ? s.r : -1);
-    // real tokens in this step
-    const unsigned vm = __ballot_sync(kFull, s.valid);
-    const unsigned kmask = k == 32 ? kFull : ((1u << k) - 1u);
-    const bool real = lane < tps && ((vm >> (lane * k)) & kmask) != 0u;
-    s.nreal = __popc(__ballot_sync(kFull, real));
-    return s;
+    const int k = p.k, S = p.S, E = p.E, R = p.R;
+    const int per_w = S * k;
+    const int n = NW * per_w;
+    bool bad = false;
+    // coalesced raw load: consecutive threads take consecutive routes of a
+    // warp's slice (the slice is contiguous in topk_idx)
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int w = i / per_w;
+        const int rem = i - w * per_w;
+        const int t = rg.w0(w) + c * S + rem / k;
+        int code = kAbsent;
+        if (t < rg.w1(w)) {
+            const long long e = (long long)idx[(size_t)rg.w0(w) * k + (size_t)c * per_w + rem];
+            bad |= (e < -1 || e >= E);
+            code = (e >= 0 && e < E) ? (int)e : -1;
+        }
+        codes[i] = code;
+    }
+    __syncthreads();
+    // one thread per token: rank of each route, first route of each rank
+    int nreal = 0;
+    for (int u = threadIdx.x; u < NW * S; u += blockDim.x) {
+        const int w = u / S;
+        const int t = rg.w0(w) + c * S + (u - w * S);
+        if (t >= rg.w1(w)) continue;
+        int32_t *cd = codes + (size_t)u * k;
+        unsigned long long mask = 0ull;
+        for (int j = 0; j < k; ++j) {
+            const int e = cd[j];
+            if (e < 0) continue;
+            const int r = e / p.epr;
+            const bool f = !((mask >> r) & 1ull);
+            mask |= 1ull << r;
+            cd[j] = e | (r << 16) | ((int)f << 30);
+        }
+        nreal += mask != 0ull;
+        if (first_pass)
+            for (int r = 0; r < R; ++r) p.recv_pos[(size_t)t * R + r] = -1;
+    }
+    if (first_pass) {
+        if (bad) atomicOr(&misc[0], 1);
+        if (nreal) atomicAdd(&misc[1], nreal);
+    }
+    __syncthreads();
 }
 
 template <typename IdxT>
@@ -109,13 +138,14 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     extern __shared__ __align__(16) int32_t smem[];
     const int NW = blockDim.x >> 5;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int E = p.E, R = p.R, k = p.k, T = p.T;
+    const int E = p.E, R = p.R, k = p.k, T = p.T, S = p.S;
     int32_t *hist_e = smem;              // [NW][E] per-warp counts, then cursors
     int32_t *hist_r = hist_e + NW * E;   // [NW][R]
     int32_t *tot_e = hist_r + NW * R;    // [E]  CTA totals (read by peer CTAs)
     int32_t *tot_r = tot_e + E;          // [R]
     int32_t *misc = tot_r + R;           // [4]  0: bad-index flag, 1: real tokens
-    int32_t *scan = misc + 4;            // [34]
+    int32_t *scan = misc + 4;            // [36]
+    int32_t *codes = scan + 36;          // [NW][S*k] staged routes
 
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
@@ -127,30 +157,24 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
     const int tps = 32 / k;
-    const int c0 = min(T, crank * p.tpc), c1 = min(T, c0 + p.tpc);
-    const int w0 = min(c1, c0 + wid * p.tpw), w1 = min(c1, w0 + p.tpw);
+    Ranges rg;
+    rg.c0 = min(T, crank * p.tpc);
+    rg.c1 = min(T, rg.c0 + p.tpc);
+    rg.tpw = p.tpw;
+    const int nchunks = (p.tpw + S - 1) / S;
+    int32_t *my_codes = codes + (size_t)wid * S * k;
 
-    // tokens not sent to a rank keep -1 (pass 2 overwrites the sent pairs)
-    for (long long i = (long long)w0 * R + lane; i < (long long)w1 * R; i += 32)
-        p.recv_pos[i] = -1;
-
-    // ---- pass 1: warp-private histograms
-    bool bad = false;
-    int nreal = 0;
-    for (int t0 = w0; t0 < w1; t0 += tps) {
-        Step s = make_step(idx, t0, w1, k, E, p.epr, tps, lane);
-        bad |= s.bad;
-        nreal += s.nreal;
-        if (s.valid && lane == __ffs(s.pe) - 1) hist_e[wid * E + s.e] += __popc(s.pe);
-        if (s.first && lane == __ffs(s.pr) - 1) hist_r[wid * R + s.r] += __popc(s.pr);
-        __syncwarp();
+    // ---- pass 1: per-warp histograms
+    for (int c = 0; c < nchunks; ++c) {
+        stage_chunk(p, idx, rg, c, NW, codes, misc, true);
+        for (int i = lane; i < S * k; i += 32) {
+            const int code = my_codes[i];
+            if (code < 0) continue;
+            atomicAdd(&hist_e[wid * E + (code & 0xffff)], 1);
+            if (code & (1 << 30)) atomicAdd(&hist_r[wid * R + ((code >> 16) & 0x3f)], 1);
+        }
+        __syncthreads();
     }
-    bad = __any_sync(kFull, bad);
-    if (lane == 0) {
-        if (bad) atomicOr(&misc[0], 1);
-        atomicAdd(&misc[1], nreal);
-    }
-    __syncthreads();
 
     // ---- exclusive scan over this CTA's warps, per expert / per rank
     for (int e = tid; e < E; e += blockDim.x) {
@@ -234,35 +258,53 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     }
     cluster.sync();  // peers are done reading; cursors visible CTA-wide
 
-    // ---- pass 2: positions
+    // ---- pass 2: positions, in (token, slot) order
     const unsigned lt = lanemask_lt();
-    for (int t0 = w0; t0 < w1; t0 += tps) {
-        Step s = make_step(idx, t0, w1, k, E, p.epr, tps, lane);
-        const int tl = lane / k;
-        const int t = t0 + tl;
-        int base = s.valid ? hist_e[wid * E + s.e] : 0;
-        int base_r = s.first ? hist_r[wid * R + s.r] : 0;
-        __syncwarp();
-        if (s.valid && lane == __ffs(s.pe) - 1) hist_e[wid * E + s.e] = base + __popc(s.pe);
-        if (s.first && lane == __ffs(s.pr) - 1) hist_r[wid * R + s.r] = base_r + __popc(s.pr);
-        if (s.act) p.pos[(size_t)t * k + (lane - tl * k)] = s.valid ? base + __popc(s.pe & lt) : -1;
-        if (s.first) p.recv_pos[(size_t)t * R + s.r] = base_r + __popc(s.pr & lt);
-        __syncwarp();
+    const int tl = lane / k;
+    const int j = lane - tl * k;
+    for (int c = 0; c < nchunks; ++c) {
+        if (nchunks > 1) stage_chunk(p, idx, rg, c, NW, codes, misc, false);
+        const int tb = rg.w0(wid) + c * S;  // first token of this warp's slice
+        for (int s0 = 0; s0 < S; s0 += tps) {
+            const int s = s0 + tl;
+            const bool lane_ok = tl < tps && s < S;
+            const int code = lane_ok ? my_codes[s * k + j] : kAbsent;
+            const bool valid = code >= 0;
+            const int e = valid ? (code & 0xffff) : -1;
+            const bool first = valid && (code & (1 << 30));
+            const int r = (code >> 16) & 0x3f;
+            const unsigned pe = __match_any_sync(kFull, e);
+            const unsigned pr = __match_any_sync(kFull, first ? r : -1);
+            const int base = valid ? hist_e[wid * E + e] : 0;
+            const int base_r = first ? hist_r[wid * R + r] : 0;
+            __syncwarp();
+            if (valid && lane == __ffs(pe) - 1) hist_e[wid * E + e] = base + __popc(pe);
+            if (first && lane == __ffs(pr) - 1) hist_r[wid * R + r] = base_r + __popc(pr);
+            const size_t t = (size_t)(tb + s);
+            if (code != kAbsent) p.pos[t * k + j] = valid ? base + __popc(pe & lt) : -1;
+            if (first) p.recv_pos[t * R + r] = base_r + __popc(pr & lt);
+            __syncwarp();
+        }
+        if (nchunks > 1) __syncthreads();  // codes are restaged next chunk
     }
 }
 
-size_t layout_smem_bytes(int NW, int E, int R)
+size_t layout_smem_bytes(int NW, int E, int R, int S, int k)
 {
-    return sizeof(int32_t) * ((size_t)NW * (E + R) + E + R + 4 + 34);
+    return sizeof(int32_t) * ((size_t)NW * (E + R) + E + R + 4 + 36 + (size_t)NW * S * k);
 }
 
 // cudaOccupancyMaxActiveClusters for (cluster size, threads, smem), cached
 // per device; 0 means such a cluster cannot be scheduled.
 template <typename IdxT>
-int max_cluster_ok(int csize, int threads, size_t smem, int dev)
+int max_clusters(int csize, int threads, size_t smem, int dev)
 {
-    struct Entry { int dev, csize, threads; size_t smem; int result; };
-    static Entry cache[32];
+    struct Entry {
+        int dev, csize, threads;
+        size_t smem;
+        int result;
+    };
+    static Entry cache[64];
     static int n_cache = 0;
     for (int i = 0; i < n_cache; ++i)
         if (cache[i].dev == dev && cache[i].csize == csize && cache[i].threads == threads &&
@@ -284,58 +326,84 @@ int max_cluster_ok(int csize, int threads, size_t smem, int dev)
         cudaGetLastError();
         n = 0;
     }
-    if (n_cache < 32) cache[n_cache++] = Entry{dev, csize, threads, smem, n};
+    if (n_cache < 64) cache[n_cache++] = Entry{dev, csize, threads, smem, n};
     return n;
+}
+
+struct Geometry {
+    int csize, NW, tpc, tpw, S;
+    size_t smem;
+};
+
+// Cluster size, warps per CTA and staging chunk for a layout problem.
+Geometry plan(int T, int k, int E, int R, int csize)
+{
+    Geometry g;
+    const int tps = 32 / k;
+    g.csize = csize;
+    g.tpc = (T + csize - 1) / csize;
+    const int steps = (g.tpc + tps - 1) / tps;
+    const int nw_ranks = (R + 31) / 32;  // the rank scan gives one rank per thread
+    // about 4 steps per warp: enough warps to spread the walk, few enough
+    // that the per-expert scans over warps stay short
+    int NW = (steps + 3) / 4;
+    if (NW > 32) NW = 32;
+    if (NW < nw_ranks) NW = nw_ranks;
+    if (NW < 1) NW = 1;
+    for (;;) {
+        int tpw = (g.tpc + NW - 1) / NW;
+        tpw = ((tpw + tps - 1) / tps) * tps;
+        if (tpw < tps) tpw = tps;
+        const size_t base = layout_smem_bytes(NW, E, R, 0, k);
+        long long avail = (long long)kMaxDynSmem - (long long)base;
+        int S = avail > 0 ? (int)(avail / ((long long)NW * k * 4)) : 0;
+        S = (S / tps) * tps;
+        if (S > tpw) S = tpw;
+        if (S >= tps || NW <= nw_ranks) {
+            g.NW = NW;
+            g.tpw = tpw;
+            g.S = S < tps ? tps : S;
+            g.smem = layout_smem_bytes(NW, E, R, g.S, k);
+            return g;
+        }
+        --NW;
+    }
 }
 
 template <typename IdxT>
 cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
 {
-    static int attr_set_mask = 0;  // per device (up to 32), set once
+    static unsigned attr_set_mask = 0;  // per device (up to 32), set once
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 32 && !(attr_set_mask & (1 << dev))) {
+    if (dev < 32 && !(attr_set_mask & (1u << dev))) {
         err = cudaFuncSetAttribute(layout_kernel<IdxT>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   kMaxDynSmem);
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
         if (err != cudaSuccess) return err;
-        attr_set_mask |= 1 << dev;
+        attr_set_mask |= 1u << dev;
     }
 
     LayoutParams p = p0;
-    const int T = p.T, k = p.k, E = p.E, R = p.R;
-    const int tps = 32 / k;
-    const long long routes = (long long)T * k;
+    const long long routes = (long long)p.T * p.k;
     // one CTA up to ~4K routes, then up to an 8-CTA cluster
     int csize = (int)((routes + 4095) / 4096);
     csize = csize < 1 ? 1 : (csize > 8 ? 8 : csize);
-    int nw_max = 32;
-    while (nw_max > 1 && layout_smem_bytes(nw_max, E, R) > (size_t)kMaxDynSmem) --nw_max;
-    // largest cluster (<= csize) that the device can co-schedule at this size
-    while (csize > 1 && max_cluster_ok<IdxT>(csize, nw_max * 32,
-                                             layout_smem_bytes(nw_max, E, R), dev) == 0)
-        csize >>= 1;
-    const int tpc = (T + csize - 1) / csize;
-    int steps = (tpc + tps - 1) / tps;
-    int NW = steps < 1 ? 1 : (steps > nw_max ? nw_max : steps);
-    // the rank scan gives one rank to each thread
-    const int nw_ranks = (R + 31) / 32;
-    if (NW < nw_ranks) NW = nw_ranks;
-    int tpw = (tpc + NW - 1) / NW;
-    tpw = ((tpw + tps - 1) / tps) * tps;
-    if (tpw < tps) tpw = tps;
-    p.tpc = tpc;
-    p.tpw = tpw;
+    Geometry g = plan(p.T, p.k, p.E, p.R, csize);
+    while (g.csize > 1 && max_clusters<IdxT>(g.csize, g.NW * 32, g.smem, dev) == 0)
+        g = plan(p.T, p.k, p.E, p.R, g.csize >> 1);
+    p.tpc = g.tpc;
+    p.tpw = g.tpw;
+    p.S = g.S;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(csize, 1, 1);
-    cfg.blockDim = dim3(NW * 32, 1, 1);
-    cfg.dynamicSmemBytes = layout_smem_bytes(NW, E, R);
+    cfg.gridDim = dim3(g.csize, 1, 1);
+    cfg.blockDim = dim3(g.NW * 32, 1, 1);
+    cfg.dynamicSmemBytes = g.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.x = g.csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
