@@ -19,6 +19,7 @@ struct LayoutParams {
     int tpc;  // tokens per CTA of the cluster
     int tpw;  // tokens per warp (a multiple of 32 / k)
     int S;    // tokens per warp staged in shared memory at a time (multiple of 32 / k)
+    int nww;  // walker warps: warps that own a token range and a histogram row
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 

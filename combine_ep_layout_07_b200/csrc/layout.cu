@@ -8,25 +8,29 @@
 // Reproduction: padding rows of -1) and experts on ranks in contiguous
 // blocks of E/R (issue #760, Reproduction: local_experts).
 //
-// Design (one launch, one thread-block cluster of up to 8 CTAs):
+// Design (one launch, one thread-block cluster of up to 8 CTAs of 1024
+// threads):
 //  * tokens are split into contiguous ranges: CTA c of the cluster, then
-//    warp w of the CTA; each warp walks its range in steps of floor(32/k)
-//    whole tokens, one route per lane, so lane order inside a step is
-//    (token, slot) order;
+//    walker warp w of the CTA; each walker walks its range in steps of
+//    floor(32/k) whole tokens, one route per lane, so lane order inside a
+//    step is (token, slot) order;
 //  * staging: the CTA loads its routes with coalesced loads into shared
 //    memory (one DRAM round trip instead of one per step), then one thread
 //    per token validates the indices, computes each route's rank e / (E/R)
 //    and marks the first route of every (token, rank) pair;
-//  * pass 1: per-warp histograms of experts and of first routes per rank,
+//  * pass 1: per-walker histograms of experts and of first routes per rank,
 //    counted with shared-memory atomics (order does not matter for counts);
-//  * scans: per expert, an exclusive scan over the CTA's warps; the CTA
-//    totals are exchanged through distributed shared memory, giving each CTA
-//    its base and every CTA the global exclusive scan over experts / ranks;
+//  * scans: per expert, an exclusive scan over the CTA's walkers; each CTA
+//    pushes its totals into every peer's shared memory (distributed shared
+//    memory stores), one cluster barrier, then every CTA reads them locally
+//    to get its base and the global exclusive scan over experts / ranks;
 //  * pass 2: the ordered walk -- __match_any_sync groups a step's lanes by
-//    expert (and first-routes by rank); each lane takes the warp cursor plus
-//    the number of lower lanes in its group, the group leader advances it.
-// Rows therefore come out ordered by token, then slot, inside every expert
-// segment and every rank segment, independent of scheduling.
+//    expert (and first-routes by rank); each lane takes the walker's cursor
+//    plus the number of lower lanes in its group, the group leader advances it.
+// Expert-proportional work (zeroing, scans, writing counts and offsets) uses
+// all 1024 threads, so it stays short even for a single token.
+// Rows come out ordered by token, then slot, inside every expert segment and
+// every rank segment, independent of scheduling.
 #include <cooperative_groups.h>
 
 #include "epx_internal.cuh"
@@ -73,26 +77,25 @@ __device__ int block_exclusive_scan(int v, int *sm, int *total)
 
 struct Ranges {
     int c0, c1;  // this CTA's tokens
-    int tpw;     // tokens per warp
+    int tpw;     // tokens per walker warp
     __device__ int w0(int w) const { return min(c1, c0 + w * tpw); }
     __device__ int w1(int w) const { return min(c1, c0 + (w + 1) * tpw); }
 };
 
-// Stage chunk c (tokens [w0 + c*S, w0 + c*S + S) of every warp w) into
+// Stage chunk c (tokens [w0 + c*S, w0 + c*S + S) of every walker w) into
 // codes[w][s*k + j].  first_pass also fills recv_pos with -1 for the staged
 // tokens and counts bad indices / real tokens into misc[0] / misc[1].
 template <typename IdxT>
 __device__ void stage_chunk(const LayoutParams &p, const IdxT *__restrict__ idx,
-                            const Ranges &rg, int c, int NW, int32_t *codes,
-                            int32_t *misc, bool first_pass)
+                            const Ranges &rg, int c, int32_t *codes, int32_t *misc,
+                            bool first_pass)
 {
-    const int k = p.k, S = p.S, E = p.E, R = p.R;
+    const int k = p.k, S = p.S, E = p.E, R = p.R, NWW = p.nww;
     const int per_w = S * k;
-    const int n = NW * per_w;
     bool bad = false;
     // coalesced raw load: consecutive threads take consecutive routes of a
-    // warp's slice (the slice is contiguous in topk_idx)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    // walker's slice (the slice is contiguous in topk_idx)
+    for (int i = threadIdx.x; i < NWW * per_w; i += blockDim.x) {
         const int w = i / per_w;
         const int rem = i - w * per_w;
         const int t = rg.w0(w) + c * S + rem / k;
@@ -104,10 +107,19 @@ __device__ void stage_chunk(const LayoutParams &p, const IdxT *__restrict__ idx,
         }
         codes[i] = code;
     }
+    if (first_pass) {
+        const int per_wr = S * R;
+        for (int i = threadIdx.x; i < NWW * per_wr; i += blockDim.x) {
+            const int w = i / per_wr;
+            const int rem = i - w * per_wr;
+            if (rg.w0(w) + c * S + rem / R < rg.w1(w))
+                p.recv_pos[(size_t)(rg.w0(w) + c * S) * R + rem] = -1;
+        }
+    }
     __syncthreads();
     // one thread per token: rank of each route, first route of each rank
     int nreal = 0;
-    for (int u = threadIdx.x; u < NW * S; u += blockDim.x) {
+    for (int u = threadIdx.x; u < NWW * S; u += blockDim.x) {
         const int w = u / S;
         const int t = rg.w0(w) + c * S + (u - w * S);
         if (t >= rg.w1(w)) continue;
@@ -122,8 +134,6 @@ __device__ void stage_chunk(const LayoutParams &p, const IdxT *__restrict__ idx,
             cd[j] = e | (r << 16) | ((int)f << 30);
         }
         nreal += mask != 0ull;
-        if (first_pass)
-            for (int r = 0; r < R; ++r) p.recv_pos[(size_t)t * R + r] = -1;
     }
     if (first_pass) {
         if (bad) atomicOr(&misc[0], 1);
@@ -136,22 +146,26 @@ template <typename IdxT>
 __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 {
     extern __shared__ __align__(16) int32_t smem[];
-    const int NW = blockDim.x >> 5;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int E = p.E, R = p.R, k = p.k, T = p.T, S = p.S;
-    int32_t *hist_e = smem;              // [NW][E] per-warp counts, then cursors
-    int32_t *hist_r = hist_e + NW * E;   // [NW][R]
-    int32_t *tot_e = hist_r + NW * R;    // [E]  CTA totals (read by peer CTAs)
-    int32_t *tot_r = tot_e + E;          // [R]
-    int32_t *misc = tot_r + R;           // [4]  0: bad-index flag, 1: real tokens
-    int32_t *scan = misc + 4;            // [36]
-    int32_t *codes = scan + 36;          // [NW][S*k] staged routes
+    const int E = p.E, R = p.R, k = p.k, T = p.T, S = p.S, NWW = p.nww;
 
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
     const int csize = (int)cluster.num_blocks();
 
-    for (int i = tid; i < NW * (E + R); i += blockDim.x) hist_e[i] = 0;
+    const int W = E + R + 2;                 // one CTA's totals: experts, ranks, bad, real
+    int32_t *hist_e = smem;                  // [NWW][E] per-walker counts, then cursors
+    int32_t *hist_r = hist_e + NWW * E;      // [NWW][R]
+    int32_t *all_tot = hist_r + NWW * R;     // [csize][W], row c written by CTA c
+    int32_t *misc = all_tot + csize * W;     // [4]  0: bad-index flag, 1: real tokens
+    int32_t *scan = misc + 4;                // [36]
+    int32_t *codes = scan + 36;              // [NWW][S*k] staged routes
+
+    // every CTA of the cluster must be running before a peer writes into its
+    // shared memory: arrive now, wait just before the first remote store
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+
+    for (int i = tid; i < NWW * (E + R); i += blockDim.x) hist_e[i] = 0;
     if (tid < 4) misc[tid] = 0;
     __syncthreads();
 
@@ -162,58 +176,59 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     rg.c1 = min(T, rg.c0 + p.tpc);
     rg.tpw = p.tpw;
     const int nchunks = (p.tpw + S - 1) / S;
-    int32_t *my_codes = codes + (size_t)wid * S * k;
 
-    // ---- pass 1: per-warp histograms
+    // ---- pass 1: per-walker histograms (shared-memory atomics, any order)
     for (int c = 0; c < nchunks; ++c) {
-        stage_chunk(p, idx, rg, c, NW, codes, misc, true);
-        for (int i = lane; i < S * k; i += 32) {
-            const int code = my_codes[i];
+        stage_chunk(p, idx, rg, c, codes, misc, true);
+        const int per_w = S * k;
+        for (int i = tid; i < NWW * per_w; i += blockDim.x) {
+            const int code = codes[i];
             if (code < 0) continue;
-            atomicAdd(&hist_e[wid * E + (code & 0xffff)], 1);
-            if (code & (1 << 30)) atomicAdd(&hist_r[wid * R + ((code >> 16) & 0x3f)], 1);
+            const int w = i / per_w;
+            atomicAdd(&hist_e[w * E + (code & 0xffff)], 1);
+            if (code & (1 << 30)) atomicAdd(&hist_r[w * R + ((code >> 16) & 0x3f)], 1);
         }
         __syncthreads();
     }
 
-    // ---- exclusive scan over this CTA's warps, per expert / per rank
-    for (int e = tid; e < E; e += blockDim.x) {
+    // ---- exclusive scan over walkers; push this CTA's totals to every CTA
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    for (int e = tid; e < E + R; e += blockDim.x) {
+        int32_t *h = e < E ? hist_e + e : hist_r + (e - E);
+        const int stride = e < E ? E : R;
         int run = 0;
-        for (int w = 0; w < NW; ++w) {
-            int v = hist_e[w * E + e];
-            hist_e[w * E + e] = run;
+        for (int w = 0; w < NWW; ++w) {
+            const int v = h[w * stride];
+            h[w * stride] = run;
             run += v;
         }
-        tot_e[e] = run;
+        for (int c = 0; c < csize; ++c) cluster.map_shared_rank(all_tot, c)[crank * W + e] = run;
     }
-    for (int r = tid; r < R; r += blockDim.x) {
-        int run = 0;
-        for (int w = 0; w < NW; ++w) {
-            int v = hist_r[w * R + r];
-            hist_r[w * R + r] = run;
-            run += v;
+    if (tid == 0)
+        for (int c = 0; c < csize; ++c) {
+            int32_t *dst = cluster.map_shared_rank(all_tot, c) + crank * W;
+            dst[E + R] = misc[0];
+            dst[E + R + 1] = misc[1];
         }
-        tot_r[r] = run;
-    }
-    cluster.sync();  // every CTA's totals are now readable by its peers
+    cluster.sync();  // all totals have arrived in every CTA's shared memory
 
-    // ---- cluster-wide: base of this CTA, global scan over experts / ranks
+    // ---- global exclusive scans (local reads only), cursors, CTA 0 writes out
     {
         const int per = (E + blockDim.x - 1) / blockDim.x;
         const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
         int local = 0;
         for (int e = e0; e < e1; ++e)
-            for (int c = 0; c < csize; ++c) local += cluster.map_shared_rank(tot_e, c)[e];
+            for (int c = 0; c < csize; ++c) local += all_tot[c * W + e];
         int total_e;
         int run = block_exclusive_scan(local, scan, &total_e);
         for (int e = e0; e < e1; ++e) {
             int base = 0, tot = 0;
             for (int c = 0; c < csize; ++c) {
-                int v = cluster.map_shared_rank(tot_e, c)[e];
+                const int v = all_tot[c * W + e];
                 base += c < crank ? v : 0;
                 tot += v;
             }
-            for (int w = 0; w < NW; ++w) hist_e[w * E + e] += run + base;
+            for (int w = 0; w < NWW; ++w) hist_e[w * E + e] += run + base;
             if (crank == 0) {
                 p.cnt_e[e] = tot;
                 p.off_e[e] = run;
@@ -223,75 +238,75 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
         const int r = tid;
         int tot_rr = 0, base_r = 0;
-        if (r < R) {
+        if (r < R)
             for (int c = 0; c < csize; ++c) {
-                int v = cluster.map_shared_rank(tot_r, c)[r];
+                const int v = all_tot[c * W + E + r];
                 base_r += c < crank ? v : 0;
                 tot_rr += v;
             }
-        }
         int total_r;
-        int off_r = block_exclusive_scan(tot_rr, scan, &total_r);
+        const int off_r = block_exclusive_scan(tot_rr, scan, &total_r);
         if (r < R) {
-            for (int w = 0; w < NW; ++w) hist_r[w * R + r] += off_r + base_r;
+            for (int w = 0; w < NWW; ++w) hist_r[w * R + r] += off_r + base_r;
             if (crank == 0) {
                 p.cnt_r[r] = tot_rr;
                 p.off_r[r] = off_r;
             }
         }
-        if (tid == 0) {
+        if (tid == 0 && crank == 0) {
             int errc = 0, nr = 0;
             for (int c = 0; c < csize; ++c) {
-                const int32_t *m = cluster.map_shared_rank(misc, c);
-                errc |= m[0];
-                nr += m[1];
+                errc |= all_tot[c * W + E + R];
+                nr += all_tot[c * W + E + R + 1];
             }
-            if (crank == 0) {
-                p.off_e[E] = total_e;
-                p.off_r[R] = total_r;
-                p.totals[0] = total_e;
-                p.totals[1] = total_r;
-                p.totals[2] = nr;
-                p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
-            }
+            p.off_e[E] = total_e;
+            p.off_r[R] = total_r;
+            p.totals[0] = total_e;
+            p.totals[1] = total_r;
+            p.totals[2] = nr;
+            p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
         }
     }
-    cluster.sync();  // peers are done reading; cursors visible CTA-wide
+    __syncthreads();  // cursors visible to the walkers
 
-    // ---- pass 2: positions, in (token, slot) order
+    // ---- pass 2: positions, in (token, slot) order, by the walker warps
     const unsigned lt = lanemask_lt();
     const int tl = lane / k;
     const int j = lane - tl * k;
     for (int c = 0; c < nchunks; ++c) {
-        if (nchunks > 1) stage_chunk(p, idx, rg, c, NW, codes, misc, false);
-        const int tb = rg.w0(wid) + c * S;  // first token of this warp's slice
-        for (int s0 = 0; s0 < S; s0 += tps) {
-            const int s = s0 + tl;
-            const bool lane_ok = tl < tps && s < S;
-            const int code = lane_ok ? my_codes[s * k + j] : kAbsent;
-            const bool valid = code >= 0;
-            const int e = valid ? (code & 0xffff) : -1;
-            const bool first = valid && (code & (1 << 30));
-            const int r = (code >> 16) & 0x3f;
-            const unsigned pe = __match_any_sync(kFull, e);
-            const unsigned pr = __match_any_sync(kFull, first ? r : -1);
-            const int base = valid ? hist_e[wid * E + e] : 0;
-            const int base_r = first ? hist_r[wid * R + r] : 0;
-            __syncwarp();
-            if (valid && lane == __ffs(pe) - 1) hist_e[wid * E + e] = base + __popc(pe);
-            if (first && lane == __ffs(pr) - 1) hist_r[wid * R + r] = base_r + __popc(pr);
-            const size_t t = (size_t)(tb + s);
-            if (code != kAbsent) p.pos[t * k + j] = valid ? base + __popc(pe & lt) : -1;
-            if (first) p.recv_pos[t * R + r] = base_r + __popc(pr & lt);
-            __syncwarp();
+        if (nchunks > 1) stage_chunk(p, idx, rg, c, codes, misc, false);
+        if (wid < NWW) {
+            const int32_t *my_codes = codes + (size_t)wid * S * k;
+            const int tb = rg.w0(wid) + c * S;  // first token of this walker's slice
+            for (int s0 = 0; s0 < S; s0 += tps) {
+                const int s = s0 + tl;
+                const bool lane_ok = tl < tps && s < S;
+                const int code = lane_ok ? my_codes[s * k + j] : kAbsent;
+                const bool valid = code >= 0;
+                const int e = valid ? (code & 0xffff) : -1;
+                const bool first = valid && (code & (1 << 30));
+                const int r = (code >> 16) & 0x3f;
+                const unsigned pe = __match_any_sync(kFull, e);
+                const unsigned pr = __match_any_sync(kFull, first ? r : -1);
+                const int base = valid ? hist_e[wid * E + e] : 0;
+                const int base_r = first ? hist_r[wid * R + r] : 0;
+                __syncwarp();
+                if (valid && lane == __ffs(pe) - 1) hist_e[wid * E + e] = base + __popc(pe);
+                if (first && lane == __ffs(pr) - 1) hist_r[wid * R + r] = base_r + __popc(pr);
+                const size_t t = (size_t)(tb + s);
+                if (code != kAbsent) p.pos[t * k + j] = valid ? base + __popc(pe & lt) : -1;
+                if (first) p.recv_pos[t * R + r] = base_r + __popc(pr & lt);
+                __syncwarp();
+            }
         }
         if (nchunks > 1) __syncthreads();  // codes are restaged next chunk
     }
 }
 
-size_t layout_smem_bytes(int NW, int E, int R, int S, int k)
+size_t layout_smem_bytes(int NWW, int E, int R, int S, int k, int csize)
 {
-    return sizeof(int32_t) * ((size_t)NW * (E + R) + E + R + 4 + 36 + (size_t)NW * S * k);
+    return sizeof(int32_t) *
+           ((size_t)NWW * (E + R) + (size_t)csize * (E + R + 2) + 4 + 36 + (size_t)NWW * S * k);
 }
 
 // cudaOccupancyMaxActiveClusters for (cluster size, threads, smem), cached
@@ -331,42 +346,44 @@ int max_clusters(int csize, int threads, size_t smem, int dev)
 }
 
 struct Geometry {
-    int csize, NW, tpc, tpw, S;
+    int csize, threads, nww, tpc, tpw, S;
     size_t smem;
 };
 
-// Cluster size, warps per CTA and staging chunk for a layout problem.
+// Cluster size, walker warps and staging chunk for a layout problem.  The
+// CTA always has 1024 threads: the expert-proportional work (zeroing, scans,
+// writing counts and offsets) is spread over all of them, while only the
+// walker warps own token ranges.
 Geometry plan(int T, int k, int E, int R, int csize)
 {
     Geometry g;
     const int tps = 32 / k;
     g.csize = csize;
+    g.threads = 1024;
     g.tpc = (T + csize - 1) / csize;
     const int steps = (g.tpc + tps - 1) / tps;
-    const int nw_ranks = (R + 31) / 32;  // the rank scan gives one rank per thread
-    // about 4 steps per warp: enough warps to spread the walk, few enough
-    // that the per-expert scans over warps stay short
-    int NW = (steps + 3) / 4;
-    if (NW > 32) NW = 32;
-    if (NW < nw_ranks) NW = nw_ranks;
-    if (NW < 1) NW = 1;
+    // about 4 ordered steps per walker: enough walkers to spread the walk,
+    // few enough that the per-expert scans over walkers stay short
+    int nww = (steps + 3) / 4;
+    if (nww > 32) nww = 32;
+    if (nww < 1) nww = 1;
     for (;;) {
-        int tpw = (g.tpc + NW - 1) / NW;
+        int tpw = (g.tpc + nww - 1) / nww;
         tpw = ((tpw + tps - 1) / tps) * tps;
         if (tpw < tps) tpw = tps;
-        const size_t base = layout_smem_bytes(NW, E, R, 0, k);
-        long long avail = (long long)kMaxDynSmem - (long long)base;
-        int S = avail > 0 ? (int)(avail / ((long long)NW * k * 4)) : 0;
+        const size_t base = layout_smem_bytes(nww, E, R, 0, k, csize);
+        const long long avail = (long long)kMaxDynSmem - (long long)base;
+        int S = avail > 0 ? (int)(avail / ((long long)nww * k * 4)) : 0;
         S = (S / tps) * tps;
         if (S > tpw) S = tpw;
-        if (S >= tps || NW <= nw_ranks) {
-            g.NW = NW;
+        if (S >= tps || nww == 1) {
+            g.nww = nww;
             g.tpw = tpw;
             g.S = S < tps ? tps : S;
-            g.smem = layout_smem_bytes(NW, E, R, g.S, k);
+            g.smem = layout_smem_bytes(nww, E, R, g.S, k, csize);
             return g;
         }
-        --NW;
+        --nww;
     }
 }
 
@@ -390,15 +407,16 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
     int csize = (int)((routes + 4095) / 4096);
     csize = csize < 1 ? 1 : (csize > 8 ? 8 : csize);
     Geometry g = plan(p.T, p.k, p.E, p.R, csize);
-    while (g.csize > 1 && max_clusters<IdxT>(g.csize, g.NW * 32, g.smem, dev) == 0)
+    while (g.csize > 1 && max_clusters<IdxT>(g.csize, g.threads, g.smem, dev) == 0)
         g = plan(p.T, p.k, p.E, p.R, g.csize >> 1);
     p.tpc = g.tpc;
     p.tpw = g.tpw;
     p.S = g.S;
+    p.nww = g.nww;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(g.csize, 1, 1);
-    cfg.blockDim = dim3(g.NW * 32, 1, 1);
+    cfg.blockDim = dim3(g.threads, 1, 1);
     cfg.dynamicSmemBytes = g.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
