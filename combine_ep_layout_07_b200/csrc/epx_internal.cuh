@@ -16,10 +16,13 @@ constexpr unsigned kFull = 0xffffffffu;
 struct LayoutParams {
     const void *idx;
     int T, k, E, R, epr;
-    int tpc;  // tokens per CTA of the cluster
-    int tpw;  // tokens per warp (a multiple of 32 / k)
-    int S;    // tokens per warp staged in shared memory at a time (multiple of 32 / k)
-    int nww;  // walker warps: warps that own a token range and a histogram row
+    float inv_epr;  // 1.0f / epr (rank of expert e = floor((e + 0.5) * inv_epr))
+    int tpc;        // tokens per CTA of the cluster
+    int tpw;        // tokens per walker warp (a multiple of 32 / k)
+    int S;          // tokens per walker staged in shared memory at a time
+    int nww;        // walker warps: warps that own a token range and a histogram row
+    int tpe, per;   // walker scans: threads per expert group, experts per group
+    int tpr;        // walker scans: threads per rank
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 
