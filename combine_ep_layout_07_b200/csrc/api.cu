@@ -113,7 +113,7 @@ ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
     p.k = L->k;
     p.E = L->E;
     p.R = L->R;
-    p.epr = L->E / L->R;
+    p.inv_epr = 1.0f / (float)(L->E / L->R);
     p.cnt_e = L->cnt_e;
     p.off_e = L->off_e;
     p.cnt_r = L->cnt_r;

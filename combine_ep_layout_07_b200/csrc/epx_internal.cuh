@@ -15,14 +15,14 @@ constexpr unsigned kFull = 0xffffffffu;
 
 struct LayoutParams {
     const void *idx;
-    int T, k, E, R, epr;
-    float inv_epr;  // 1.0f / epr (rank of expert e = floor((e + 0.5) * inv_epr))
+    int T, k, E, R;
+    float inv_epr;  // 1.0f / (E / R): rank of expert e = floor((e + 0.5) * inv_epr)
     int tpc;        // tokens per CTA of the cluster
-    int tpw;        // tokens per walker warp (a multiple of 32 / k)
-    int S;          // tokens per walker staged in shared memory at a time
-    int nww;        // walker warps: warps that own a token range and a histogram row
-    int tpe, per;   // walker scans: threads per expert group, experts per group
-    int tpr;        // walker scans: threads per rank
+    int tch;        // tokens per chunk (rows of the count matrix)
+    int wde, wdr;   // 32-bit words per count-matrix row for experts / ranks
+    int wds;        // row stride in words (odd, so column walks avoid bank conflicts)
+    int nseg;       // threads per column in the column scan (power of two <= 32)
+    int lg_nseg;
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 

@@ -8,31 +8,31 @@
 // Reproduction: padding rows of -1) and experts on ranks in contiguous
 // blocks of E/R (issue #760, Reproduction: local_experts).
 //
-// Design: one launch of one CTA, or of one thread-block cluster of up to 16
-// CTAs, each of 1024 threads.
-//  * tokens are split into contiguous ranges: CTA c of the cluster, then
-//    walker warp w of the CTA; a walker walks its range in steps of
-//    floor(32/k) whole tokens, one route per lane, so lane order inside a
-//    step is (token, slot) order;
-//  * staging + counting: the CTA loads its routes with coalesced loads into
-//    shared memory (one DRAM round trip), then one thread per token
-//    validates the indices, computes each route's rank, marks the first
-//    route of every (token, rank) pair and counts both into the walker's
-//    histogram row with shared-memory atomics (order does not matter for
-//    counts);
-//  * walker scans: per expert (and per rank) an exclusive scan over the
-//    walkers, several threads per expert, combined with warp shuffles;
+// A route's row is off_e[e] + (routes to e from earlier tokens) + (earlier
+// slots of its own token with the same expert); a (token, rank) pair's row
+// is off_r[r] + (earlier tokens that reach r).  Both middle terms are column
+// prefix sums of a token x expert (and token x rank) count matrix, so they
+// are computed here without any ordering primitive:
+//  * one launch of one CTA, or of one thread-block cluster of up to 16 CTAs
+//    of 1024 threads; CTA c owns a contiguous range of tokens;
+//  * build: one thread per token loads its k indices, validates them,
+//    computes each route's rank, marks the first route of every
+//    (token, rank) pair and counts the token's row of the count matrix in
+//    shared memory -- counts are packed two 16-bit columns per 32-bit word,
+//    and the count seen before incrementing is the route's rank among equal
+//    experts of its own token;
+//  * column scan: every column of the matrix is prefix-summed over the
+//    tokens, several threads per column combined with warp shuffles (packed
+//    16-bit halves add independently); the column sums are the CTA totals;
 //  * cluster exchange: each CTA pushes its totals into every peer's shared
-//    memory (distributed shared memory stores) and one cluster barrier later
-//    reads them all locally; a single CTA skips this;
+//    memory (distributed shared memory stores); after one cluster barrier
+//    every CTA reads them locally; a single CTA skips this;
 //  * global scan: one block-wide scan of packed 64-bit (expert, rank) counts
-//    gives both exclusive scans at once; the walker cursors become
-//    offset + CTA base + walker prefix;
-//  * ordered walk: __match_any_sync groups a step's lanes by expert (and the
-//    first routes by rank); each lane takes its walker's cursor plus the
-//    number of lower lanes in its group and the group leader advances it.
-// Rows come out ordered by token, then slot, inside every expert segment and
-// every rank segment, independent of scheduling.
+//    gives both exclusive scans at once, plus this CTA's base;
+//  * positions: one thread per token again, reading its prefixes back.
+// When a CTA's tokens do not fit in shared memory at once, it counts all of
+// them first (atomics into its totals) and then builds, scans and places the
+// tokens chunk by chunk with a running cursor per column.
 #include <cooperative_groups.h>
 
 #include "epx_internal.cuh"
@@ -42,14 +42,17 @@ namespace cg = cooperative_groups;
 namespace epx {
 namespace {
 
-// staged route code: -2 = no token here, -1 = no route (or a dropped bad
-// index), else expert | rank << 16 | (first route of its rank) << 30
-constexpr int kAbsent = -2;
-constexpr int kMaxPer = EPX_MAX_EXPERTS / 1024;  // experts per thread at most
-constexpr int kScanInts = 2 * 34;                 // 64-bit block-scan scratch
+constexpr int kScanInts = 2 * 34;  // 64-bit block-scan scratch
+constexpr int kMaxPer = EPX_MAX_EXPERTS / 1024;
 
-// Exclusive scan of one 64-bit value per thread across the CTA.  No barrier
-// after the last read of `sm`: the caller separates reuses with a barrier.
+// route code in shared memory: -1 = no route (or a dropped bad index), else
+// expert | rank << 12 | (rank among equal experts of the token) << 18 |
+// (first route of its rank) << 23
+__device__ __forceinline__ int code_e(int c) { return c & 0xfff; }
+__device__ __forceinline__ int code_r(int c) { return (c >> 12) & 0x3f; }
+__device__ __forceinline__ int code_dup(int c) { return (c >> 18) & 0x1f; }
+__device__ __forceinline__ bool code_first(int c) { return (c >> 23) & 1; }
+
 __device__ unsigned long long block_exclusive_scan64(unsigned long long v,
                                                      unsigned long long *sm,
                                                      unsigned long long *total)
@@ -80,27 +83,6 @@ __device__ unsigned long long block_exclusive_scan64(unsigned long long v,
     return sm[wid] + inc - v;
 }
 
-// Exclusive scan inside aligned groups of `width` lanes (a power of two);
-// every lane of the warp takes part.  *total gets the group's sum.
-__device__ __forceinline__ int group_exclusive_scan(int v, int width, int *total)
-{
-    const int sub = (threadIdx.x & 31) & (width - 1);
-    int inc = v;
-    for (int o = 1; o < width; o <<= 1) {
-        const int n = __shfl_up_sync(kFull, inc, o, width);
-        if (sub >= o) inc += n;
-    }
-    *total = __shfl_sync(kFull, inc, width - 1, width);
-    return inc - v;
-}
-
-struct Ranges {
-    int c0, c1;  // this CTA's tokens
-    int tpw;     // tokens per walker warp
-    __device__ int w0(int w) const { return min(c1, c0 + w * tpw); }
-    __device__ int w1(int w) const { return min(c1, c0 + (w + 1) * tpw); }
-};
-
 __device__ __forceinline__ int rank_of(int e, float inv_epr)
 {
     // exact for e < 2^22: (e + 1/2) / epr is at least 1/(2 epr) away from an
@@ -108,87 +90,144 @@ __device__ __forceinline__ int rank_of(int e, float inv_epr)
     return __float2int_rd(__fmul_rn(__fadd_rn((float)e, 0.5f), inv_epr));
 }
 
-// Stage chunk c (tokens [w0 + c*S, w0 + c*S + S) of every walker w) into
-// codes[w][s*k + j].  In the first pass also: fill recv_pos with -1 for the
-// staged tokens, count every route into its walker's histograms and record
-// bad indices / real tokens in misc[0] / misc[1].
+// Thread-per-token pass over tokens [t0, t0 + n).  With M != nullptr it
+// builds the count-matrix rows (zeroed beforehand) and the route codes; with
+// tot != nullptr it counts into the CTA totals with atomics instead.  Returns
+// the number of this thread's tokens with a valid route; *bad is set if an
+// index < -1 or >= E was seen.
 template <typename IdxT>
-__device__ void stage_chunk(const LayoutParams &p, const IdxT *__restrict__ idx,
-                            const Ranges &rg, int c, int32_t *codes, int32_t *hist_e,
-                            int32_t *hist_r, int32_t *misc, bool first_pass)
+__device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx, int t0, int n,
+                            uint32_t *M, int32_t *codes, int32_t *tot, bool *bad)
 {
-    const int k = p.k, S = p.S, E = p.E, R = p.R, NWW = p.nww;
-    const int per_w = S * k;
-    const int n = NWW * per_w;
-    bool bad = false;
-    // coalesced raw loads, four in flight per thread: consecutive threads
-    // take consecutive routes of a walker's slice (contiguous in topk_idx)
-    for (int i0 = threadIdx.x; i0 < n; i0 += 4 * blockDim.x) {
-        long long e[4];
-        bool in[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * blockDim.x;
-            const int w = i / per_w;
-            const int rem = i - w * per_w;
-            in[u] = i < n && rg.w0(w) + c * S + rem / k < rg.w1(w);
-            e[u] = in[u] ? (long long)idx[(size_t)rg.w0(w) * k + (size_t)c * per_w + rem] : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * blockDim.x;
-            if (i < n) {
-                bad |= in[u] && (e[u] < -1 || e[u] >= E);
-                codes[i] = !in[u] ? kAbsent : ((e[u] >= 0 && e[u] < E) ? (int)e[u] : -1);
-            }
-        }
-    }
-    if (first_pass) {
-        const int per_wr = S * R;
-        for (int i = threadIdx.x; i < NWW * per_wr; i += blockDim.x) {
-            const int w = i / per_wr;
-            const int rem = i - w * per_wr;
-            if (rg.w0(w) + c * S + rem / R < rg.w1(w))
-                p.recv_pos[(size_t)(rg.w0(w) + c * S) * R + rem] = -1;
-        }
-    }
-    __syncthreads();
-    // one thread per token: rank of each route, first route of each rank,
-    // and (first pass) the counts
+    const int k = p.k, E = p.E;
     int nreal = 0;
-    for (int u = threadIdx.x; u < NWW * S; u += blockDim.x) {
-        const int w = u / S;
-        const int t = rg.w0(w) + c * S + (u - w * S);
-        if (t >= rg.w1(w)) continue;
-        int32_t *cd = codes + (size_t)u * k;
+    for (int u = threadIdx.x; u < n; u += blockDim.x) {
+        const IdxT *row = idx + (size_t)(t0 + u) * k;
+        uint32_t *mrow = M ? M + (size_t)u * p.wds : nullptr;
         unsigned long long mask = 0ull;
-        for (int j = 0; j < k; ++j) {
-            const int e = cd[j];
-            if (e < 0) continue;
-            const int r = rank_of(e, p.inv_epr);
-            const bool f = !((mask >> r) & 1ull);
-            mask |= 1ull << r;
-            cd[j] = e | (r << 16) | ((int)f << 30);
-            if (first_pass) {
-                atomicAdd(&hist_e[w * E + e], 1);
-                if (f) atomicAdd(&hist_r[w * R + r], 1);
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            long long ev[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) ev[q] = j0 + q < k ? (long long)row[j0 + q] : -1;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int j = j0 + q;
+                if (j >= k) break;
+                const long long e = ev[q];
+                *bad |= (e < -1 || e >= E);
+                int code = -1;
+                if (e >= 0 && e < E) {
+                    const int ei = (int)e;
+                    const int r = rank_of(ei, p.inv_epr);
+                    const bool first = !((mask >> r) & 1ull);
+                    mask |= 1ull << r;
+                    if (mrow) {
+                        const int sh = (ei & 1) * 16;
+                        const uint32_t w = mrow[ei >> 1];
+                        const int dup = (int)((w >> sh) & 0xffffu);
+                        mrow[ei >> 1] = w + (1u << sh);
+                        if (first) mrow[p.wde + (r >> 1)] += 1u << ((r & 1) * 16);
+                        code = ei | (r << 12) | (dup << 18) | ((int)first << 23);
+                    } else {
+                        atomicAdd(&tot[ei], 1);
+                        if (first) atomicAdd(&tot[E + r], 1);
+                    }
+                }
+                if (codes) codes[(size_t)u * k + j] = code;
             }
         }
         nreal += mask != 0ull;
     }
-    if (first_pass) {
-        if (__any_sync(kFull, bad) && (threadIdx.x & 31) == 0) atomicOr(&misc[0], 1);
-        if (nreal) atomicAdd(&misc[1], nreal);
+    return nreal;
+}
+
+// Exclusive prefix of every column of M (n rows, wde + wdr packed columns)
+// over its rows.  With csum != nullptr the column sums go to csum[E + R]
+// (experts first, then ranks).
+__device__ void column_scan(const LayoutParams &p, uint32_t *M, int n, int32_t *csum)
+{
+    const int wdt = p.wde + p.wdr;
+    const int nseg = p.nseg;
+    const int s = threadIdx.x & (nseg - 1);
+    const int rps = (n + nseg - 1) >> p.lg_nseg;
+    const int ra = min(n, s * rps), rb = min(n, ra + rps);
+    const int cols_per_pass = blockDim.x >> p.lg_nseg;
+    for (int cbase = 0; cbase < wdt; cbase += cols_per_pass) {
+        const int c = cbase + (threadIdx.x >> p.lg_nseg);
+        const bool ok = c < wdt;
+        uint32_t sum = 0;
+        if (ok)
+            for (int r = ra; r < rb; ++r) sum += M[(size_t)r * p.wds + c];
+        // exclusive scan of the packed sums across the column's segments
+        uint32_t inc = sum;
+        for (int o = 1; o < nseg; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, inc, o, nseg);
+            if (s >= o) inc += v;
+        }
+        const uint32_t total = __shfl_sync(kFull, inc, nseg - 1, nseg);
+        if (ok) {
+            uint32_t run = inc - sum;
+            for (int r = ra; r < rb; ++r) {
+                const uint32_t v = M[(size_t)r * p.wds + c];
+                M[(size_t)r * p.wds + c] = run;
+                run += v;
+            }
+            if (csum && s == 0) {
+                const bool er = c < p.wde;
+                const int col0 = er ? 2 * c : 2 * (c - p.wde);
+                const int lim = er ? p.E : p.R;
+                int32_t *dst = er ? csum : csum + p.E;
+                dst[col0] = (int32_t)(total & 0xffffu);
+                if (col0 + 1 < lim) dst[col0 + 1] = (int32_t)(total >> 16);
+            }
+        }
     }
-    __syncthreads();
+}
+
+// Thread-per-token: write pos and recv_pos of tokens [t0, t0 + n) from the
+// scanned matrix, the route codes and the per-column bases.
+__device__ void place_tokens(const LayoutParams &p, int t0, int n, const uint32_t *M,
+                             const int32_t *codes, const int32_t *base)
+{
+    const int k = p.k, E = p.E, R = p.R;
+    for (int u = threadIdx.x; u < n; u += blockDim.x) {
+        const size_t t = (size_t)(t0 + u);
+        const uint32_t *mrow = M + (size_t)u * p.wds;
+        unsigned long long hit = 0ull;
+        for (int j = 0; j < k; ++j) {
+            const int c = codes[(size_t)u * k + j];
+            int v = -1;
+            if (c >= 0) {
+                const int e = code_e(c);
+                v = base[e] + (int)((mrow[e >> 1] >> ((e & 1) * 16)) & 0xffffu) + code_dup(c);
+                if (code_first(c)) hit |= 1ull << code_r(c);
+            }
+            p.pos[t * k + j] = v;
+        }
+        for (int r = 0; r < R; ++r) {
+            int v = -1;
+            if ((hit >> r) & 1ull)
+                v = base[E + r] + (int)((mrow[p.wde + (r >> 1)] >> ((r & 1) * 16)) & 0xffffu);
+            p.recv_pos[t * R + r] = v;
+        }
+    }
+}
+
+__device__ void zero_words(uint32_t *a, int n)
+{
+    // a is 16-byte aligned; vector stores for the bulk, scalars for the tail
+    uint4 *a4 = reinterpret_cast<uint4 *>(a);
+    const int n4 = n >> 2;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) a4[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) a[i] = 0u;
 }
 
 template <typename IdxT, bool CLUSTER>
 __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 {
     extern __shared__ __align__(16) int32_t smem[];
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int E = p.E, R = p.R, k = p.k, T = p.T, S = p.S, NWW = p.nww;
+    const int tid = threadIdx.x;
+    const int E = p.E, R = p.R, T = p.T;
 
     int crank = 0, csize = 1;
     if (CLUSTER) {
@@ -200,140 +239,102 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     }
 
-    const int W = E + R + 2;  // one CTA's totals: experts, ranks, bad, real
+    const int W = E + R + 2;  // one CTA's published totals: experts, ranks, bad, real
     unsigned long long *scan = reinterpret_cast<unsigned long long *>(smem);
-    int32_t *hist_e = smem + kScanInts;      // [NWW][E] walker counts, then cursors
-    int32_t *hist_r = hist_e + NWW * E;      // [NWW][R]
-    int32_t *all_tot = hist_r + NWW * R;     // [csize][W], row c = CTA c's totals
-    int32_t *misc = all_tot + csize * W;     // [4]  0: bad-index flag, 1: real tokens
-    int32_t *codes = misc + 4;               // [NWW][S*k] staged routes
-
-    for (int i = tid; i < NWW * (E + R); i += blockDim.x) hist_e[i] = 0;
-    if (tid < 4) misc[tid] = 0;
-    __syncthreads();
+    uint32_t *M = reinterpret_cast<uint32_t *>(smem + kScanInts);  // [tch][wds]
+    const size_t m_words = ((size_t)p.tch * p.wds + 3) & ~(size_t)3;
+    int32_t *codes = smem + kScanInts + m_words;   // [tch][k]
+    int32_t *tot = codes + (size_t)p.tch * p.k;    // [E + R] CTA totals / chunk sums
+    int32_t *base = tot + E + R;                   // [E + R] this CTA's row bases
+    int32_t *all_tot = base + E + R;               // [csize][W]
+    int32_t *misc = all_tot + csize * W;           // [2] bad flag, real tokens
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
-    Ranges rg;
-    rg.c0 = min(T, crank * p.tpc);
-    rg.c1 = min(T, rg.c0 + p.tpc);
-    rg.tpw = p.tpw;
-    const int nchunks = (p.tpw + S - 1) / S;
+    const int c0 = min(T, crank * p.tpc);
+    const int nt = min(T, c0 + p.tpc) - c0;
+    const int nchunks = (nt + p.tch - 1) / p.tch;
+    bool bad = false;
+    int nreal = 0;
 
-    // ---- staging and counting
-    for (int c = 0; c < nchunks; ++c) stage_chunk(p, idx, rg, c, codes, hist_e, hist_r, misc, true);
-
-    if (CLUSTER) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-
-    // ---- exclusive scans over walkers; publish this CTA's totals
-    auto publish = [&](int slot, int v) {
-        if (CLUSTER) {
-            cg::cluster_group cluster = cg::this_cluster();
-            for (int c = 0; c < csize; ++c) cluster.map_shared_rank(all_tot, c)[crank * W + slot] = v;
-        } else {
-            all_tot[slot] = v;
-        }
-    };
-    const int tpe = p.tpe, per = p.per;
-    const int g = tid / tpe, sub = tid & (tpe - 1);
-    const int wps = (NWW + tpe - 1) / tpe;
-    const int wa = min(NWW, sub * wps), wb = min(NWW, wa + wps);
-#pragma unroll
-    for (int q = 0; q < kMaxPer; ++q) {
-        if (q >= per) break;
-        const int e = g * per + q;
-        const bool ok = e < E;
-        int s = 0;
-        if (ok)
-            for (int w = wa; w < wb; ++w) s += hist_e[w * E + e];
-        int tot;
-        int run = group_exclusive_scan(s, tpe, &tot);
-        if (ok) {
-            for (int w = wa; w < wb; ++w) {
-                const int v = hist_e[w * E + e];
-                hist_e[w * E + e] = run;
-                run += v;
-            }
-            if (sub == tpe - 1) publish(e, tot);
-        }
-    }
-    const int tpr = p.tpr;
-    const int gr = tid / tpr, subr = tid & (tpr - 1);
-    const int wpr = (NWW + tpr - 1) / tpr;
-    const int wra = min(NWW, subr * wpr), wrb = min(NWW, wra + wpr);
-    {
-        const bool ok = gr < R;
-        int s = 0;
-        if (ok)
-            for (int w = wra; w < wrb; ++w) s += hist_r[w * R + gr];
-        int tot;
-        int run = group_exclusive_scan(s, tpr, &tot);
-        if (ok) {
-            for (int w = wra; w < wrb; ++w) {
-                const int v = hist_r[w * R + gr];
-                hist_r[w * R + gr] = run;
-                run += v;
-            }
-            if (subr == tpr - 1) publish(E + gr, tot);
-        }
-    }
-    if (tid == 0) {
-        publish(E + R, misc[0]);
-        publish(E + R + 1, misc[1]);
-    }
-    if (CLUSTER)
-        cg::this_cluster().sync();  // all totals have arrived in every CTA
-    else
+    if (tid < 2) misc[tid] = 0;
+    if (nchunks <= 1) {
+        zero_words(M, p.tch * p.wds);
         __syncthreads();
+        nreal = build_tokens(p, idx, c0, nt, M, codes, nullptr, &bad);
+        __syncthreads();
+        column_scan(p, M, nt, tot);
+    } else {
+        for (int i = tid; i < E + R; i += blockDim.x) tot[i] = 0;
+        __syncthreads();
+        nreal = build_tokens(p, idx, c0, nt, nullptr, nullptr, tot, &bad);
+    }
+    if (__any_sync(kFull, bad) && (tid & 31) == 0) atomicOr(&misc[0], 1);
+    if (nreal) atomicAdd(&misc[1], nreal);
+    __syncthreads();
 
-    // ---- global exclusive scans (one packed 64-bit block scan), cursors
+    // ---- publish this CTA's totals (to every CTA of the cluster)
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+        for (int i = tid; i < E + R + 2; i += blockDim.x) {
+            const int v = i < E + R ? tot[i] : misc[i - E - R];
+            for (int c = 0; c < csize; ++c) cluster.map_shared_rank(all_tot, c)[crank * W + i] = v;
+        }
+        cluster.sync();
+    } else {
+        for (int i = tid; i < E + R + 2; i += blockDim.x)
+            all_tot[i] = i < E + R ? tot[i] : misc[i - E - R];
+        __syncthreads();
+    }
+
+    // ---- global exclusive scans (one packed 64-bit block scan) and bases
     {
-        int glob[kMaxPer], base[kMaxPer];
+        const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+        int glob[kMaxPer], cbase[kMaxPer];
         unsigned int contrib_e = 0;
 #pragma unroll
         for (int q = 0; q < kMaxPer; ++q) {
             glob[q] = 0;
-            base[q] = 0;
-            const int e = g * per + q;
+            cbase[q] = 0;
+            const int e = tid * per + q;
             if (q < per && e < E) {
                 for (int c = 0; c < csize; ++c) {
                     const int v = all_tot[c * W + e];
-                    base[q] += c < crank ? v : 0;
+                    cbase[q] += c < crank ? v : 0;
                     glob[q] += v;
                 }
                 contrib_e += glob[q];
             }
         }
-        int glob_r = 0, base_r = 0;
-        if (gr < R)
+        int glob_r = 0, cbase_r = 0;
+        if (tid < R)
             for (int c = 0; c < csize; ++c) {
-                const int v = all_tot[c * W + E + gr];
-                base_r += c < crank ? v : 0;
+                const int v = all_tot[c * W + E + tid];
+                cbase_r += c < crank ? v : 0;
                 glob_r += v;
             }
-        const unsigned long long v =
-            ((unsigned long long)(sub == tpe - 1 ? contrib_e : 0u) << 32) |
-            (unsigned long long)(gr < R && subr == tpr - 1 ? (unsigned)glob_r : 0u);
+        const unsigned long long v = ((unsigned long long)contrib_e << 32) | (unsigned)glob_r;
         unsigned long long total;
         const unsigned long long ex = block_exclusive_scan64(v, scan, &total);
         unsigned int run = (unsigned int)(ex >> 32);
 #pragma unroll
         for (int q = 0; q < kMaxPer; ++q) {
-            const int e = g * per + q;
+            const int e = tid * per + q;
             if (q < per && e < E) {
-                for (int w = wa; w < wb; ++w) hist_e[w * E + e] += (int)run + base[q];
-                if (crank == 0 && sub == 0) {
+                base[e] = (int)run + cbase[q];
+                if (crank == 0) {
                     p.cnt_e[e] = glob[q];
                     p.off_e[e] = (int)run;
                 }
                 run += glob[q];
             }
         }
-        if (gr < R) {
+        if (tid < R) {
             const int off_r = (int)(unsigned int)(ex & 0xffffffffull);
-            for (int w = wra; w < wrb; ++w) hist_r[w * R + gr] += off_r + base_r;
-            if (crank == 0 && subr == 0) {
-                p.cnt_r[gr] = glob_r;
-                p.off_r[gr] = off_r;
+            base[E + tid] = off_r + cbase_r;
+            if (crank == 0) {
+                p.cnt_r[tid] = glob_r;
+                p.off_r[tid] = off_r;
             }
         }
         if (tid == 0 && crank == 0) {
@@ -352,48 +353,31 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
             p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
         }
     }
-    __syncthreads();  // cursors visible to the walkers
+    __syncthreads();
 
-    // ---- ordered walk: positions in (token, slot) order
-    const int tps = 32 / k;
-    const unsigned lt = lanemask_lt();
-    const int tl = lane / k;
-    const int j = lane - tl * k;
-    for (int c = 0; c < nchunks; ++c) {
-        if (nchunks > 1) stage_chunk(p, idx, rg, c, codes, hist_e, hist_r, misc, false);
-        if (wid < NWW) {
-            const int32_t *my_codes = codes + (size_t)wid * S * k;
-            const int tb = rg.w0(wid) + c * S;  // first token of this walker's slice
-            for (int s0 = 0; s0 < S; s0 += tps) {
-                const int s = s0 + tl;
-                const bool lane_ok = tl < tps && s < S;
-                const int code = lane_ok ? my_codes[s * k + j] : kAbsent;
-                const bool valid = code >= 0;
-                const int e = valid ? (code & 0xffff) : -1;
-                const bool first = valid && (code & (1 << 30));
-                const int r = (code >> 16) & 0x3f;
-                const unsigned pe = __match_any_sync(kFull, e);
-                const unsigned pr = __match_any_sync(kFull, first ? r : -1);
-                const int base = valid ? hist_e[wid * E + e] : 0;
-                const int base_r = first ? hist_r[wid * R + r] : 0;
-                __syncwarp();
-                if (valid && lane == __ffs(pe) - 1) hist_e[wid * E + e] = base + __popc(pe);
-                if (first && lane == __ffs(pr) - 1) hist_r[wid * R + r] = base_r + __popc(pr);
-                const size_t t = (size_t)(tb + s);
-                if (code != kAbsent) p.pos[t * k + j] = valid ? base + __popc(pe & lt) : -1;
-                if (first) p.recv_pos[t * R + r] = base_r + __popc(pr & lt);
-                __syncwarp();
-            }
-        }
-        if (nchunks > 1) __syncthreads();  // codes are restaged next chunk
+    // ---- positions
+    if (nchunks <= 1) {
+        place_tokens(p, c0, nt, M, codes, base);
+        return;
+    }
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const int t0 = c0 + ch * p.tch;
+        const int n = min(p.tch, c0 + nt - t0);
+        zero_words(M, p.tch * p.wds);
+        __syncthreads();
+        bool b2 = false;
+        build_tokens(p, idx, t0, n, M, codes, nullptr, &b2);
+        __syncthreads();
+        column_scan(p, M, n, tot);  // tot <- this chunk's column sums
+        __syncthreads();
+        place_tokens(p, t0, n, M, codes, base);
+        __syncthreads();
+        for (int i = tid; i < E + R; i += blockDim.x) base[i] += tot[i];
+        __syncthreads();
     }
 }
 
-size_t layout_smem_bytes(int nww, int E, int R, int S, int k, int csize)
-{
-    return sizeof(int32_t) * ((size_t)kScanInts + (size_t)nww * (E + R) +
-                              (size_t)csize * (E + R + 2) + 4 + (size_t)nww * S * k);
-}
+// ------------------------------------------------------------------- host
 
 int pow2_floor(int v)
 {
@@ -402,60 +386,51 @@ int pow2_floor(int v)
     return p;
 }
 
-int pow2_ceil(int v)
+int log2_exact(int v)
 {
-    int p = 1;
-    while (p < v) p *= 2;
-    return p;
+    int l = 0;
+    while ((1 << l) < v) ++l;
+    return l;
 }
 
 struct Geometry {
-    int csize, nww, tpc, tpw, S, tpe, per, tpr;
+    int csize, tpc, tch, wde, wdr, wds, nseg;
     size_t smem;
 };
 
-// Cluster size, walker warps, staging chunk and scan mapping for a layout
-// problem (1024 threads per CTA).
+size_t fixed_smem_ints(int E, int R, int csize)
+{
+    return (size_t)kScanInts + 2 * (size_t)(E + R) + (size_t)csize * (E + R + 2) + 2;
+}
+
+// Cluster size, chunking and column-scan mapping for a layout problem.
 Geometry plan(int T, int k, int E, int R, int csize)
 {
     Geometry g;
-    const int tps = 32 / k;
+    g.wde = (E + 1) / 2;
+    g.wdr = (R + 1) / 2;
+    g.wds = (g.wde + g.wdr) | 1;
+    // the exchange area grows with the cluster: shrink the cluster if the
+    // fixed part would crowd out the count matrix
+    while (csize > 1 && fixed_smem_ints(E, R, csize) * 4 + (size_t)(g.wds + 4 + k) * 4 * 16 >
+                            (size_t)kMaxDynSmem)
+        csize >>= 1;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    const int steps = (g.tpc + tps - 1) / tps;
-    // one ordered step per walker when possible (at most 32 walkers)
-    int nww = steps < 1 ? 1 : (steps > 32 ? 32 : steps);
-    for (;;) {
-        int tpw = (g.tpc + nww - 1) / nww;
-        tpw = ((tpw + tps - 1) / tps) * tps;
-        if (tpw < tps) tpw = tps;
-        const size_t base = layout_smem_bytes(nww, E, R, 0, k, csize);
-        const long long avail = (long long)kMaxDynSmem - (long long)base;
-        int S = avail > 0 ? (int)(avail / ((long long)nww * k * 4)) : 0;
-        S = (S / tps) * tps;
-        if (S > tpw) S = tpw;
-        if (S >= tps || nww == 1) {
-            g.nww = nww;
-            g.tpw = tpw;
-            g.S = S < tps ? tps : S;
-            g.smem = layout_smem_bytes(nww, E, R, g.S, k, csize);
-            break;
-        }
-        --nww;
-    }
-    const int wcap = pow2_ceil(g.nww);
-    if (E <= 1024) {
-        g.per = 1;
-        g.tpe = pow2_floor(1024 / E);
-        if (g.tpe > 32) g.tpe = 32;
-        if (g.tpe > wcap) g.tpe = wcap;
-    } else {
-        g.per = (E + 1023) / 1024;
-        g.tpe = 1;
-    }
-    g.tpr = pow2_floor(1024 / R);
-    if (g.tpr > 32) g.tpr = 32;
-    if (g.tpr > wcap) g.tpr = wcap;
+    const size_t fixed = fixed_smem_ints(E, R, csize) * 4;
+    const size_t per_tok = (size_t)(g.wds + k) * 4;
+    long long cap = ((long long)kMaxDynSmem - (long long)fixed - 16) / (long long)per_tok;
+    if (cap > 1024) cap = 1024;             // one token per thread
+    if (cap > 65535 / k) cap = 65535 / k;   // 16-bit column counts cannot overflow
+    if (cap < 1) cap = 1;
+    g.tch = g.tpc < cap ? (g.tpc < 1 ? 1 : g.tpc) : (int)cap;
+    const int wdt = g.wde + g.wdr;
+    int nseg = pow2_floor(1024 / (wdt < 1024 ? wdt : 1024));
+    if (nseg > 32) nseg = 32;
+    while (nseg > 1 && nseg / 2 >= g.tch) nseg >>= 1;  // no more segments than rows
+    g.nseg = nseg;
+    const size_t m_words = ((size_t)g.tch * g.wds + 3) & ~(size_t)3;
+    g.smem = (m_words + (size_t)g.tch * k) * 4 + fixed;  // fixed includes the scan scratch
     return g;
 }
 
@@ -528,13 +503,12 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
     while (g.csize > 1 && max_clusters<IdxT>(g.csize, g.smem, dev) == 0)
         g = plan(p.T, p.k, p.E, p.R, g.csize > 8 ? 8 : g.csize >> 1);
     p.tpc = g.tpc;
-    p.tpw = g.tpw;
-    p.S = g.S;
-    p.nww = g.nww;
-    p.tpe = g.tpe;
-    p.per = g.per;
-    p.tpr = g.tpr;
-    p.inv_epr = 1.0f / (float)p.epr;
+    p.tch = g.tch;
+    p.wde = g.wde;
+    p.wdr = g.wdr;
+    p.wds = g.wds;
+    p.nseg = g.nseg;
+    p.lg_nseg = log2_exact(g.nseg);
 
     if (g.csize == 1) {
         layout_kernel<IdxT, false><<<1, 1024, g.smem, s>>>(p);
