@@ -21,8 +21,7 @@ struct LayoutParams {
     int tch;        // tokens per chunk (rows of the count matrix)
     int wde, wdr;   // 32-bit words per count-matrix row for experts / ranks
     int wds;        // row stride in words (odd, so column walks avoid bank conflicts)
-    int nseg;       // threads per column in the column scan (power of two <= 32)
-    int lg_nseg;
+    int seg_words;  // words of the column-scan segment sums
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 

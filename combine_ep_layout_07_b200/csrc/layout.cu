@@ -142,74 +142,92 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
 }
 
 // Exclusive prefix of every column of M (n rows, wde + wdr packed columns)
-// over its rows.  With csum != nullptr the column sums go to csum[E + R]
-// (experts first, then ranks).
-__device__ void column_scan(const LayoutParams &p, uint32_t *M, int n, int32_t *csum)
+// over its rows.  Lanes take consecutive columns (conflict-free shared
+// memory), warps take row segments: pass 1 sums each segment, pass 2 turns
+// the segment into an exclusive prefix starting from the sum of the segments
+// above it.  seg has max(1024, wde + wdr) words.  The column sums go to
+// csum[E + R] (experts first, then ranks).
+__device__ void column_scan(const LayoutParams &p, uint32_t *M, int n, uint32_t *seg,
+                            int32_t *csum)
 {
     const int wdt = p.wde + p.wdr;
-    const int nseg = p.nseg;
-    const int s = threadIdx.x & (nseg - 1);
-    const int rps = (n + nseg - 1) >> p.lg_nseg;
-    const int ra = min(n, s * rps), rb = min(n, ra + rps);
-    const int cols_per_pass = blockDim.x >> p.lg_nseg;
-    for (int cbase = 0; cbase < wdt; cbase += cols_per_pass) {
-        const int c = cbase + (threadIdx.x >> p.lg_nseg);
-        const bool ok = c < wdt;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int ncb = (wdt + 31) >> 5;                     // 32-column blocks
+    const int nsg = ncb >= nwarps ? 1 : nwarps / ncb;    // row segments per block
+    const int rps = (n + nsg - 1) / nsg;
+    // pass 1: segment sums
+    for (int job = wid; job < ncb * nsg; job += nwarps) {
+        const int cb = job / nsg, sg = job - cb * nsg;
+        const int c = cb * 32 + lane;
+        const int ra = min(n, sg * rps), rb = min(n, ra + rps);
         uint32_t sum = 0;
-        if (ok)
+        if (c < wdt)
             for (int r = ra; r < rb; ++r) sum += M[(size_t)r * p.wds + c];
-        // exclusive scan of the packed sums across the column's segments
-        uint32_t inc = sum;
-        for (int o = 1; o < nseg; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(kFull, inc, o, nseg);
-            if (s >= o) inc += v;
+        if (c < wdt) seg[sg * wdt + c] = sum;
+    }
+    __syncthreads();
+    // pass 2: prefixes
+    for (int job = wid; job < ncb * nsg; job += nwarps) {
+        const int cb = job / nsg, sg = job - cb * nsg;
+        const int c = cb * 32 + lane;
+        if (c >= wdt) continue;
+        const int ra = min(n, sg * rps), rb = min(n, ra + rps);
+        uint32_t run = 0, total = 0;
+        for (int q = 0; q < nsg; ++q) {
+            const uint32_t v = seg[q * wdt + c];
+            run += q < sg ? v : 0u;
+            total += v;
         }
-        const uint32_t total = __shfl_sync(kFull, inc, nseg - 1, nseg);
-        if (ok) {
-            uint32_t run = inc - sum;
-            for (int r = ra; r < rb; ++r) {
-                const uint32_t v = M[(size_t)r * p.wds + c];
-                M[(size_t)r * p.wds + c] = run;
-                run += v;
-            }
-            if (csum && s == 0) {
-                const bool er = c < p.wde;
-                const int col0 = er ? 2 * c : 2 * (c - p.wde);
-                const int lim = er ? p.E : p.R;
-                int32_t *dst = er ? csum : csum + p.E;
-                dst[col0] = (int32_t)(total & 0xffffu);
-                if (col0 + 1 < lim) dst[col0 + 1] = (int32_t)(total >> 16);
-            }
+        for (int r = ra; r < rb; ++r) {
+            const uint32_t v = M[(size_t)r * p.wds + c];
+            M[(size_t)r * p.wds + c] = run;
+            run += v;
+        }
+        if (sg == 0) {
+            const bool er = c < p.wde;
+            const int col0 = er ? 2 * c : 2 * (c - p.wde);
+            const int lim = er ? p.E : p.R;
+            int32_t *dst = er ? csum : csum + p.E;
+            dst[col0] = (int32_t)(total & 0xffffu);
+            if (col0 + 1 < lim) dst[col0 + 1] = (int32_t)(total >> 16);
         }
     }
 }
 
-// Thread-per-token: write pos and recv_pos of tokens [t0, t0 + n) from the
-// scanned matrix, the route codes and the per-column bases.
+// Write pos and recv_pos of tokens [t0, t0 + n) from the scanned matrix,
+// the route codes, the chunk's column sums and the per-column bases; one
+// thread per route, then one per (token, rank), so stores are coalesced.
+__device__ __forceinline__ int div_small(int i, float inv)
+{
+    // floor(i / d) for i < 2^22 with inv = 1/d (same argument as rank_of)
+    return __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), inv));
+}
+
 __device__ void place_tokens(const LayoutParams &p, int t0, int n, const uint32_t *M,
-                             const int32_t *codes, const int32_t *base)
+                             const int32_t *codes, const int32_t *csum, const int32_t *base)
 {
     const int k = p.k, E = p.E, R = p.R;
-    for (int u = threadIdx.x; u < n; u += blockDim.x) {
-        const size_t t = (size_t)(t0 + u);
-        const uint32_t *mrow = M + (size_t)u * p.wds;
-        unsigned long long hit = 0ull;
-        for (int j = 0; j < k; ++j) {
-            const int c = codes[(size_t)u * k + j];
-            int v = -1;
-            if (c >= 0) {
-                const int e = code_e(c);
-                v = base[e] + (int)((mrow[e >> 1] >> ((e & 1) * 16)) & 0xffffu) + code_dup(c);
-                if (code_first(c)) hit |= 1ull << code_r(c);
-            }
-            p.pos[t * k + j] = v;
+    const float inv_k = 1.0f / (float)k, inv_r = 1.0f / (float)R;
+    for (int i = threadIdx.x; i < n * k; i += blockDim.x) {
+        const int u = div_small(i, inv_k);
+        const int c = codes[i];
+        int v = -1;
+        if (c >= 0) {
+            const int e = code_e(c);
+            v = base[e] + (int)((M[(size_t)u * p.wds + (e >> 1)] >> ((e & 1) * 16)) & 0xffffu) +
+                code_dup(c);
         }
-        for (int r = 0; r < R; ++r) {
-            int v = -1;
-            if ((hit >> r) & 1ull)
-                v = base[E + r] + (int)((mrow[p.wde + (r >> 1)] >> ((r & 1) * 16)) & 0xffffu);
-            p.recv_pos[t * R + r] = v;
-        }
+        p.pos[(size_t)t0 * k + i] = v;
+    }
+    for (int i = threadIdx.x; i < n * R; i += blockDim.x) {
+        const int u = div_small(i, inv_r);
+        const int r = i - u * R;
+        const int col = p.wde + (r >> 1), sh = (r & 1) * 16;
+        const int here = (int)((M[(size_t)u * p.wds + col] >> sh) & 0xffffu);
+        const int next = u + 1 < n ? (int)((M[(size_t)(u + 1) * p.wds + col] >> sh) & 0xffffu)
+                                   : csum[E + r];
+        p.recv_pos[(size_t)t0 * R + i] = next > here ? base[E + r] + here : -1;
     }
 }
 
@@ -244,7 +262,8 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     uint32_t *M = reinterpret_cast<uint32_t *>(smem + kScanInts);  // [tch][wds]
     const size_t m_words = ((size_t)p.tch * p.wds + 3) & ~(size_t)3;
     int32_t *codes = smem + kScanInts + m_words;   // [tch][k]
-    int32_t *tot = codes + (size_t)p.tch * p.k;    // [E + R] CTA totals / chunk sums
+    uint32_t *seg = reinterpret_cast<uint32_t *>(codes + (size_t)p.tch * p.k);  // column-scan sums
+    int32_t *tot = reinterpret_cast<int32_t *>(seg) + p.seg_words;  // [E + R] totals / chunk sums
     int32_t *base = tot + E + R;                   // [E + R] this CTA's row bases
     int32_t *all_tot = base + E + R;               // [csize][W]
     int32_t *misc = all_tot + csize * W;           // [2] bad flag, real tokens
@@ -262,7 +281,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         __syncthreads();
         nreal = build_tokens(p, idx, c0, nt, M, codes, nullptr, &bad);
         __syncthreads();
-        column_scan(p, M, nt, tot);
+        column_scan(p, M, nt, seg, tot);
     } else {
         for (int i = tid; i < E + R; i += blockDim.x) tot[i] = 0;
         __syncthreads();
@@ -357,7 +376,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
     // ---- positions
     if (nchunks <= 1) {
-        place_tokens(p, c0, nt, M, codes, base);
+        place_tokens(p, c0, nt, M, codes, tot, base);
         return;
     }
     for (int ch = 0; ch < nchunks; ++ch) {
@@ -368,9 +387,9 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         bool b2 = false;
         build_tokens(p, idx, t0, n, M, codes, nullptr, &b2);
         __syncthreads();
-        column_scan(p, M, n, tot);  // tot <- this chunk's column sums
+        column_scan(p, M, n, seg, tot);  // tot <- this chunk's column sums
         __syncthreads();
-        place_tokens(p, t0, n, M, codes, base);
+        place_tokens(p, t0, n, M, codes, tot, base);
         __syncthreads();
         for (int i = tid; i < E + R; i += blockDim.x) base[i] += tot[i];
         __syncthreads();
@@ -379,22 +398,8 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
 // ------------------------------------------------------------------- host
 
-int pow2_floor(int v)
-{
-    int p = 1;
-    while (p * 2 <= v) p *= 2;
-    return p;
-}
-
-int log2_exact(int v)
-{
-    int l = 0;
-    while ((1 << l) < v) ++l;
-    return l;
-}
-
 struct Geometry {
-    int csize, tpc, tch, wde, wdr, wds, nseg;
+    int csize, tpc, tch, wde, wdr, wds, seg_words;
     size_t smem;
 };
 
@@ -417,20 +422,17 @@ Geometry plan(int T, int k, int E, int R, int csize)
         csize >>= 1;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    const size_t fixed = fixed_smem_ints(E, R, csize) * 4;
+    const int wdt_all = g.wde + g.wdr;
+    const size_t fixed = (fixed_smem_ints(E, R, csize) + (wdt_all > 1024 ? wdt_all : 1024)) * 4;
     const size_t per_tok = (size_t)(g.wds + k) * 4;
     long long cap = ((long long)kMaxDynSmem - (long long)fixed - 16) / (long long)per_tok;
     if (cap > 1024) cap = 1024;             // one token per thread
     if (cap > 65535 / k) cap = 65535 / k;   // 16-bit column counts cannot overflow
     if (cap < 1) cap = 1;
     g.tch = g.tpc < cap ? (g.tpc < 1 ? 1 : g.tpc) : (int)cap;
-    const int wdt = g.wde + g.wdr;
-    int nseg = pow2_floor(1024 / (wdt < 1024 ? wdt : 1024));
-    if (nseg > 32) nseg = 32;
-    while (nseg > 1 && nseg / 2 >= g.tch) nseg >>= 1;  // no more segments than rows
-    g.nseg = nseg;
     const size_t m_words = ((size_t)g.tch * g.wds + 3) & ~(size_t)3;
-    g.smem = (m_words + (size_t)g.tch * k) * 4 + fixed;  // fixed includes the scan scratch
+    g.seg_words = wdt_all > 1024 ? wdt_all : 1024;
+    g.smem = (m_words + (size_t)g.tch * k) * 4 + fixed;  // fixed: scan scratch, seg sums, totals
     return g;
 }
 
@@ -507,8 +509,7 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
     p.wde = g.wde;
     p.wdr = g.wdr;
     p.wds = g.wds;
-    p.nseg = g.nseg;
-    p.lg_nseg = log2_exact(g.nseg);
+    p.seg_words = g.seg_words;
 
     if (g.csize == 1) {
         layout_kernel<IdxT, false><<<1, 1024, g.smem, s>>>(p);
