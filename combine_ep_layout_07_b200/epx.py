@@ -22,11 +22,13 @@ import torch
 __all__ = [
     "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
     "combine_reduce", "read_totals", "roundtrip_host", "roundtrip_device_bytes",
+    "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES",
     "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libepx.so")
 MAX_TOPK, MAX_RANKS, MAX_EXPERTS = 32, 64, 4096
+NOALLOC_SCRATCH_BYTES = 64 << 20  # EPX_NOALLOC_SCRATCH_BYTES
 
 EP_OK = 0
 _STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_MISALIGNED", 3: "EP_ERR_CAPACITY",
@@ -78,6 +80,7 @@ def lib():
                                    ctypes.POINTER(I64), ctypes.POINTER(I32), P], I32),
         "ep_roundtrip_device_bytes": ([I32, I32, I32, I32, I32, I32], SZ),
         "ep_roundtrip_host": ([P, P, P, I32, I32, I32, I32, I32, I32, P, SZ, P, P], I32),
+        "ep_roundtrip_host_noalloc": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -243,4 +246,23 @@ def roundtrip_host(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.T
     _check(lib().ep_roundtrip_host(x_host.data_ptr(), idx_host.data_ptr(), w_host.data_ptr(),
                                    T, H, k, E, R, bits, dev_mem.data_ptr(), dev_mem.numel(),
                                    out_host.data_ptr(), _stream(stream)), "ep_roundtrip_host")
+    return out_host
+
+
+def roundtrip_host_noalloc(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.Tensor,
+                           E: int, R: int, out_host: torch.Tensor, stream=None):
+    """ep_roundtrip_host_noalloc: like roundtrip_host, for callers that cannot
+    allocate device memory -- the device scratch is the library's fixed
+    NOALLOC_SCRATCH_BYTES array (asynchronous; calls that overlap on the GPU
+    race on that array)."""
+    T, H = x_host.shape
+    k = idx_host.shape[1]
+    bits = {torch.int64: 64, torch.int32: 32}[idx_host.dtype]
+    for t in (x_host, idx_host, w_host, out_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host buffers must be contiguous CPU tensors")
+    _check(lib().ep_roundtrip_host_noalloc(x_host.data_ptr(), idx_host.data_ptr(),
+                                           w_host.data_ptr(), T, H, k, E, R, bits,
+                                           out_host.data_ptr(), _stream(stream)),
+           "ep_roundtrip_host_noalloc")
     return out_host

@@ -208,6 +208,35 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
                               int32_t idx_bits, void *dev_mem, size_t bytes,
                               void *out_host, void *stream);
 
+/*
+ * Host round trip that allocates nothing.  The pages have no counterpart:
+ * this entry point serves callers that cannot allocate device memory when
+ * they need a pass -- code running while another component owns the device
+ * allocator (a caching allocator or a pool fixed at start-up), plugins
+ * loaded into a host that forbids allocation after initialisation, latency
+ * paths that cannot afford an allocation's implicit synchronisation.
+ *
+ * Same arguments and result as ep_roundtrip_host, minus dev_mem/bytes: the
+ * device scratch is a fixed array of EPX_NOALLOC_SCRATCH_BYTES inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Sizes whose ep_roundtrip_device_bytes(...) exceeds it return
+ * EP_ERR_UNSUPPORTED and launch nothing (64 MiB covers, for example,
+ * 128 tokens of hidden 7168 with top-8, or 8 tokens of hidden 3584 with
+ * top-16).  No cudaMalloc, cudaFree or other allocating call is made.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array and it keeps the
+ * last call's contents (nothing in it needs to start at zero); calls whose
+ * device work overlaps -- on different streams or from different host
+ * threads -- race on it, so order them on one stream or synchronise.
+ */
+#define EPX_NOALLOC_SCRATCH_BYTES (64u << 20)
+ep_status_t ep_roundtrip_host_noalloc(const void *x_host, const void *topk_idx_host,
+                                      const float *topk_weights_host, int32_t T,
+                                      int32_t H, int32_t k, int32_t E, int32_t R,
+                                      int32_t idx_bits, void *out_host, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
