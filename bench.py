@@ -455,13 +455,8 @@ def run_epx(args):
     k_ms = {"layout": [r[0] for r in rec],
             "dispatch_expand": [r[1] - r[0] for r in rec],
             "combine_reduce": [r[2] - r[1] for r in rec]}
-    total_ms = sum(step_ms)
-    if pg:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
-    units = tot["T_real"] * args.steps * world
-    value = units / (total_ms / 1e3)
+    total_ms = reduce_max(pg, sum(step_ms), dev)
+    value = whole_job_value(tot["T_real"] * args.steps, world, total_ms)
 
     # ---- e2e through the host-buffer C-ABI call
     e2e = None if args.no_e2e else run_e2e(torch, epx, wl, args, dev, stream, pg, world,
@@ -548,17 +543,28 @@ def run_e2e(torch, epx, wl, args, dev, stream, pg, world, T_real):
         epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem, out_h, stream=stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(pg, e0.elapsed_time(e1), dev)
     h2d = x_h.numel() * 2 + i_h.numel() * i_h.element_size() + w_h.numel() * 4
     d2h = out_h.numel() * 2
-    return {"value": T_real * n * world / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_value(T_real * n, world, ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n,
             "path": "ep_roundtrip_host: pinned host -> device, layout, dispatch/expand, "
                     "stand-in expert, combine, device -> host"}
+
+
+def reduce_max(pg, value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: units every rank processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
 
 
 def finish(pg):

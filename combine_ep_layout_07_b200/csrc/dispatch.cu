@@ -214,7 +214,9 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
             cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     }
     const int gy = p.T < 65535 ? p.T : 65535;
-    if (variant == 0) variant = 1;
+    // automatic: TMA bulk copies for large batches (measured faster at 4096
+    // rows of 14 KB), register copies for small ones (fewer fixed costs)
+    if (variant == 0) variant = p.T >= 1024 ? 2 : 1;
     if (variant == 2) {
         // chunks so that at least ~2 CTAs per SM exist; chunk <= 32 KB
         int chunks = (2 * nsm + p.T - 1) / p.T;
