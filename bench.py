@@ -125,9 +125,9 @@ def sources_hash(kernel):
     return h.hexdigest()[:16]
 
 
-def committed_traffic(kernel, workload):
+def committed_traffic(kernel, workload, engine=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source; otherwise None."""
+    on the current kernel source (and copy engine); otherwise None."""
     try:
         lines = open(TRAFFIC_FILE).read().splitlines()
     except OSError:
@@ -138,7 +138,7 @@ def committed_traffic(kernel, workload):
             continue
         kv = dict(x.split("=", 1) for x in ln.split() if "=" in x)
         if (kv.get("kernel") == kernel and kv.get("workload") == workload
-                and kv.get("source") == want):
+                and kv.get("source") == want and kv.get("engine") in (None, engine)):
             return float(kv["dram_bytes_per_launch"])
     return None
 
@@ -476,7 +476,10 @@ def run_epx(args):
         kernels[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
                          "alg_bytes": bytes_[name], "gbs": gbs, "frac": gbs / peak}
     dom = max(kernels, key=lambda n: kernels[n]["us"])
-    traffic = committed_traffic(dom, args.workload)
+    engine = {"dispatch_expand": "bulk" if args.dispatch_variant == 2 or
+              (args.dispatch_variant == 0 and T >= 1024) else "vec",
+              "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split"}
+    traffic = committed_traffic(dom, args.workload, engine.get(dom))
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind ==
