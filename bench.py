@@ -327,7 +327,10 @@ def workload_config(wl, args, lay_totals, flush_desc=None):
            "parallelism": f"replicas x{dist_env()[1]}"}
     if flush_desc:
         cfg["l2"] = flush_desc
-    cfg["launch"] = "eager" if getattr(args, "eager", True) else "cuda graph per step"
+    cfg["launch"] = ("eager, events between kernels" if getattr(args, "eager", True) else
+                     "one CUDA graph per step, kernels chained by programmatic dependent "
+                     "launch; per-kernel split from a second run of the same steps with "
+                     "events between kernels")
     return cfg
 
 
@@ -393,33 +396,45 @@ def run_epx(args):
     flush_desc = ("L2 flushed between steps (256 MiB write, outside the timed events)" if flush
                   else f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)")
 
-    graph = None
-    gev = None
+    graph = graph_k = None
+    gev = gks = None
     if not args.eager:
-        # one step captured as a CUDA graph with timing events inside it, so
-        # the three kernels run back to back with no host launch gaps
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        graph = torch.cuda.CUDAGraph()
+        # Two captured graphs of one step: `graph` has timing events only at
+        # its ends, so consecutive kernels overlap their launches
+        # (programmatic dependent launch); `graph_k` also has events between
+        # the kernels (which serialises them) for the per-kernel split.
         with torch.cuda.stream(stream):
             step_kernels()          # launchers set their function attributes here
         torch.cuda.synchronize(dev)
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
-            step_kernels(gev, st=torch.cuda.current_stream())
+            cs = torch.cuda.current_stream()
+            gev[0].record(cs)
+            step_kernels(st=cs)
+            gev[1].record(cs)
+        gks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        graph_k = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_k, stream=stream):
+            step_kernels(gks, st=torch.cuda.current_stream())
         torch.cuda.synchronize(dev)
 
-    def run_step(events_out=None):
+    def run_step(out=None, split=False):
         if flush:
             flush_buf.add_(1)
         if graph is not None:
-            graph.replay()
-            if events_out is not None:
+            (graph_k if split else graph).replay()
+            if out is not None:
                 torch.cuda.current_stream().synchronize()
-                events_out.append([gev[0].elapsed_time(gev[j]) for j in (1, 2, 3)])
+                if split:
+                    out.append([gks[0].elapsed_time(gks[j]) for j in (1, 2, 3)])
+                else:
+                    out.append(gev[0].elapsed_time(gev[1]))
         else:
-            if events_out is not None:
+            if out is not None:
                 ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
                 step_kernels(ev)
-                events_out.append(ev)
+                out.append(ev)
             else:
                 step_kernels()
 
@@ -427,6 +442,8 @@ def run_epx(args):
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             run_step()
+            if graph_k is not None:
+                run_step(split=True)
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
@@ -434,7 +451,7 @@ def run_epx(args):
     sampler = ClockSampler(gpu_uuid(torch, local)) if rank == 0 else None
     if sampler:
         sampler.start()
-    rec = []
+    rec, rec_k = [], []
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
@@ -446,15 +463,22 @@ def run_epx(args):
     t_hi = time.time()
     if pg:
         pg.barrier()
+    if graph_k is not None:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                run_step(rec_k, split=True)
+        torch.cuda.synchronize(dev)
     if sampler:
         sampler.stop()
 
     if graph is None:   # cumulative times from each step's first event
-        rec = [[e[0].elapsed_time(e[j]) for j in (1, 2, 3)] for e in rec]
-    step_ms = [r[2] for r in rec]
-    k_ms = {"layout": [r[0] for r in rec],
-            "dispatch_expand": [r[1] - r[0] for r in rec],
-            "combine_reduce": [r[2] - r[1] for r in rec]}
+        rec_k = [[e[0].elapsed_time(e[j]) for j in (1, 2, 3)] for e in rec]
+        step_ms = [r[2] for r in rec_k]
+    else:
+        step_ms = rec
+    k_ms = {"layout": [r[0] for r in rec_k],
+            "dispatch_expand": [r[1] - r[0] for r in rec_k],
+            "combine_reduce": [r[2] - r[1] for r in rec_k]}
     total_ms = reduce_max(pg, sum(step_ms), dev)
     value = whole_job_value(tot["T_real"] * args.steps, world, total_ms)
 
@@ -462,7 +486,7 @@ def run_epx(args):
     e2e = None if args.no_e2e else run_e2e(torch, epx, wl, args, dev, stream, pg, world,
                                            tot["T_real"])
     if graph is not None:
-        del graph
+        del graph, graph_k
 
     if rank != 0:
         finish(pg)

@@ -96,6 +96,8 @@ __global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
     __shared__ int s_pos[EPX_MAX_TOPK];
     __shared__ float s_w[EPX_MAX_TOPK];
     __shared__ int s_n;
+    pdl_launch_dependents();
+    pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
             int n = build_routes(p, t, s_pos, s_w);
@@ -117,6 +119,8 @@ __global__ void __launch_bounds__(128) combine_warp_per_token_kernel(CombinePara
     __shared__ int s_pos[4][EPX_MAX_TOPK];
     __shared__ float s_w[4][EPX_MAX_TOPK];
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_launch_dependents();
+    pdl_wait_previous();
     for (int t = blockIdx.x * 4 + wid; t < p.T; t += gridDim.x * 4) {
         const int n = build_routes(p, t, s_pos[wid], s_w[wid]);
         for (int v = lane; v < p.V; v += 32)
@@ -142,10 +146,8 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
         int blocks = (p.T + 3) / 4;
         if (blocks > 65535 * 16) blocks = 65535 * 16;
         if (big_k)
-            combine_warp_per_token_kernel<16><<<blocks, 128, 0, s>>>(p);
-        else
-            combine_warp_per_token_kernel<8><<<blocks, 128, 0, s>>>(p);
-        return cudaGetLastError();
+            return launch_pdl(combine_warp_per_token_kernel<16>, dim3(blocks), dim3(128), 0, s, p);
+        return launch_pdl(combine_warp_per_token_kernel<8>, dim3(blocks), dim3(128), 0, s, p);
     }
     // split: enough CTAs for ~4 per SM, at least 32 vectors per CTA
     int chunks = (4 * nsm + p.T - 1) / p.T;
@@ -157,10 +159,8 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     int threads = p.vpc < 128 ? ((p.vpc + 31) / 32) * 32 : 128;
     const int gy = p.T < 65535 ? p.T : 65535;
     if (big_k)
-        combine_split_kernel<16><<<dim3(chunks, gy), threads, 0, s>>>(p);
-    else
-        combine_split_kernel<8><<<dim3(chunks, gy), threads, 0, s>>>(p);
-    return cudaGetLastError();
+        return launch_pdl(combine_split_kernel<16>, dim3(chunks, gy), dim3(threads), 0, s, p);
+    return launch_pdl(combine_split_kernel<8>, dim3(chunks, gy), dim3(threads), 0, s, p);
 }
 
 }  // namespace epx

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
 {
     __shared__ uint4 *s_dst[kMaxDst];
     __shared__ int s_n;
+    pdl_launch_dependents();
+    pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
             int n = build_dst_list(p, t, s_dst);
@@ -174,8 +176,10 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
     __shared__ uint4 *s_dst[kMaxDst];
     __shared__ __align__(8) uint64_t bar;
     const int lane = threadIdx.x;
+    pdl_launch_dependents();
     if (lane == 0) mbar_init(&bar, 1);
     __syncwarp();
+    pdl_wait_previous();
     unsigned phase = 0;
     const int v0 = blockIdx.x * p.vpc;
     const int nv = min(p.V, v0 + p.vpc) - v0;
@@ -236,8 +240,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
             if (e != cudaSuccess) return e;
             attr_set_mask |= 1 << dev;
         }
-        dispatch_bulk_kernel<<<dim3(chunks, gy), 32, smem, s>>>(p);
-        return cudaGetLastError();
+        return launch_pdl(dispatch_bulk_kernel, dim3(chunks, gy), dim3(32), smem, s, p);
     }
     // vector engine: 128 threads x 2 vectors per pass
     int chunks = (4 * nsm + p.T - 1) / p.T;
@@ -246,8 +249,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
     if (chunks < 1) chunks = 1;
     p.vpc = (p.V + chunks - 1) / chunks;
     chunks = (p.V + p.vpc - 1) / p.vpc;
-    dispatch_vec_kernel<2, false><<<dim3(chunks, gy), 128, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_vec_kernel<2, false>, dim3(chunks, gy), dim3(128), 0, s, p);
 }
 
 }  // namespace epx

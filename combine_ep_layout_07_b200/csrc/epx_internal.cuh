@@ -18,10 +18,8 @@ struct LayoutParams {
     int T, k, E, R;
     float inv_epr;  // 1.0f / (E / R): rank of expert e = floor((e + 0.5) * inv_epr)
     int tpc;        // tokens per CTA of the cluster
-    int tch;        // tokens per chunk (rows of the count matrix)
-    int wde, wdr;   // 32-bit words per count-matrix row for experts / ranks
-    int wds;        // row stride in words (odd, so column walks avoid bank conflicts)
-    int seg_words;  // words of the column-scan segment sums
+    int tch;        // tokens per chunk: a multiple of 32, the count matrix's width
+    int wde, wdr;   // count-matrix rows (two 16-bit counts per 32-bit word) for experts / ranks
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 
@@ -72,7 +70,51 @@ cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;
 
+// Launch `kernel` on `s` with programmatic stream serialisation (the kernel
+// may begin while its predecessor in the stream finishes; it synchronises
+// with pdl_wait_previous) and, when cluster > 1, a 1-D cluster.
+template <typename Params>
+cudaError_t launch_pdl(void (*kernel)(Params), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, const Params &p, int cluster = 1)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // ----------------------------------------------------- device utilities
+
+// Programmatic dependent launch.  Every kernel of the path lets the next one
+// in its stream start launching right away (its prologue overlaps this
+// kernel), and waits for the previous one to finish -- with its memory
+// visible -- before it touches any global memory.  Without the launch
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait_previous()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 __device__ __forceinline__ unsigned lanemask_lt()
 {

@@ -10,29 +10,30 @@
 //
 // A route's row is off_e[e] + (routes to e from earlier tokens) + (earlier
 // slots of its own token with the same expert); a (token, rank) pair's row
-// is off_r[r] + (earlier tokens that reach r).  Both middle terms are column
-// prefix sums of a token x expert (and token x rank) count matrix, so they
-// are computed here without any ordering primitive:
+// is off_r[r] + (earlier tokens that reach r).  Both middle terms are prefix
+// sums over tokens of a (expert | rank) x token count matrix, so they are
+// computed here without any ordering primitive:
 //  * one launch of one CTA, or of one thread-block cluster of up to 16 CTAs
 //    of 1024 threads; CTA c owns a contiguous range of tokens;
 //  * build: one thread per token loads its k indices, validates them,
 //    computes each route's rank, marks the first route of every
-//    (token, rank) pair and counts the token's row of the count matrix in
-//    shared memory -- counts are packed two 16-bit columns per 32-bit word,
-//    and the count seen before incrementing is the route's rank among equal
-//    experts of its own token;
-//  * column scan: every column of the matrix is prefix-summed over the
-//    tokens, several threads per column combined with warp shuffles (packed
-//    16-bit halves add independently); the column sums are the CTA totals;
+//    (token, rank) pair and counts its column of the matrix in shared
+//    memory -- counts are packed two 16-bit rows per 32-bit word, and the
+//    count seen before incrementing is the route's rank among equal experts
+//    of its own token;
+//  * row scan: each warp takes whole matrix rows and scans them 32 tokens at
+//    a time with shuffles (packed 16-bit halves add independently), carrying
+//    the running sum; the carry at the end is the CTA total of the row;
 //  * cluster exchange: each CTA pushes its totals into every peer's shared
 //    memory (distributed shared memory stores); after one cluster barrier
 //    every CTA reads them locally; a single CTA skips this;
-//  * global scan: one block-wide scan of packed 64-bit (expert, rank) counts
-//    gives both exclusive scans at once, plus this CTA's base;
-//  * positions: one thread per token again, reading its prefixes back.
+//  * global scan: one warp scans the experts, another the ranks, giving the
+//    exclusive offsets and this CTA's base per expert / rank;
+//  * placement: one thread per route, then one per (token, rank), so the
+//    stores of pos / recv_pos are coalesced.
 // When a CTA's tokens do not fit in shared memory at once, it counts all of
 // them first (atomics into its totals) and then builds, scans and places the
-// tokens chunk by chunk with a running cursor per column.
+// tokens chunk by chunk with a running base per row.
 #include <cooperative_groups.h>
 
 #include "epx_internal.cuh"
@@ -42,46 +43,10 @@ namespace cg = cooperative_groups;
 namespace epx {
 namespace {
 
-constexpr int kScanInts = 2 * 34;  // 64-bit block-scan scratch
-constexpr int kMaxPer = EPX_MAX_EXPERTS / 1024;
-
 // route code in shared memory: -1 = no route (or a dropped bad index), else
-// expert | rank << 12 | (rank among equal experts of the token) << 18 |
-// (first route of its rank) << 23
+// expert | (rank among equal experts of the token) << 12
 __device__ __forceinline__ int code_e(int c) { return c & 0xfff; }
-__device__ __forceinline__ int code_r(int c) { return (c >> 12) & 0x3f; }
-__device__ __forceinline__ int code_dup(int c) { return (c >> 18) & 0x1f; }
-__device__ __forceinline__ bool code_first(int c) { return (c >> 23) & 1; }
-
-__device__ unsigned long long block_exclusive_scan64(unsigned long long v,
-                                                     unsigned long long *sm,
-                                                     unsigned long long *total)
-{
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int nw = (blockDim.x + 31) >> 5;
-    unsigned long long inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long n = __shfl_up_sync(kFull, inc, o);
-        if (lane >= o) inc += n;
-    }
-    if (lane == 31) sm[wid] = inc;
-    __syncthreads();
-    if (wid == 0) {
-        const unsigned long long s = lane < nw ? sm[lane] : 0ull;
-        unsigned long long si = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long n = __shfl_up_sync(kFull, si, o);
-            if (lane >= o) si += n;
-        }
-        if (lane < nw) sm[lane] = si - s;
-        if (lane == 31) sm[32] = si;
-    }
-    __syncthreads();
-    *total = sm[32];
-    return sm[wid] + inc - v;
-}
+__device__ __forceinline__ int code_dup(int c) { return (c >> 12) & 0x1f; }
 
 __device__ __forceinline__ int rank_of(int e, float inv_epr)
 {
@@ -90,20 +55,37 @@ __device__ __forceinline__ int rank_of(int e, float inv_epr)
     return __float2int_rd(__fmul_rn(__fadd_rn((float)e, 0.5f), inv_epr));
 }
 
-// Thread-per-token pass over tokens [t0, t0 + n).  With M != nullptr it
-// builds the count-matrix rows (zeroed beforehand) and the route codes; with
-// tot != nullptr it counts into the CTA totals with atomics instead.  Returns
-// the number of this thread's tokens with a valid route; *bad is set if an
-// index < -1 or >= E was seen.
+__device__ __forceinline__ int div_small(int i, float inv)
+{
+    // floor(i / d) for 0 <= i < 2^22 with inv = 1/d (same argument as rank_of)
+    return __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), inv));
+}
+
+__device__ __forceinline__ uint32_t half16(uint32_t w, int sh) { return (w >> sh) & 0xffffu; }
+
+struct Smem {
+    uint32_t *M;              // [wde + wdr][tch + 1] counts, then in-chunk prefixes
+    int32_t *codes;           // [tch][k]
+    unsigned long long *hit;  // [tch] ranks each token reaches
+    int32_t *tot;             // [E + R] CTA totals / chunk sums
+    int32_t *base;            // [E + R] this CTA's first row per expert / rank
+    int32_t *all_tot;         // [csize][E + R + 2] published totals (+ bad flag, real tokens)
+    int32_t *misc;            // [2] bad flag, real tokens
+};
+
+// Thread-per-token pass over tokens [t0, t0 + n).  With count_only it adds
+// each route into the CTA totals with atomics; otherwise it counts the
+// token's matrix column (zeroed beforehand) and records codes and rank masks.
+// Returns this thread's number of tokens with a valid route; *bad is set if
+// an index < -1 or >= E was seen.
 template <typename IdxT>
 __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx, int t0, int n,
-                            uint32_t *M, int32_t *codes, int32_t *tot, bool *bad)
+                            const Smem &sm, bool count_only, bool *bad)
 {
-    const int k = p.k, E = p.E;
+    const int k = p.k, E = p.E, ld = p.tch + 1;
     int nreal = 0;
     for (int u = threadIdx.x; u < n; u += blockDim.x) {
         const IdxT *row = idx + (size_t)(t0 + u) * k;
-        uint32_t *mrow = M ? M + (size_t)u * p.wds : nullptr;
         unsigned long long mask = 0ull;
         for (int j0 = 0; j0 < k; j0 += 8) {
             long long ev[8];
@@ -121,101 +103,108 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
                     const int r = rank_of(ei, p.inv_epr);
                     const bool first = !((mask >> r) & 1ull);
                     mask |= 1ull << r;
-                    if (mrow) {
-                        const int sh = (ei & 1) * 16;
-                        const uint32_t w = mrow[ei >> 1];
-                        const int dup = (int)((w >> sh) & 0xffffu);
-                        mrow[ei >> 1] = w + (1u << sh);
-                        if (first) mrow[p.wde + (r >> 1)] += 1u << ((r & 1) * 16);
-                        code = ei | (r << 12) | (dup << 18) | ((int)first << 23);
+                    if (count_only) {
+                        atomicAdd(&sm.tot[ei], 1);
+                        if (first) atomicAdd(&sm.tot[E + r], 1);
                     } else {
-                        atomicAdd(&tot[ei], 1);
-                        if (first) atomicAdd(&tot[E + r], 1);
+                        const int sh = (ei & 1) * 16;
+                        uint32_t *cell = sm.M + (size_t)(ei >> 1) * ld + u;
+                        const uint32_t w = *cell;
+                        *cell = w + (1u << sh);
+                        if (first) sm.M[(size_t)(p.wde + (r >> 1)) * ld + u] += 1u << ((r & 1) * 16);
+                        code = ei | ((int)half16(w, sh) << 12);
                     }
                 }
-                if (codes) codes[(size_t)u * k + j] = code;
+                if (!count_only) sm.codes[(size_t)u * k + j] = code;
             }
         }
+        if (!count_only) sm.hit[u] = mask;
         nreal += mask != 0ull;
     }
     return nreal;
 }
 
-// Exclusive prefix of every column of M (n rows, wde + wdr packed columns)
-// over its rows.  Lanes take consecutive columns (conflict-free shared
-// memory), warps take row segments: pass 1 sums each segment, pass 2 turns
-// the segment into an exclusive prefix starting from the sum of the segments
-// above it.  seg has max(1024, wde + wdr) words.  The column sums go to
-// csum[E + R] (experts first, then ranks).
-__device__ void column_scan(const LayoutParams &p, uint32_t *M, int n, uint32_t *seg,
-                            int32_t *csum)
+// Exclusive prefix over the n tokens of every matrix row; warps take whole
+// rows, lanes 32 consecutive tokens at a time (conflict-free), carrying the
+// running sum.  The row totals, unpacked, go to tot[E + R].
+__device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
 {
-    const int wdt = p.wde + p.wdr;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    const int ncb = (wdt + 31) >> 5;                     // 32-column blocks
-    const int nsg = ncb >= nwarps ? 1 : nwarps / ncb;    // row segments per block
-    const int rps = (n + nsg - 1) / nsg;
-    // pass 1: segment sums
-    for (int job = wid; job < ncb * nsg; job += nwarps) {
-        const int cb = job / nsg, sg = job - cb * nsg;
-        const int c = cb * 32 + lane;
-        const int ra = min(n, sg * rps), rb = min(n, ra + rps);
-        uint32_t sum = 0;
-        if (c < wdt)
-            for (int r = ra; r < rb; ++r) sum += M[(size_t)r * p.wds + c];
-        if (c < wdt) seg[sg * wdt + c] = sum;
-    }
-    __syncthreads();
-    // pass 2: prefixes
-    for (int job = wid; job < ncb * nsg; job += nwarps) {
-        const int cb = job / nsg, sg = job - cb * nsg;
-        const int c = cb * 32 + lane;
-        if (c >= wdt) continue;
-        const int ra = min(n, sg * rps), rb = min(n, ra + rps);
-        uint32_t run = 0, total = 0;
-        for (int q = 0; q < nsg; ++q) {
-            const uint32_t v = seg[q * wdt + c];
-            run += q < sg ? v : 0u;
-            total += v;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int wdt = p.wde + p.wdr, ld = p.tch + 1;
+    for (int w = wid; w < wdt; w += nwarps) {
+        uint32_t *row = sm.M + (size_t)w * ld;
+        uint32_t carry = 0;
+        for (int s = 0; s < n; s += 32) {
+            const uint32_t v = s + lane < n ? row[s + lane] : 0u;
+            uint32_t inc = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t t = __shfl_up_sync(kFull, inc, o);
+                if (lane >= o) inc += t;
+            }
+            if (s + lane < n) row[s + lane] = carry + inc - v;
+            carry += __shfl_sync(kFull, inc, 31);
         }
-        for (int r = ra; r < rb; ++r) {
-            const uint32_t v = M[(size_t)r * p.wds + c];
-            M[(size_t)r * p.wds + c] = run;
-            run += v;
-        }
-        if (sg == 0) {
-            const bool er = c < p.wde;
-            const int col0 = er ? 2 * c : 2 * (c - p.wde);
+        if (lane == 0) {
+            const bool er = w < p.wde;
+            const int c0 = er ? 2 * w : 2 * (w - p.wde);
             const int lim = er ? p.E : p.R;
-            int32_t *dst = er ? csum : csum + p.E;
-            dst[col0] = (int32_t)(total & 0xffffu);
-            if (col0 + 1 < lim) dst[col0 + 1] = (int32_t)(total >> 16);
+            int32_t *dst = er ? sm.tot : sm.tot + p.E;
+            dst[c0] = (int32_t)(carry & 0xffffu);
+            if (c0 + 1 < lim) dst[c0 + 1] = (int32_t)(carry >> 16);
         }
     }
 }
 
-// Write pos and recv_pos of tokens [t0, t0 + n) from the scanned matrix,
-// the route codes, the chunk's column sums and the per-column bases; one
-// thread per route, then one per (token, rank), so stores are coalesced.
-__device__ __forceinline__ int div_small(int i, float inv)
+// One warp: exclusive scan of `count` columns of the published totals
+// (column c of CTA q at all_tot[q * W + first + c]); writes this CTA's base
+// per column and (CTA 0) the global counts and offsets.  Returns the total.
+__device__ int warp_global_scan(const Smem &sm, int W, int first, int count, int csize,
+                                int crank, int32_t *base, int32_t *cnt, int32_t *off)
 {
-    // floor(i / d) for i < 2^22 with inv = 1/d (same argument as rank_of)
-    return __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), inv));
+    const int lane = threadIdx.x & 31;
+    const int per = (count + 31) >> 5;
+    const int a = min(count, lane * per), b = min(count, a + per);
+    int mine = 0;
+    for (int c = a; c < b; ++c)
+        for (int q = 0; q < csize; ++q) mine += sm.all_tot[q * W + first + c];
+    int inc = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += t;
+    }
+    int run = inc - mine;
+    for (int c = a; c < b; ++c) {
+        int glob = 0, cb = 0;
+        for (int q = 0; q < csize; ++q) {
+            const int v = sm.all_tot[q * W + first + c];
+            cb += q < crank ? v : 0;
+            glob += v;
+        }
+        base[c] = run + cb;
+        if (crank == 0) {
+            cnt[c] = glob;
+            off[c] = run;
+        }
+        run += glob;
+    }
+    return __shfl_sync(kFull, inc, 31);
 }
 
-__device__ void place_tokens(const LayoutParams &p, int t0, int n, const uint32_t *M,
-                             const int32_t *codes, const int32_t *csum, const int32_t *base)
+// pos / recv_pos of tokens [t0, t0 + n): one thread per route, then one per
+// (token, rank); stores are coalesced.
+__device__ void place_tokens(const LayoutParams &p, const Smem &sm, int t0, int n)
 {
-    const int k = p.k, E = p.E, R = p.R;
+    const int k = p.k, E = p.E, R = p.R, ld = p.tch + 1;
     const float inv_k = 1.0f / (float)k, inv_r = 1.0f / (float)R;
     for (int i = threadIdx.x; i < n * k; i += blockDim.x) {
         const int u = div_small(i, inv_k);
-        const int c = codes[i];
+        const int c = sm.codes[i];
         int v = -1;
         if (c >= 0) {
             const int e = code_e(c);
-            v = base[e] + (int)((M[(size_t)u * p.wds + (e >> 1)] >> ((e & 1) * 16)) & 0xffffu) +
+            v = sm.base[e] + (int)half16(sm.M[(size_t)(e >> 1) * ld + u], (e & 1) * 16) +
                 code_dup(c);
         }
         p.pos[(size_t)t0 * k + i] = v;
@@ -223,11 +212,11 @@ __device__ void place_tokens(const LayoutParams &p, int t0, int n, const uint32_
     for (int i = threadIdx.x; i < n * R; i += blockDim.x) {
         const int u = div_small(i, inv_r);
         const int r = i - u * R;
-        const int col = p.wde + (r >> 1), sh = (r & 1) * 16;
-        const int here = (int)((M[(size_t)u * p.wds + col] >> sh) & 0xffffu);
-        const int next = u + 1 < n ? (int)((M[(size_t)(u + 1) * p.wds + col] >> sh) & 0xffffu)
-                                   : csum[E + r];
-        p.recv_pos[(size_t)t0 * R + i] = next > here ? base[E + r] + here : -1;
+        int v = -1;
+        if ((sm.hit[u] >> r) & 1ull)
+            v = sm.base[E + r] +
+                (int)half16(sm.M[(size_t)(p.wde + (r >> 1)) * ld + u], (r & 1) * 16);
+        p.recv_pos[(size_t)t0 * R + i] = v;
     }
 }
 
@@ -240,12 +229,18 @@ __device__ void zero_words(uint32_t *a, int n)
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) a[i] = 0u;
 }
 
+__host__ __device__ size_t matrix_words(int wdt, int tch)
+{
+    return ((size_t)wdt * (tch + 1) + 3) & ~(size_t)3;
+}
+
 template <typename IdxT, bool CLUSTER>
 __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 {
     extern __shared__ __align__(16) int32_t smem[];
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, wid = tid >> 5;
     const int E = p.E, R = p.R, T = p.T;
+    pdl_launch_dependents();
 
     int crank = 0, csize = 1;
     if (CLUSTER) {
@@ -257,16 +252,16 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     }
 
-    const int W = E + R + 2;  // one CTA's published totals: experts, ranks, bad, real
-    unsigned long long *scan = reinterpret_cast<unsigned long long *>(smem);
-    uint32_t *M = reinterpret_cast<uint32_t *>(smem + kScanInts);  // [tch][wds]
-    const size_t m_words = ((size_t)p.tch * p.wds + 3) & ~(size_t)3;
-    int32_t *codes = smem + kScanInts + m_words;   // [tch][k]
-    uint32_t *seg = reinterpret_cast<uint32_t *>(codes + (size_t)p.tch * p.k);  // column-scan sums
-    int32_t *tot = reinterpret_cast<int32_t *>(seg) + p.seg_words;  // [E + R] totals / chunk sums
-    int32_t *base = tot + E + R;                   // [E + R] this CTA's row bases
-    int32_t *all_tot = base + E + R;               // [csize][W]
-    int32_t *misc = all_tot + csize * W;           // [2] bad flag, real tokens
+    const int W = E + R + 2;
+    const int wdt = p.wde + p.wdr;
+    Smem sm;
+    sm.M = reinterpret_cast<uint32_t *>(smem);
+    sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.tch));
+    sm.codes = reinterpret_cast<int32_t *>(sm.hit + p.tch);
+    sm.tot = sm.codes + (size_t)p.tch * p.k;
+    sm.base = sm.tot + E + R;
+    sm.all_tot = sm.base + E + R;
+    sm.misc = sm.all_tot + csize * W;
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
     const int c0 = min(T, crank * p.tpc);
@@ -275,123 +270,84 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     bool bad = false;
     int nreal = 0;
 
-    if (tid < 2) misc[tid] = 0;
+    // prologue in shared memory only, so it may overlap the previous kernel
+    if (tid < 2) sm.misc[tid] = 0;
     if (nchunks <= 1) {
-        zero_words(M, p.tch * p.wds);
-        __syncthreads();
-        nreal = build_tokens(p, idx, c0, nt, M, codes, nullptr, &bad);
-        __syncthreads();
-        column_scan(p, M, nt, seg, tot);
+        zero_words(sm.M, wdt * (p.tch + 1));
     } else {
-        for (int i = tid; i < E + R; i += blockDim.x) tot[i] = 0;
-        __syncthreads();
-        nreal = build_tokens(p, idx, c0, nt, nullptr, nullptr, tot, &bad);
+        for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
     }
-    if (__any_sync(kFull, bad) && (tid & 31) == 0) atomicOr(&misc[0], 1);
-    if (nreal) atomicAdd(&misc[1], nreal);
+    __syncthreads();
+    pdl_wait_previous();
+
+    if (nchunks <= 1) {
+        nreal = build_tokens(p, idx, c0, nt, sm, false, &bad);
+        __syncthreads();
+        row_scan(p, sm, nt);
+    } else {
+        nreal = build_tokens(p, idx, c0, nt, sm, true, &bad);
+    }
+    if (__any_sync(kFull, bad) && (tid & 31) == 0) atomicOr(&sm.misc[0], 1);
+    if (nreal) atomicAdd(&sm.misc[1], nreal);
     __syncthreads();
 
     // ---- publish this CTA's totals (to every CTA of the cluster)
     if (CLUSTER) {
         cg::cluster_group cluster = cg::this_cluster();
         asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-        for (int i = tid; i < E + R + 2; i += blockDim.x) {
-            const int v = i < E + R ? tot[i] : misc[i - E - R];
-            for (int c = 0; c < csize; ++c) cluster.map_shared_rank(all_tot, c)[crank * W + i] = v;
+        for (int i = tid; i < W; i += blockDim.x) {
+            const int v = i < E + R ? sm.tot[i] : sm.misc[i - E - R];
+            for (int c = 0; c < csize; ++c) cluster.map_shared_rank(sm.all_tot, c)[crank * W + i] = v;
         }
         cluster.sync();
     } else {
-        for (int i = tid; i < E + R + 2; i += blockDim.x)
-            all_tot[i] = i < E + R ? tot[i] : misc[i - E - R];
+        for (int i = tid; i < W; i += blockDim.x)
+            sm.all_tot[i] = i < E + R ? sm.tot[i] : sm.misc[i - E - R];
         __syncthreads();
     }
 
-    // ---- global exclusive scans (one packed 64-bit block scan) and bases
-    {
-        const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
-        int glob[kMaxPer], cbase[kMaxPer];
-        unsigned int contrib_e = 0;
-#pragma unroll
-        for (int q = 0; q < kMaxPer; ++q) {
-            glob[q] = 0;
-            cbase[q] = 0;
-            const int e = tid * per + q;
-            if (q < per && e < E) {
-                for (int c = 0; c < csize; ++c) {
-                    const int v = all_tot[c * W + e];
-                    cbase[q] += c < crank ? v : 0;
-                    glob[q] += v;
-                }
-                contrib_e += glob[q];
-            }
-        }
-        int glob_r = 0, cbase_r = 0;
-        if (tid < R)
-            for (int c = 0; c < csize; ++c) {
-                const int v = all_tot[c * W + E + tid];
-                cbase_r += c < crank ? v : 0;
-                glob_r += v;
-            }
-        const unsigned long long v = ((unsigned long long)contrib_e << 32) | (unsigned)glob_r;
-        unsigned long long total;
-        const unsigned long long ex = block_exclusive_scan64(v, scan, &total);
-        unsigned int run = (unsigned int)(ex >> 32);
-#pragma unroll
-        for (int q = 0; q < kMaxPer; ++q) {
-            const int e = tid * per + q;
-            if (q < per && e < E) {
-                base[e] = (int)run + cbase[q];
-                if (crank == 0) {
-                    p.cnt_e[e] = glob[q];
-                    p.off_e[e] = (int)run;
-                }
-                run += glob[q];
-            }
-        }
-        if (tid < R) {
-            const int off_r = (int)(unsigned int)(ex & 0xffffffffull);
-            base[E + tid] = off_r + cbase_r;
-            if (crank == 0) {
-                p.cnt_r[tid] = glob_r;
-                p.off_r[tid] = off_r;
-            }
-        }
-        if (tid == 0 && crank == 0) {
-            int errc = 0, nr = 0;
-            for (int c = 0; c < csize; ++c) {
-                errc |= all_tot[c * W + E + R];
-                nr += all_tot[c * W + E + R + 1];
-            }
-            const int n_route = (int)(total >> 32);
-            const int n_recv = (int)(total & 0xffffffffull);
+    // ---- global scans: warp 0 experts, warp 1 ranks, warp 2 the flags
+    if (wid == 0) {
+        const int n_route = warp_global_scan(sm, W, 0, E, csize, crank, sm.base, p.cnt_e, p.off_e);
+        if (crank == 0 && tid == 0) {
             p.off_e[E] = n_route;
-            p.off_r[R] = n_recv;
             p.totals[0] = n_route;
-            p.totals[1] = n_recv;
-            p.totals[2] = nr;
-            p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
         }
+    } else if (wid == 1) {
+        const int n_recv = warp_global_scan(sm, W, E, R, csize, crank, sm.base + E, p.cnt_r, p.off_r);
+        if (crank == 0 && (tid & 31) == 0) {
+            p.off_r[R] = n_recv;
+            p.totals[1] = n_recv;
+        }
+    } else if (wid == 2 && (tid & 31) == 0 && crank == 0) {
+        int errc = 0, nr = 0;
+        for (int c = 0; c < csize; ++c) {
+            errc |= sm.all_tot[c * W + E + R];
+            nr += sm.all_tot[c * W + E + R + 1];
+        }
+        p.totals[2] = nr;
+        p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
     }
     __syncthreads();
 
     // ---- positions
     if (nchunks <= 1) {
-        place_tokens(p, c0, nt, M, codes, tot, base);
+        place_tokens(p, sm, c0, nt);
         return;
     }
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = c0 + ch * p.tch;
         const int n = min(p.tch, c0 + nt - t0);
-        zero_words(M, p.tch * p.wds);
+        zero_words(sm.M, wdt * (p.tch + 1));
         __syncthreads();
         bool b2 = false;
-        build_tokens(p, idx, t0, n, M, codes, nullptr, &b2);
+        build_tokens(p, idx, t0, n, sm, false, &b2);
         __syncthreads();
-        column_scan(p, M, n, seg, tot);  // tot <- this chunk's column sums
+        row_scan(p, sm, n);  // tot <- this chunk's row sums
         __syncthreads();
-        place_tokens(p, t0, n, M, codes, tot, base);
+        place_tokens(p, sm, t0, n);
         __syncthreads();
-        for (int i = tid; i < E + R; i += blockDim.x) base[i] += tot[i];
+        for (int i = tid; i < E + R; i += blockDim.x) sm.base[i] += sm.tot[i];
         __syncthreads();
     }
 }
@@ -399,40 +355,41 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 // ------------------------------------------------------------------- host
 
 struct Geometry {
-    int csize, tpc, tch, wde, wdr, wds, seg_words;
+    int csize, tpc, tch, wde, wdr;
     size_t smem;
 };
 
-size_t fixed_smem_ints(int E, int R, int csize)
+size_t fixed_bytes(int E, int R, int csize)
 {
-    return (size_t)kScanInts + 2 * (size_t)(E + R) + (size_t)csize * (E + R + 2) + 2;
+    return sizeof(int32_t) * (2 * (size_t)(E + R) + (size_t)csize * (E + R + 2) + 2) + 16;
 }
 
-// Cluster size, chunking and column-scan mapping for a layout problem.
+// Cluster size and chunk width for a layout problem.
 Geometry plan(int T, int k, int E, int R, int csize)
 {
     Geometry g;
     g.wde = (E + 1) / 2;
     g.wdr = (R + 1) / 2;
-    g.wds = (g.wde + g.wdr) | 1;
+    const int wdt = g.wde + g.wdr;
+    // bytes per token of chunk width: a matrix column, its codes, its rank mask
+    const size_t per_tok = (size_t)wdt * 4 + (size_t)k * 4 + 8;
     // the exchange area grows with the cluster: shrink the cluster if the
-    // fixed part would crowd out the count matrix
-    while (csize > 1 && fixed_smem_ints(E, R, csize) * 4 + (size_t)(g.wds + 4 + k) * 4 * 16 >
+    // fixed part would leave room for fewer than 64 tokens per chunk
+    while (csize > 1 && fixed_bytes(E, R, csize) + (size_t)wdt * 4 + 64 * per_tok + 32 >
                             (size_t)kMaxDynSmem)
         csize >>= 1;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    const int wdt_all = g.wde + g.wdr;
-    const size_t fixed = (fixed_smem_ints(E, R, csize) + (wdt_all > 1024 ? wdt_all : 1024)) * 4;
-    const size_t per_tok = (size_t)(g.wds + k) * 4;
-    long long cap = ((long long)kMaxDynSmem - (long long)fixed - 16) / (long long)per_tok;
-    if (cap > 1024) cap = 1024;             // one token per thread
-    if (cap > 65535 / k) cap = 65535 / k;   // 16-bit column counts cannot overflow
+    long long cap = ((long long)kMaxDynSmem - (long long)fixed_bytes(E, R, csize) -
+                     (long long)wdt * 4 - 32) / (long long)per_tok;
+    if (cap > 1024) cap = 1024;            // one token per thread
+    if (cap > 65535 / k) cap = 65535 / k;  // 16-bit counts cannot overflow
+    if (cap >= 32) cap &= ~31LL;           // whole warps of tokens when there is room
     if (cap < 1) cap = 1;
-    g.tch = g.tpc < cap ? (g.tpc < 1 ? 1 : g.tpc) : (int)cap;
-    const size_t m_words = ((size_t)g.tch * g.wds + 3) & ~(size_t)3;
-    g.seg_words = wdt_all > 1024 ? wdt_all : 1024;
-    g.smem = (m_words + (size_t)g.tch * k) * 4 + fixed;  // fixed: scan scratch, seg sums, totals
+    const int want = ((g.tpc < 1 ? 1 : g.tpc) + 31) & ~31;
+    g.tch = want < cap ? want : (int)cap;
+    g.smem = matrix_words(wdt, g.tch) * 4 + (size_t)g.tch * 8 + (size_t)g.tch * k * 4 +
+             fixed_bytes(E, R, csize);
     return g;
 }
 
@@ -508,26 +465,10 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
     p.tch = g.tch;
     p.wde = g.wde;
     p.wdr = g.wdr;
-    p.wds = g.wds;
-    p.seg_words = g.seg_words;
-
-    if (g.csize == 1) {
-        layout_kernel<IdxT, false><<<1, 1024, g.smem, s>>>(p);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(g.csize, 1, 1);
-    cfg.blockDim = dim3(1024, 1, 1);
-    cfg.dynamicSmemBytes = g.smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = g.csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, layout_kernel<IdxT, true>, p);
+    if (g.csize == 1)
+        return launch_pdl(layout_kernel<IdxT, false>, dim3(1), dim3(1024), g.smem, s, p);
+    return launch_pdl(layout_kernel<IdxT, true>, dim3(g.csize), dim3(1024), g.smem, s, p,
+                      g.csize);
 }
 
 }  // namespace

@@ -28,6 +28,8 @@ __device__ __forceinline__ int expert_of_row(const int32_t *off_e, int E, int p)
 
 __global__ void __launch_bounds__(128) standin_kernel(StandinParams p)
 {
+    pdl_launch_dependents();
+    pdl_wait_previous();
     const int64_t n_route = p.totals[0];
     const int64_t rows = n_route < p.rows ? n_route : p.rows;
     for (int64_t row = blockIdx.y; row < rows; row += gridDim.y) {
@@ -60,8 +62,7 @@ cudaError_t launch_standin(const StandinParams &p0, cudaStream_t s)
     const int chunks = (p.V + 255) / 256;
     p.vpc = (p.V + chunks - 1) / chunks;
     const int64_t gy = p.rows < 65535 ? p.rows : 65535;
-    standin_kernel<<<dim3(chunks, (unsigned)gy), 128, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(standin_kernel, dim3(chunks, (unsigned)gy), dim3(128), 0, s, p);
 }
 
 }  // namespace epx
