@@ -24,11 +24,13 @@
 //  * row scan: each warp takes whole matrix rows and scans them 32 tokens at
 //    a time with shuffles (packed 16-bit halves add independently), carrying
 //    the running sum; the carry at the end is the CTA total of the row;
-//  * cluster exchange: each CTA pushes its totals into every peer's shared
-//    memory (distributed shared memory stores); after one cluster barrier
-//    every CTA reads them locally; a single CTA skips this;
-//  * global scan: one warp scans the experts, another the ranks, giving the
-//    exclusive offsets and this CTA's base per expert / rank;
+//  * cluster exchange: each CTA adds its totals into every peer's shared
+//    memory with distributed-shared-memory atomics -- into all peers' sums
+//    and into the "lower CTAs" sums of the peers above it -- so after one
+//    cluster barrier each CTA reads two values per expert; a single CTA
+//    skips this;
+//  * global scan: one packed 64-bit block scan of the (expert, rank) totals
+//    gives both exclusive scans, plus this CTA's base per expert / rank;
 //  * placement: one thread per route, then one per (token, rank), so the
 //    stores of pos / recv_pos are coalesced.
 // When a CTA's tokens do not fit in shared memory at once, it counts all of
@@ -69,8 +71,10 @@ struct Smem {
     unsigned long long *hit;  // [tch] ranks each token reaches
     int32_t *tot;             // [E + R] CTA totals / chunk sums
     int32_t *base;            // [E + R] this CTA's first row per expert / rank
-    int32_t *all_tot;         // [csize][E + R + 2] published totals (+ bad flag, real tokens)
+    int32_t *acc_lo;          // [E + R + 2] sums of the lower CTAs' totals (cluster)
+    int32_t *acc_all;         // [E + R + 2] sums of all CTAs' totals, bad flag, real tokens
     int32_t *misc;            // [2] bad flag, real tokens
+    unsigned long long *scan; // [34] block-scan scratch
 };
 
 // Thread-per-token pass over tokens [t0, t0 + n).  With count_only it adds
@@ -156,41 +160,39 @@ __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
     }
 }
 
-// One warp: exclusive scan of `count` columns of the published totals
-// (column c of CTA q at all_tot[q * W + first + c]); writes this CTA's base
-// per column and (CTA 0) the global counts and offsets.  Returns the total.
-__device__ int warp_global_scan(const Smem &sm, int W, int first, int count, int csize,
-                                int crank, int32_t *base, int32_t *cnt, int32_t *off)
+// Exclusive scan of one 64-bit value per thread across the CTA.  No barrier
+// after the last read of `sm`: the caller separates reuses with a barrier.
+__device__ unsigned long long block_exclusive_scan64(unsigned long long v,
+                                                     unsigned long long *sm,
+                                                     unsigned long long *total)
 {
-    const int lane = threadIdx.x & 31;
-    const int per = (count + 31) >> 5;
-    const int a = min(count, lane * per), b = min(count, a + per);
-    int mine = 0;
-    for (int c = a; c < b; ++c)
-        for (int q = 0; q < csize; ++q) mine += sm.all_tot[q * W + first + c];
-    int inc = mine;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nw = (blockDim.x + 31) >> 5;
+    unsigned long long inc = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(kFull, inc, o);
-        if (lane >= o) inc += t;
+        const unsigned long long n = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += n;
     }
-    int run = inc - mine;
-    for (int c = a; c < b; ++c) {
-        int glob = 0, cb = 0;
-        for (int q = 0; q < csize; ++q) {
-            const int v = sm.all_tot[q * W + first + c];
-            cb += q < crank ? v : 0;
-            glob += v;
+    if (lane == 31) sm[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        const unsigned long long s = lane < nw ? sm[lane] : 0ull;
+        unsigned long long si = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long n = __shfl_up_sync(kFull, si, o);
+            if (lane >= o) si += n;
         }
-        base[c] = run + cb;
-        if (crank == 0) {
-            cnt[c] = glob;
-            off[c] = run;
-        }
-        run += glob;
+        if (lane < nw) sm[lane] = si - s;
+        if (lane == 31) sm[32] = si;
     }
-    return __shfl_sync(kFull, inc, 31);
+    __syncthreads();
+    *total = sm[32];
+    return sm[wid] + inc - v;
 }
+
+constexpr int kMaxPer = EPX_MAX_EXPERTS / 1024;  // experts per thread at most
 
 // pos / recv_pos of tokens [t0, t0 + n): one thread per route, then one per
 // (token, rank); stores are coalesced.
@@ -238,7 +240,7 @@ template <typename IdxT, bool CLUSTER>
 __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 {
     extern __shared__ __align__(16) int32_t smem[];
-    const int tid = threadIdx.x, wid = tid >> 5;
+    const int tid = threadIdx.x;
     const int E = p.E, R = p.R, T = p.T;
     pdl_launch_dependents();
 
@@ -247,9 +249,6 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         cg::cluster_group cluster = cg::this_cluster();
         crank = (int)cluster.block_rank();
         csize = (int)cluster.num_blocks();
-        // every CTA must be running before a peer writes into its shared
-        // memory: arrive now, wait just before the first remote store
-        asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     }
 
     const int W = E + R + 2;
@@ -257,11 +256,13 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     Smem sm;
     sm.M = reinterpret_cast<uint32_t *>(smem);
     sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.tch));
-    sm.codes = reinterpret_cast<int32_t *>(sm.hit + p.tch);
+    sm.scan = sm.hit + p.tch;
+    sm.codes = reinterpret_cast<int32_t *>(sm.scan + 34);
     sm.tot = sm.codes + (size_t)p.tch * p.k;
     sm.base = sm.tot + E + R;
-    sm.all_tot = sm.base + E + R;
-    sm.misc = sm.all_tot + csize * W;
+    sm.acc_lo = sm.base + E + R;
+    sm.acc_all = sm.acc_lo + W;
+    sm.misc = sm.acc_all + W;
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
     const int c0 = min(T, crank * p.tpc);
@@ -272,12 +273,16 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
     // prologue in shared memory only, so it may overlap the previous kernel
     if (tid < 2) sm.misc[tid] = 0;
+    if (CLUSTER)
+        for (int i = tid; i < 2 * W; i += blockDim.x) sm.acc_lo[i] = 0;  // acc_lo, acc_all
     if (nchunks <= 1) {
         zero_words(sm.M, wdt * (p.tch + 1));
     } else {
         for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
     }
     __syncthreads();
+    // peers add into this CTA's accumulators only after it zeroed them
+    if (CLUSTER) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
     pdl_wait_previous();
 
     if (nchunks <= 1) {
@@ -291,42 +296,72 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     if (nreal) atomicAdd(&sm.misc[1], nreal);
     __syncthreads();
 
-    // ---- publish this CTA's totals (to every CTA of the cluster)
+    // ---- cluster exchange: add this CTA's totals into every peer's
+    // acc_all and into the acc_lo of the peers above it
+    const int32_t *glob = sm.tot;
+    const int32_t *lower = nullptr;
     if (CLUSTER) {
         cg::cluster_group cluster = cg::this_cluster();
-        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
         for (int i = tid; i < W; i += blockDim.x) {
             const int v = i < E + R ? sm.tot[i] : sm.misc[i - E - R];
-            for (int c = 0; c < csize; ++c) cluster.map_shared_rank(sm.all_tot, c)[crank * W + i] = v;
+            if (v == 0) continue;
+            for (int c = 0; c < csize; ++c) {
+                atomicAdd(cluster.map_shared_rank(sm.acc_all, c) + i, v);
+                if (c > crank) atomicAdd(cluster.map_shared_rank(sm.acc_lo, c) + i, v);
+            }
         }
         cluster.sync();
-    } else {
-        for (int i = tid; i < W; i += blockDim.x)
-            sm.all_tot[i] = i < E + R ? sm.tot[i] : sm.misc[i - E - R];
-        __syncthreads();
+        glob = sm.acc_all;
+        lower = sm.acc_lo;
     }
 
-    // ---- global scans: warp 0 experts, warp 1 ranks, warp 2 the flags
-    if (wid == 0) {
-        const int n_route = warp_global_scan(sm, W, 0, E, csize, crank, sm.base, p.cnt_e, p.off_e);
-        if (crank == 0 && tid == 0) {
+    // ---- global exclusive scans (one packed 64-bit block scan), bases
+    {
+        const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+        unsigned int contrib_e = 0;
+#pragma unroll
+        for (int q = 0; q < kMaxPer; ++q) {
+            const int e = tid * per + q;
+            if (q < per && e < E) contrib_e += glob[e];
+        }
+        const unsigned int glob_r = tid < R ? (unsigned)glob[E + tid] : 0u;
+        unsigned long long total;
+        const unsigned long long ex = block_exclusive_scan64(
+            ((unsigned long long)contrib_e << 32) | glob_r, sm.scan, &total);
+        unsigned int run = (unsigned int)(ex >> 32);
+#pragma unroll
+        for (int q = 0; q < kMaxPer; ++q) {
+            const int e = tid * per + q;
+            if (q < per && e < E) {
+                sm.base[e] = (int)run + (lower ? lower[e] : 0);
+                if (crank == 0) {
+                    p.cnt_e[e] = glob[e];
+                    p.off_e[e] = (int)run;
+                }
+                run += glob[e];
+            }
+        }
+        if (tid < R) {
+            const int off_r = (int)(unsigned int)(ex & 0xffffffffull);
+            sm.base[E + tid] = off_r + (lower ? lower[E + tid] : 0);
+            if (crank == 0) {
+                p.cnt_r[tid] = glob[E + tid];
+                p.off_r[tid] = off_r;
+            }
+        }
+        if (tid == 0 && crank == 0) {
+            const int n_route = (int)(total >> 32);
+            const int n_recv = (int)(total & 0xffffffffull);
+            const int errc = CLUSTER ? sm.acc_all[E + R] : sm.misc[0];
+            const int nr = CLUSTER ? sm.acc_all[E + R + 1] : sm.misc[1];
             p.off_e[E] = n_route;
-            p.totals[0] = n_route;
-        }
-    } else if (wid == 1) {
-        const int n_recv = warp_global_scan(sm, W, E, R, csize, crank, sm.base + E, p.cnt_r, p.off_r);
-        if (crank == 0 && (tid & 31) == 0) {
             p.off_r[R] = n_recv;
+            p.totals[0] = n_route;
             p.totals[1] = n_recv;
+            p.totals[2] = nr;
+            p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
         }
-    } else if (wid == 2 && (tid & 31) == 0 && crank == 0) {
-        int errc = 0, nr = 0;
-        for (int c = 0; c < csize; ++c) {
-            errc |= sm.all_tot[c * W + E + R];
-            nr += sm.all_tot[c * W + E + R + 1];
-        }
-        p.totals[2] = nr;
-        p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
     }
     __syncthreads();
 
@@ -359,9 +394,10 @@ struct Geometry {
     size_t smem;
 };
 
-size_t fixed_bytes(int E, int R, int csize)
+size_t fixed_bytes(int E, int R)
 {
-    return sizeof(int32_t) * (2 * (size_t)(E + R) + (size_t)csize * (E + R + 2) + 2) + 16;
+    // scan scratch, tot, base, acc_lo, acc_all, misc
+    return 34 * 8 + sizeof(int32_t) * (2 * (size_t)(E + R) + 2 * (size_t)(E + R + 2) + 2) + 16;
 }
 
 // Cluster size and chunk width for a layout problem.
@@ -373,14 +409,9 @@ Geometry plan(int T, int k, int E, int R, int csize)
     const int wdt = g.wde + g.wdr;
     // bytes per token of chunk width: a matrix column, its codes, its rank mask
     const size_t per_tok = (size_t)wdt * 4 + (size_t)k * 4 + 8;
-    // the exchange area grows with the cluster: shrink the cluster if the
-    // fixed part would leave room for fewer than 64 tokens per chunk
-    while (csize > 1 && fixed_bytes(E, R, csize) + (size_t)wdt * 4 + 64 * per_tok + 32 >
-                            (size_t)kMaxDynSmem)
-        csize >>= 1;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    long long cap = ((long long)kMaxDynSmem - (long long)fixed_bytes(E, R, csize) -
+    long long cap = ((long long)kMaxDynSmem - (long long)fixed_bytes(E, R) -
                      (long long)wdt * 4 - 32) / (long long)per_tok;
     if (cap > 1024) cap = 1024;            // one token per thread
     if (cap > 65535 / k) cap = 65535 / k;  // 16-bit counts cannot overflow
@@ -389,7 +420,7 @@ Geometry plan(int T, int k, int E, int R, int csize)
     const int want = ((g.tpc < 1 ? 1 : g.tpc) + 31) & ~31;
     g.tch = want < cap ? want : (int)cap;
     g.smem = matrix_words(wdt, g.tch) * 4 + (size_t)g.tch * 8 + (size_t)g.tch * k * 4 +
-             fixed_bytes(E, R, csize);
+             fixed_bytes(E, R);
     return g;
 }
 
