@@ -21,9 +21,10 @@
 //    memory -- counts are packed two 16-bit rows per 32-bit word, and the
 //    count seen before incrementing is the route's rank among equal experts
 //    of its own token;
-//  * row scan: each warp takes whole matrix rows and scans them 32 tokens at
-//    a time with shuffles (packed 16-bit halves add independently), carrying
-//    the running sum; the carry at the end is the CTA total of the row;
+//  * row scan: each warp takes whole matrix rows; lane l owns a block of
+//    consecutive tokens, sums it, one shuffle scan over the lane sums gives
+//    each lane its start, and the lane writes its running prefix (packed
+//    16-bit halves add independently); the row sum is the CTA total;
 //  * cluster exchange: each CTA adds its totals into every peer's shared
 //    memory with distributed-shared-memory atomics -- into all peers' sums
 //    and into the "lower CTAs" sums of the peers above it -- so after one
@@ -31,8 +32,8 @@
 //    skips this;
 //  * global scan: one packed 64-bit block scan of the (expert, rank) totals
 //    gives both exclusive scans, plus this CTA's base per expert / rank;
-//  * placement: one thread per route, then one per (token, rank), so the
-//    stores of pos / recv_pos are coalesced.
+//  * placement: one thread per four routes, then per four (token, rank)
+//    pairs, so the stores of pos / recv_pos are coalesced 16-byte vectors.
 // When a CTA's tokens do not fit in shared memory at once, it counts all of
 // them first (atomics into its totals) and then builds, scans and places the
 // tokens chunk by chunk with a running base per row.
@@ -65,8 +66,14 @@ __device__ __forceinline__ int div_small(int i, float inv)
 
 __device__ __forceinline__ uint32_t half16(uint32_t w, int sh) { return (w >> sh) & 0xffffu; }
 
+// Column of token u in a count-matrix row.  In the row scan lane l owns the
+// G = 2^lg_g consecutive tokens [l*G, l*G + G); with G even one padding word
+// after every G tokens makes lane l's block start at l*(G+1), an odd stride,
+// so the 32 lanes hit 32 different banks.
+__device__ __forceinline__ int col_of(int u, int lg_g) { return lg_g ? u + (u >> lg_g) : u; }
+
 struct Smem {
-    uint32_t *M;              // [wde + wdr][tch + 1] counts, then in-chunk prefixes
+    uint32_t *M;              // [wde + wdr][ld] counts, then in-chunk prefixes
     int32_t *codes;           // [tch][k]
     unsigned long long *hit;  // [tch] ranks each token reaches
     int32_t *tot;             // [E + R] CTA totals / chunk sums
@@ -86,10 +93,11 @@ template <typename IdxT>
 __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx, int t0, int n,
                             const Smem &sm, bool count_only, bool *bad)
 {
-    const int k = p.k, E = p.E, ld = p.tch + 1;
+    const int k = p.k, E = p.E, ld = p.ld;
     int nreal = 0;
     for (int u = threadIdx.x; u < n; u += blockDim.x) {
         const IdxT *row = idx + (size_t)(t0 + u) * k;
+        const int cu = col_of(u, p.lg_g);
         unsigned long long mask = 0ull;
         for (int j0 = 0; j0 < k; j0 += 8) {
             long long ev[8];
@@ -112,10 +120,10 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
                         if (first) atomicAdd(&sm.tot[E + r], 1);
                     } else {
                         const int sh = (ei & 1) * 16;
-                        uint32_t *cell = sm.M + (size_t)(ei >> 1) * ld + u;
+                        uint32_t *cell = sm.M + (size_t)(ei >> 1) * ld + cu;
                         const uint32_t w = *cell;
                         *cell = w + (1u << sh);
-                        if (first) sm.M[(size_t)(p.wde + (r >> 1)) * ld + u] += 1u << ((r & 1) * 16);
+                        if (first) sm.M[(size_t)(p.wde + (r >> 1)) * ld + cu] += 1u << ((r & 1) * 16);
                         code = ei | ((int)half16(w, sh) << 12);
                     }
                 }
@@ -128,34 +136,40 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
     return nreal;
 }
 
-// Exclusive prefix over the n tokens of every matrix row; warps take whole
-// rows, lanes 32 consecutive tokens at a time (conflict-free), carrying the
-// running sum.  The row totals, unpacked, go to tot[E + R].
+// Exclusive prefix over the n tokens of every matrix row.  Warps take whole
+// rows; lane l owns tokens [l*G, l*G + G): it sums them, one shuffle scan over
+// the 32 lane sums gives every lane its start, and a second pass writes the
+// running prefix.  The row totals, unpacked, go to tot[E + R].
 __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const int wdt = p.wde + p.wdr, ld = p.tch + 1;
+    const int wdt = p.wde + p.wdr, G = 1 << p.lg_g;
+    const int ta = min(n, lane * G), tb = min(n, ta + G);
+    const int ca = col_of(ta, p.lg_g);
     for (int w = wid; w < wdt; w += nwarps) {
-        uint32_t *row = sm.M + (size_t)w * ld;
-        uint32_t carry = 0;
-        for (int s = 0; s < n; s += 32) {
-            const uint32_t v = s + lane < n ? row[s + lane] : 0u;
-            uint32_t inc = v;
+        uint32_t *row = sm.M + (size_t)w * p.ld + ca;
+        uint32_t sum = 0;
+        for (int t = 0; t < tb - ta; ++t) sum += row[t];
+        uint32_t inc = sum;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(kFull, inc, o);
-                if (lane >= o) inc += t;
-            }
-            if (s + lane < n) row[s + lane] = carry + inc - v;
-            carry += __shfl_sync(kFull, inc, 31);
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += v;
         }
+        uint32_t run = inc - sum;
+        for (int t = 0; t < tb - ta; ++t) {
+            const uint32_t v = row[t];
+            row[t] = run;
+            run += v;
+        }
+        const uint32_t total = __shfl_sync(kFull, inc, 31);
         if (lane == 0) {
             const bool er = w < p.wde;
             const int c0 = er ? 2 * w : 2 * (w - p.wde);
             const int lim = er ? p.E : p.R;
             int32_t *dst = er ? sm.tot : sm.tot + p.E;
-            dst[c0] = (int32_t)(carry & 0xffffu);
-            if (c0 + 1 < lim) dst[c0 + 1] = (int32_t)(carry >> 16);
+            dst[c0] = (int32_t)(total & 0xffffu);
+            if (c0 + 1 < lim) dst[c0 + 1] = (int32_t)(total >> 16);
         }
     }
 }
@@ -194,31 +208,60 @@ __device__ unsigned long long block_exclusive_scan64(unsigned long long v,
 
 constexpr int kMaxPer = EPX_MAX_EXPERTS / 1024;  // experts per thread at most
 
-// pos / recv_pos of tokens [t0, t0 + n): one thread per route, then one per
-// (token, rank); stores are coalesced.
+// pos / recv_pos of tokens [t0, t0 + n): one thread per four routes (or per
+// route when k is not a multiple of 4), then per four (token, rank) pairs;
+// the 16-byte stores are coalesced.
+__device__ __forceinline__ int route_pos(const LayoutParams &p, const Smem &sm, int i, int u)
+{
+    const int c = sm.codes[i];
+    if (c < 0) return -1;
+    const int e = code_e(c);
+    return sm.base[e] +
+           (int)half16(sm.M[(size_t)(e >> 1) * p.ld + col_of(u, p.lg_g)], (e & 1) * 16) +
+           code_dup(c);
+}
+
+__device__ __forceinline__ int pair_pos(const LayoutParams &p, const Smem &sm, int u, int r)
+{
+    if (!((sm.hit[u] >> r) & 1ull)) return -1;
+    return sm.base[p.E + r] +
+           (int)half16(sm.M[(size_t)(p.wde + (r >> 1)) * p.ld + col_of(u, p.lg_g)], (r & 1) * 16);
+}
+
 __device__ void place_tokens(const LayoutParams &p, const Smem &sm, int t0, int n)
 {
-    const int k = p.k, E = p.E, R = p.R, ld = p.tch + 1;
-    const float inv_k = 1.0f / (float)k, inv_r = 1.0f / (float)R;
-    for (int i = threadIdx.x; i < n * k; i += blockDim.x) {
-        const int u = div_small(i, inv_k);
-        const int c = sm.codes[i];
-        int v = -1;
-        if (c >= 0) {
-            const int e = code_e(c);
-            v = sm.base[e] + (int)half16(sm.M[(size_t)(e >> 1) * ld + u], (e & 1) * 16) +
-                code_dup(c);
+    const int k = p.k, R = p.R;
+    if ((k & 3) == 0) {
+        const int k4 = k >> 2;
+        const float inv = 1.0f / (float)k4;
+        int4 *dst = reinterpret_cast<int4 *>(p.pos + (size_t)t0 * k);
+        for (int i = threadIdx.x; i < n * k4; i += blockDim.x) {
+            const int u = div_small(i, inv);
+            const int j = 4 * i;
+            dst[i] = make_int4(route_pos(p, sm, j, u), route_pos(p, sm, j + 1, u),
+                               route_pos(p, sm, j + 2, u), route_pos(p, sm, j + 3, u));
         }
-        p.pos[(size_t)t0 * k + i] = v;
+    } else {
+        const float inv = 1.0f / (float)k;
+        for (int i = threadIdx.x; i < n * k; i += blockDim.x)
+            p.pos[(size_t)t0 * k + i] = route_pos(p, sm, i, div_small(i, inv));
     }
-    for (int i = threadIdx.x; i < n * R; i += blockDim.x) {
-        const int u = div_small(i, inv_r);
-        const int r = i - u * R;
-        int v = -1;
-        if ((sm.hit[u] >> r) & 1ull)
-            v = sm.base[E + r] +
-                (int)half16(sm.M[(size_t)(p.wde + (r >> 1)) * ld + u], (r & 1) * 16);
-        p.recv_pos[(size_t)t0 * R + i] = v;
+    if ((R & 3) == 0) {
+        const int r4 = R >> 2;
+        const float inv = 1.0f / (float)r4;
+        int4 *dst = reinterpret_cast<int4 *>(p.recv_pos + (size_t)t0 * R);
+        for (int i = threadIdx.x; i < n * r4; i += blockDim.x) {
+            const int u = div_small(i, inv);
+            const int r = 4 * (i - u * r4);
+            dst[i] = make_int4(pair_pos(p, sm, u, r), pair_pos(p, sm, u, r + 1),
+                               pair_pos(p, sm, u, r + 2), pair_pos(p, sm, u, r + 3));
+        }
+    } else {
+        const float inv = 1.0f / (float)R;
+        for (int i = threadIdx.x; i < n * R; i += blockDim.x) {
+            const int u = div_small(i, inv);
+            p.recv_pos[(size_t)t0 * R + i] = pair_pos(p, sm, u, i - u * R);
+        }
     }
 }
 
@@ -231,9 +274,9 @@ __device__ void zero_words(uint32_t *a, int n)
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += blockDim.x) a[i] = 0u;
 }
 
-__host__ __device__ size_t matrix_words(int wdt, int tch)
+__host__ __device__ size_t matrix_words(int wdt, int ld)
 {
-    return ((size_t)wdt * (tch + 1) + 3) & ~(size_t)3;
+    return ((size_t)wdt * ld + 3) & ~(size_t)3;
 }
 
 template <typename IdxT, bool CLUSTER>
@@ -255,7 +298,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     const int wdt = p.wde + p.wdr;
     Smem sm;
     sm.M = reinterpret_cast<uint32_t *>(smem);
-    sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.tch));
+    sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.ld));
     sm.scan = sm.hit + p.tch;
     sm.codes = reinterpret_cast<int32_t *>(sm.scan + 34);
     sm.tot = sm.codes + (size_t)p.tch * p.k;
@@ -276,7 +319,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     if (CLUSTER)
         for (int i = tid; i < 2 * W; i += blockDim.x) sm.acc_lo[i] = 0;  // acc_lo, acc_all
     if (nchunks <= 1) {
-        zero_words(sm.M, wdt * (p.tch + 1));
+        zero_words(sm.M, wdt * p.ld);
     } else {
         for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
     }
@@ -373,7 +416,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     for (int ch = 0; ch < nchunks; ++ch) {
         const int t0 = c0 + ch * p.tch;
         const int n = min(p.tch, c0 + nt - t0);
-        zero_words(sm.M, wdt * (p.tch + 1));
+        zero_words(sm.M, wdt * p.ld);
         __syncthreads();
         bool b2 = false;
         build_tokens(p, idx, t0, n, sm, false, &b2);
@@ -390,7 +433,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 // ------------------------------------------------------------------- host
 
 struct Geometry {
-    int csize, tpc, tch, wde, wdr;
+    int csize, tpc, tch, lg_g, ld, wde, wdr;
     size_t smem;
 };
 
@@ -407,20 +450,33 @@ Geometry plan(int T, int k, int E, int R, int csize)
     g.wde = (E + 1) / 2;
     g.wdr = (R + 1) / 2;
     const int wdt = g.wde + g.wdr;
-    // bytes per token of chunk width: a matrix column, its codes, its rank mask
-    const size_t per_tok = (size_t)wdt * 4 + (size_t)k * 4 + 8;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    long long cap = ((long long)kMaxDynSmem - (long long)fixed_bytes(E, R) -
-                     (long long)wdt * 4 - 32) / (long long)per_tok;
-    if (cap > 1024) cap = 1024;            // one token per thread
-    if (cap > 65535 / k) cap = 65535 / k;  // 16-bit counts cannot overflow
-    if (cap >= 32) cap &= ~31LL;           // whole warps of tokens when there is room
-    if (cap < 1) cap = 1;
-    const int want = ((g.tpc < 1 ? 1 : g.tpc) + 31) & ~31;
-    g.tch = want < cap ? want : (int)cap;
-    g.smem = matrix_words(wdt, g.tch) * 4 + (size_t)g.tch * 8 + (size_t)g.tch * k * 4 +
-             fixed_bytes(E, R);
+    const size_t fixed = fixed_bytes(E, R);
+    // shared memory for a chunk of w tokens: matrix (w + padding words per
+    // row), rank masks, route codes
+    auto bytes = [&](int w, int ld) {
+        return ((size_t)wdt * ld + 4) * 4 + (size_t)w * 8 + (size_t)w * k * 4 + fixed;
+    };
+    // tch = 32 * G with G a power of two: the smallest that holds the CTA's
+    // tokens, limited by shared memory, one token per thread and 16-bit counts
+    int lg = 0;
+    while ((32 << lg) < g.tpc && (32 << (lg + 1)) <= 1024 && (32 << (lg + 1)) * k <= 65535 &&
+           bytes(32 << (lg + 1), (32 << (lg + 1)) + 32) <= (size_t)kMaxDynSmem)
+        ++lg;
+    int tch = 32 << lg;
+    int ld = lg ? tch + 32 : tch;
+    if (bytes(tch, ld) > (size_t)kMaxDynSmem) {
+        // not even 32 tokens fit (very large E): smaller chunks, one per lane
+        lg = 0;
+        tch = 31;
+        while (tch > 1 && bytes(tch, tch) > (size_t)kMaxDynSmem) --tch;
+        ld = tch;
+    }
+    g.tch = tch;
+    g.lg_g = lg;
+    g.ld = ld;
+    g.smem = bytes(tch, ld);
     return g;
 }
 
@@ -494,6 +550,8 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
         g = plan(p.T, p.k, p.E, p.R, g.csize > 8 ? 8 : g.csize >> 1);
     p.tpc = g.tpc;
     p.tch = g.tch;
+    p.lg_g = g.lg_g;
+    p.ld = g.ld;
     p.wde = g.wde;
     p.wdr = g.wdr;
     if (g.csize == 1)
