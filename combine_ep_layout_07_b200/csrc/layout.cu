@@ -150,6 +150,18 @@ __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
         uint32_t *row = sm.M + (size_t)w * p.ld + ca;
         uint32_t sum = 0;
         for (int t = 0; t < tb - ta; ++t) sum += row[t];
+        if (!__any_sync(kFull, sum != 0u)) {
+            // nobody routed here: the zeroed row already is its own prefix
+            if (lane == 0) {
+                const bool er = w < p.wde;
+                const int c0 = er ? 2 * w : 2 * (w - p.wde);
+                const int lim = er ? p.E : p.R;
+                int32_t *dst = er ? sm.tot : sm.tot + p.E;
+                dst[c0] = 0;
+                if (c0 + 1 < lim) dst[c0 + 1] = 0;
+            }
+            continue;
+        }
         uint32_t inc = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
