@@ -52,6 +52,10 @@ def _load():
     lib.orc_standin.restype = None
     lib.orc_combine.argtypes = [P, P, P, I, I, I, P, P]
     lib.orc_combine.restype = None
+    lib.orc_combine_local.argtypes = [P, P, P, I, P, P, I, I, I, I, I, I, P]
+    lib.orc_combine_local.restype = None
+    lib.orc_combine_epilogue.argtypes = [P, I, P, P, I, I, I, P]
+    lib.orc_combine_epilogue.restype = None
     lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
     lib.orc_bf16_from_double.restype = ctypes.c_uint16
     lib.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -150,3 +154,37 @@ def run_all(wl: dict, idx_dtype=np.int64) -> dict:
     y = standin(expanded, lay)
     out = combine(y, wl["topk_weights"], lay)
     return dict(layout=lay, recv=recv, expanded=expanded, y=y, out=out)
+
+
+def combine_local(y: np.ndarray, topk_weights: np.ndarray, lay: dict, part_bits: int = 32):
+    """Per-(token, rank) partial rows in the receive layout: float32 or bf16
+    bits (uint16), shape [N_recv, H]."""
+    T, k = lay["T"], lay["k"]
+    y = np.ascontiguousarray(y, dtype=np.uint16)
+    H = y.shape[1]
+    if y.shape[0] == 0:
+        y = np.zeros((1, H), np.uint16)
+    w = np.ascontiguousarray(topk_weights, dtype=np.float32)
+    idx = lay["idx"]
+    n = max(lay["N_recv"], 1)
+    part = np.zeros((n, H), np.float32 if part_bits == 32 else np.uint16)
+    _load().orc_combine_local(_p(y), _p(w), _p(idx), 64 if idx.dtype == np.int64 else 32,
+                              _p(lay["pos"]), _p(lay["recv_pos"]), T, k, lay["E"], lay["R"], H,
+                              part_bits, _p(part))
+    return part[:lay["N_recv"]]
+
+
+def combine_epilogue(partial: np.ndarray, lay: dict, residual: np.ndarray = None):
+    """Sum of each token's partial rows (rank order) plus an optional bf16
+    residual row, rounded to bf16 bits [T, H]."""
+    T, R = lay["T"], lay["R"]
+    part_bits = 32 if partial.dtype == np.float32 else 16
+    H = partial.shape[1]
+    part = np.ascontiguousarray(partial)
+    if part.shape[0] == 0:
+        part = np.zeros((1, H), part.dtype)
+    res = None if residual is None else np.ascontiguousarray(residual, dtype=np.uint16)
+    out = np.zeros((T, H), np.uint16)
+    _load().orc_combine_epilogue(_p(part), part_bits, _p(lay["recv_pos"]),
+                                 _p(res) if res is not None else None, T, R, H, _p(out))
+    return out

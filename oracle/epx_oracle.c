@@ -255,3 +255,69 @@ void orc_combine(const uint16_t *y, const float *w, const int32_t *pos,
                 out_exact[(size_t)t * H + h] = acc;
         }
 }
+
+/* ------------------------------------------- two-stage combine (NEXT) */
+
+/*
+ * Local reduce before the combine all2all (DeepEP issue #48, answer on the
+ * reduction kernel before the combine all2all): every rank sums, for each
+ * token it received, its own experts' weighted outputs, giving one partial
+ * row per (token, rank) in the receive layout:
+ *   partial[recv_pos[t, r], h] = sum over valid j with rank(e_j) == r, in k
+ *                                order, of w[t, j] * y[pos[t, j], h]
+ * summed in double, then stored as fp32 (part_bits 32) or bf16 (16).
+ * `partial` holds N_recv rows of H (float or uint16).
+ */
+void orc_combine_local(const uint16_t *y, const float *w, const void *topk_idx, int idx_bits,
+                       const int32_t *pos, const int32_t *recv_pos, int T, int k, int E,
+                       int R, int H, int part_bits, void *partial)
+{
+    const int epr = E / R;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)H);
+    for (int t = 0; t < T; t++)
+        for (int r = 0; r < R; r++) {
+            int32_t d = recv_pos[(int64_t)t * R + r];
+            if (d < 0) continue;
+            for (int h = 0; h < H; h++) acc[h] = 0.0;
+            for (int j = 0; j < k; j++) {
+                int32_t p = pos[(int64_t)t * k + j];
+                if (p < 0) continue;
+                int64_t e = read_idx(topk_idx, idx_bits, (int64_t)t * k + j);
+                if ((int)(e / epr) != r) continue;
+                double wj = (double)w[(int64_t)t * k + j];
+                for (int h = 0; h < H; h++)
+                    acc[h] += wj * orc_bf16_to_double(y[(size_t)p * H + h]);
+            }
+            for (int h = 0; h < H; h++) {
+                if (part_bits == 32)
+                    ((float *)partial)[(size_t)d * H + h] = (float)acc[h];
+                else
+                    ((uint16_t *)partial)[(size_t)d * H + h] = orc_bf16_from_double(acc[h]);
+            }
+        }
+    free(acc);
+}
+
+/*
+ * Combine epilogue (DeepEP issue #760: combine_reduce_epilogue reduces the
+ * rows received back from every rank into the token's output): for every
+ * token, the partial rows of the ranks it reached, in rank order, summed in
+ * double, plus an optional residual row, rounded once to bf16.  A token that
+ * reached no rank gives its residual row (or +0 without one).
+ */
+void orc_combine_epilogue(const void *partial, int part_bits, const int32_t *recv_pos,
+                          const uint16_t *residual, int T, int R, int H, uint16_t *out)
+{
+    for (int t = 0; t < T; t++)
+        for (int h = 0; h < H; h++) {
+            double acc = residual ? orc_bf16_to_double(residual[(size_t)t * H + h]) : 0.0;
+            for (int r = 0; r < R; r++) {
+                int32_t d = recv_pos[(int64_t)t * R + r];
+                if (d < 0) continue;
+                acc += part_bits == 32
+                           ? (double)((const float *)partial)[(size_t)d * H + h]
+                           : orc_bf16_to_double(((const uint16_t *)partial)[(size_t)d * H + h]);
+            }
+            out[(size_t)t * H + h] = orc_bf16_from_double(acc);
+        }
+}

@@ -11,6 +11,11 @@
   bf16 error bound, bit-exact round trip of x through identity experts with
   normalised weights, weights used without renormalisation, zero rows for
   padding tokens, and the worked example of issue #760 (golden fixture).
+* two-stage combine (local reduce, then epilogue): with unit expert outputs
+  every partial is the token's local gate-weight sum (the issue #760 fake
+  expert output); the issue #760 worked example through both stages; the
+  partials of all ranks add up to the single-stage sum; the residual-add
+  epilogue returns the residual for zero partials.
 """
 import bisect
 import json
@@ -380,3 +385,83 @@ def test_bad_indices_are_counted_and_dropped():
     assert lay["n_bad"] == 3
     assert lay["N_route"] == 4
     assert list(lay["pos"][0]) == [0, -1, -1, -1]
+
+
+# ------------------------------------------------ two-stage combine pins
+
+def _rank_of(idx, E, R):
+    return np.where(idx >= 0, idx // (E // R), -1)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "dp_padded"])
+def test_local_partials_of_unit_expert_output_are_local_weight_sums(name):
+    """DeepEP issue #760, Reproduction: the fake expert output makes each
+    received row the sum of its valid local gate weights (top-k weights
+    masked to the rank's own experts).  With every expert output = 1 that is
+    exactly what the local reduce must produce, per (token, rank)."""
+    wl = wlmod.make(name, seed=4)
+    lay = oracle.layout(wl["topk_idx"], wl["E"], wl["R"])
+    ones = np.full((lay["N_route"], wl["H"]), 0x3F80, np.uint16)
+    part = oracle.combine_local(ones, wl["topk_weights"], lay, part_bits=32)
+    rk = _rank_of(wl["topk_idx"], wl["E"], wl["R"])
+    w = wl["topk_weights"].astype(np.float64)
+    for t in range(lay["T"]):
+        for r in range(lay["R"]):
+            d = lay["recv_pos"][t, r]
+            if d < 0:
+                assert not np.any(rk[t] == r)
+                continue
+            masked = np.where(rk[t] == r, w[t], 0.0).sum()   # masked_fill(idx<0, 0).sum
+            assert np.all(part[d] == np.float32(masked))
+
+
+def test_two_stage_worked_example_issue760():
+    """Sixteen ranks each hold one route of weight 1/16: every partial row is
+    1/16 and the epilogue gives exactly 1 for the real row, 0 for padding
+    rows (the value the page checks with an all-reduced max error)."""
+    for T in (1, 2, 4, 8):
+        wl = wlmod.make_lowbatch(T)
+        lay = oracle.layout(wl["topk_idx"], wl["E"], wl["R"])
+        ones = np.full((lay["N_route"], wl["H"]), 0x3F80, np.uint16)
+        for bits in (32, 16):
+            part = oracle.combine_local(ones, wl["topk_weights"], lay, part_bits=bits)
+            pf = part if bits == 32 else wlmod.bf16_bits_to_f32(part)
+            assert part.shape[0] == 16 and np.all(pf == 0.0625)
+            out = wlmod.bf16_bits_to_f32(oracle.combine_epilogue(part, lay))
+            assert np.all(out[0] == 1.0) and np.all(out[1:] == 0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill"])
+def test_two_stage_sums_to_single_stage(name):
+    """The partials of all ranks add up to the whole weighted sum: summed in
+    double they match the single-stage sum up to fp32 rounding of each
+    partial, and the epilogue output matches the closed form."""
+    wl = wlmod.make(name, seed=0)
+    res = oracle.run_all(wl)
+    lay = res["layout"]
+    _, exact = oracle.combine(res["y"], wl["topk_weights"], lay, exact=True)
+    part = oracle.combine_local(res["y"], wl["topk_weights"], lay, part_bits=32)
+    acc = np.zeros_like(exact)
+    for t in range(lay["T"]):
+        rows = lay["recv_pos"][t][lay["recv_pos"][t] >= 0]
+        if rows.size:
+            acc[t] = part[rows].astype(np.float64).sum(axis=0)
+    scale = np.abs(part).astype(np.float64).max() if part.size else 0.0
+    assert np.all(np.abs(acc - exact) <= lay["R"] * 2.0 ** -23 * scale + 1e-30)
+    out = wlmod.bf16_bits_to_f32(oracle.combine_epilogue(part, lay)).astype(np.float64)
+    cf = _closed_form(wl)
+    assert np.all(np.abs(out - cf) <= 2.0 ** -7 * np.abs(cf) + 1e-30)
+
+
+def test_epilogue_residual_add():
+    wl = wlmod.make("tiny", seed=6)
+    res = oracle.run_all(wl)
+    lay = res["layout"]
+    part = oracle.combine_local(res["y"], wl["topk_weights"], lay, part_bits=32)
+    # zero partials: the output is the residual row, bit for bit
+    out0 = oracle.combine_epilogue(np.zeros_like(part), lay, residual=wl["x"])
+    np.testing.assert_array_equal(out0, wl["x"])
+    # residual = x: out = x + sum  (every term has the sign of x: no cancellation)
+    out = wlmod.bf16_bits_to_f32(oracle.combine_epilogue(part, lay, residual=wl["x"]))
+    want = wlmod.bf16_bits_to_f32(wl["x"]).astype(np.float64) + _closed_form(wl)
+    assert np.all(np.abs(out - want) <= 2.0 ** -7 * np.abs(want) + 1e-30)
