@@ -209,6 +209,63 @@ ep_status_t ep_combine_reduce(const void *expert_out, const float *topk_weights,
     return ep_combine_reduce_variant(expert_out, topk_weights, H, L, out, y_rows, 0, stream);
 }
 
+ep_status_t ep_combine_local_reduce(const void *expert_out, const float *topk_weights, int32_t H,
+                                    const ep_layout_t *L, void *partial, int64_t partial_cap,
+                                    int32_t partial_bits, int64_t y_rows, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || y_rows < 0 || partial_cap < 0) return EP_ERR_INVALID_ARG;
+    if (partial_bits != 32 && partial_bits != 16) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!expert_out || !topk_weights || !partial) return EP_ERR_INVALID_ARG;
+    if (!aligned(expert_out, 16) || !aligned(partial, 16)) return EP_ERR_MISALIGNED;
+    if (!aligned(topk_weights, 4)) return EP_ERR_MISALIGNED;
+    LocalParams p;
+    memset(&p, 0, sizeof p);
+    p.y = static_cast<const uint4 *>(expert_out);
+    p.w = topk_weights;
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.off_e = L->off_e;
+    p.T = L->T;
+    p.k = L->k;
+    p.R = L->R;
+    p.epr = L->E / L->R;
+    p.V = H / 8;
+    p.y_rows = y_rows;
+    p.partial = partial;
+    p.part_cap = partial_cap;
+    p.part_bits = partial_bits;
+    p.err = L->totals + 3;
+    return from_cuda(launch_local_reduce(p, as_stream(stream)));
+}
+
+ep_status_t ep_combine_epilogue(const void *partial, int32_t partial_bits, int32_t H,
+                                const ep_layout_t *L, int64_t partial_cap, const void *residual,
+                                void *out, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || partial_cap < 0) return EP_ERR_INVALID_ARG;
+    if (partial_bits != 32 && partial_bits != 16) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!partial || !out) return EP_ERR_INVALID_ARG;
+    if (!aligned(partial, 16) || !aligned(out, 16)) return EP_ERR_MISALIGNED;
+    if (residual && !aligned(residual, 16)) return EP_ERR_MISALIGNED;
+    EpilogueParams p;
+    memset(&p, 0, sizeof p);
+    p.partial = partial;
+    p.part_bits = partial_bits;
+    p.recv_pos = L->recv_pos;
+    p.residual = static_cast<const uint4 *>(residual);
+    p.T = L->T;
+    p.R = L->R;
+    p.V = H / 8;
+    p.part_cap = partial_cap;
+    p.out = static_cast<uint4 *>(out);
+    p.err = L->totals + 3;
+    return from_cuda(launch_epilogue(p, as_stream(stream)));
+}
+
 ep_status_t ep_layout_read_totals(const ep_layout_t *L, int64_t *n_route, int64_t *n_recv,
                                   int64_t *t_real, int32_t *dev_err, void *stream)
 {

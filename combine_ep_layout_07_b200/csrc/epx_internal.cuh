@@ -51,6 +51,32 @@ struct CombineParams {
     int32_t *err;
 };
 
+struct LocalParams {
+    const uint4 *y;
+    const float *w;
+    const int32_t *pos;
+    const int32_t *recv_pos;
+    const int32_t *off_e;
+    int T, k, R, epr;
+    int V, vpc;
+    int64_t y_rows;
+    void *partial;    // [part_cap, H] fp32 or bf16, receive layout
+    int64_t part_cap;
+    int part_bits;    // 32 or 16
+    int32_t *err;
+};
+
+struct EpilogueParams {
+    const void *partial;
+    int part_bits;
+    const int32_t *recv_pos;
+    const uint4 *residual;  // bf16 [T, H] or nullptr
+    int T, R, V, vpc;
+    int64_t part_cap;
+    uint4 *out;
+    int32_t *err;
+};
+
 struct StandinParams {
     const uint4 *ex;
     const int32_t *off_e;
@@ -68,6 +94,8 @@ cudaError_t launch_layout(const LayoutParams &p, int idx_bits, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchParams &p, int variant, cudaStream_t s);
 cudaError_t launch_standin(const StandinParams &p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
+cudaError_t launch_local_reduce(const LocalParams &p, cudaStream_t s);
+cudaError_t launch_epilogue(const EpilogueParams &p, cudaStream_t s);
 
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;

@@ -21,7 +21,8 @@ import torch
 
 __all__ = [
     "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
-    "combine_reduce", "read_totals", "roundtrip_host", "roundtrip_device_bytes",
+    "combine_reduce", "combine_local_reduce", "combine_epilogue", "read_totals",
+    "roundtrip_host", "roundtrip_device_bytes",
     "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES",
     "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
 ]
@@ -76,6 +77,8 @@ def lib():
         "ep_standin_expert": ([P, I32, LP, P, I64, P], I32),
         "ep_combine_reduce": ([P, P, I32, LP, P, I64, P], I32),
         "ep_combine_reduce_variant": ([P, P, I32, LP, P, I64, I32, P], I32),
+        "ep_combine_local_reduce": ([P, P, I32, LP, P, I64, I32, I64, P], I32),
+        "ep_combine_epilogue": ([P, I32, I32, LP, I64, P, P, P], I32),
         "ep_layout_read_totals": ([LP, ctypes.POINTER(I64), ctypes.POINTER(I64),
                                    ctypes.POINTER(I64), ctypes.POINTER(I32), P], I32),
         "ep_roundtrip_device_bytes": ([I32, I32, I32, I32, I32, I32], SZ),
@@ -216,6 +219,39 @@ def combine_reduce(expert_out: torch.Tensor, topk_weights: torch.Tensor, lay: La
                                                               torch.float32),
         H, lay.ref, _dev(out, "out", torch.bfloat16), expert_out.shape[0], variant,
         _stream(stream)), "ep_combine_reduce")
+    return out
+
+
+def combine_local_reduce(expert_out: torch.Tensor, topk_weights: torch.Tensor, lay: Layout,
+                         partial: torch.Tensor = None, partial_dtype=torch.float32,
+                         stream=None):
+    """ep_combine_local_reduce: one partial row per (token, rank) in the
+    receive layout, [T*min(k,R), H] fp32 or bf16 (rows past N_recv untouched)."""
+    H = expert_out.shape[1]
+    if topk_weights.shape != (lay.T, lay.k):
+        raise ValueError("topk_weights must be [T, k]")
+    if partial is None:
+        partial = torch.empty((lay.recv_cap, H), dtype=partial_dtype, device=expert_out.device)
+    bits = {torch.float32: 32, torch.bfloat16: 16}[partial.dtype]
+    _check(lib().ep_combine_local_reduce(
+        _dev(expert_out, "expert_out", torch.bfloat16),
+        _dev(topk_weights, "topk_weights", torch.float32), H, lay.ref,
+        _dev(partial, "partial"), partial.shape[0], bits, expert_out.shape[0],
+        _stream(stream)), "ep_combine_local_reduce")
+    return partial
+
+
+def combine_epilogue(partial: torch.Tensor, lay: Layout, residual: torch.Tensor = None,
+                     out: torch.Tensor = None, stream=None):
+    """ep_combine_epilogue: out[t] = bf16(residual[t] + sum of t's partial rows)."""
+    H = partial.shape[1]
+    bits = {torch.float32: 32, torch.bfloat16: 16}[partial.dtype]
+    if out is None:
+        out = torch.empty((lay.T, H), dtype=torch.bfloat16, device=partial.device)
+    res = None if residual is None else _dev(residual, "residual", torch.bfloat16)
+    _check(lib().ep_combine_epilogue(_dev(partial, "partial"), bits, H, lay.ref,
+                                     partial.shape[0], res, _dev(out, "out", torch.bfloat16),
+                                     _stream(stream)), "ep_combine_epilogue")
     return out
 
 

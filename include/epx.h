@@ -182,6 +182,39 @@ ep_status_t ep_combine_reduce_variant(const void *expert_out,
                                       void *stream);
 
 /*
+ * Two-stage combine, first stage: the local reduce a rank runs before the
+ * combine all2all (DeepEP issue #48, answer on the reduction kernel before
+ * the combine all2all).  For every (token t, rank r) pair of the layout:
+ *   partial[recv_pos[t, r], h] = sum over valid j whose expert lives on r,
+ *                                in k order, of topk_weights[t, j] *
+ *                                expert_out[pos[t, j], h]
+ * accumulated in fp32 and stored as fp32 (partial_bits 32) or bf16 (16).
+ * partial: device [partial_cap, H] in the receive layout (rank r's rows are
+ * [off_r[r], off_r[r+1])); worst case partial_cap = T*min(k, R).  These rows
+ * are what a consumer that takes over the epilogue receives (the "skip the
+ * epilogue" option of DeepEP issue #760).  expert_out / topk_weights as in
+ * ep_combine_reduce.
+ */
+ep_status_t ep_combine_local_reduce(const void *expert_out, const float *topk_weights,
+                                    int32_t H, const ep_layout_t *L, void *partial,
+                                    int64_t partial_cap, int32_t partial_bits,
+                                    int64_t y_rows, void *stream);
+
+/*
+ * Two-stage combine, second stage: the combine epilogue (DeepEP issue #760,
+ * combine_reduce_epilogue).  For every token:
+ *   out[t, h] = bf16_rn( residual[t, h] + sum over ranks r with
+ *                        recv_pos[t, r] >= 0, in rank order, of
+ *                        partial[recv_pos[t, r], h] )
+ * in fp32; residual (device bf16 [T, H], 16-byte aligned) may be NULL, which
+ * drops that term -- the residual add is the downstream fusion the issue's
+ * second proposal asks for.  out: device bf16 [T, H].
+ */
+ep_status_t ep_combine_epilogue(const void *partial, int32_t partial_bits, int32_t H,
+                                const ep_layout_t *L, int64_t partial_cap,
+                                const void *residual, void *out, void *stream);
+
+/*
  * Copy the layout's totals to the host and synchronise `stream`.  Any
  * pointer may be NULL.  Returns EP_ERR_BAD_INDEX or EP_ERR_CAPACITY when
  * the device error word has the matching bit set (the totals are still
