@@ -60,6 +60,10 @@ KERNEL_SOURCES = {
                        "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "layout": ["combine_ep_layout_07_b200/csrc/layout.cu",
                "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "combine_local": ["combine_ep_layout_07_b200/csrc/combine_two_stage.cu",
+                      "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "combine_epilogue": ["combine_ep_layout_07_b200/csrc/combine_two_stage.cu",
+                         "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
 }
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 
@@ -86,6 +90,9 @@ def parse_args(argv=None):
                     help="launch the three calls from Python each step instead of replaying "
                          "one captured CUDA graph per step")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--two-stage", choices=["fp32", "bf16"], default=None,
+                    help="combine as a per-(token, rank) local reduce with fp32 or bf16 "
+                         "partials followed by the epilogue, instead of the fused reduce")
     return ap.parse_args(argv)
 
 
@@ -106,15 +113,21 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes):
+def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None):
     """Algorithmic HBM bytes per step of each kernel (each byte the definition
-    must move once; no re-reads)."""
+    must move once; no re-reads).  With part_bytes (4 or 2) the combine is the
+    two-stage form: local reduce + epilogue through N_recv partial rows."""
     row = H * 2
     layout = T * k * idx_bytes + T * k * 4 + T * R * 4
     dispatch = T_real * row + (N_recv + N_route) * row + T * k * 4 + T * R * 4
-    combine = N_route * row + T * row + T * k * (4 + 4)
-    return dict(layout=layout, dispatch_expand=dispatch, combine_reduce=combine,
-                total=layout + dispatch + combine)
+    out = dict(layout=layout, dispatch_expand=dispatch)
+    if part_bytes is None:
+        out["combine_reduce"] = N_route * row + T * row + T * k * (4 + 4)
+    else:
+        out["combine_local"] = N_route * row + N_recv * H * part_bytes + T * k * 8 + T * R * 4
+        out["combine_epilogue"] = N_recv * H * part_bytes + T * row + T * R * 4
+    out["total"] = sum(out.values())
+    return out
 
 
 def sources_hash(kernel):
@@ -323,7 +336,9 @@ def workload_config(wl, args, lay_totals, flush_desc=None):
            "R": wl["R"], "k": wl["k"], "seed": args.seed, "idx_bits": args.idx_bits,
            "T_real": int(lay_totals["T_real"]), "N_recv": int(lay_totals["N_recv"]),
            "N_route": int(lay_totals["N_route"]),
-           "timed": "layout + dispatch_expand + combine_reduce",
+           "timed": "layout + dispatch_expand + " + (
+               "combine_reduce" if not getattr(args, "two_stage", None) else
+               "combine_local_reduce (%s partials) + combine_epilogue" % args.two_stage),
            "parallelism": f"replicas x{dist_env()[1]}"}
     if flush_desc:
         cfg["l2"] = flush_desc
@@ -367,20 +382,33 @@ def run_epx(args):
     y = torch.empty_like(expanded)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
 
+    part = None
+    if args.two_stage:
+        part = torch.empty((lay.recv_cap, H), device=dev,
+                           dtype=torch.float32 if args.two_stage == "fp32" else torch.bfloat16)
+    calls = [
+        ("layout", lambda st: epx.layout(idx, E, R, out=lay, stream=st)),
+        ("dispatch_expand", lambda st: epx.dispatch_expand(
+            x, lay, recv=recv, expanded=expanded, variant=args.dispatch_variant, stream=st)),
+    ]
+    if part is None:
+        calls.append(("combine_reduce", lambda st: epx.combine_reduce(
+            y, w, lay, out=out, variant=args.combine_variant, stream=st)))
+    else:
+        calls.append(("combine_local", lambda st: epx.combine_local_reduce(
+            y, w, lay, partial=part, stream=st)))
+        calls.append(("combine_epilogue", lambda st: epx.combine_epilogue(
+            part, lay, out=out, stream=st)))
+    names = [n for n, _ in calls]
+
     def step_kernels(events=None, st=None):
         st = stream if st is None else st
+        for i, (_, fn) in enumerate(calls):
+            if events is not None:
+                events[i].record(st)
+            fn(st)
         if events is not None:
-            events[0].record(st)
-        epx.layout(idx, E, R, out=lay, stream=st)
-        if events is not None:
-            events[1].record(st)
-        epx.dispatch_expand(x, lay, recv=recv, expanded=expanded,
-                            variant=args.dispatch_variant, stream=st)
-        if events is not None:
-            events[2].record(st)
-        epx.combine_reduce(y, w, lay, out=out, variant=args.combine_variant, stream=st)
-        if events is not None:
-            events[3].record(st)
+            events[len(calls)].record(st)
 
     with torch.cuda.stream(stream):
         epx.layout(idx, E, R, out=lay, stream=stream)
@@ -389,7 +417,8 @@ def run_epx(args):
     tot = epx.read_totals(lay, stream=stream)
 
     bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
-                       args.idx_bits // 8)
+                       args.idx_bits // 8,
+                       None if part is None else part.element_size())
     working = bytes_["total"]
     flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
@@ -413,7 +442,8 @@ def run_epx(args):
             gev[0].record(cs)
             step_kernels(st=cs)
             gev[1].record(cs)
-        gks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        gks = [torch.cuda.Event(enable_timing=True, external=True)
+               for _ in range(len(calls) + 1)]
         graph_k = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_k, stream=stream):
             step_kernels(gks, st=torch.cuda.current_stream())
@@ -427,12 +457,12 @@ def run_epx(args):
             if out is not None:
                 torch.cuda.current_stream().synchronize()
                 if split:
-                    out.append([gks[0].elapsed_time(gks[j]) for j in (1, 2, 3)])
+                    out.append([gks[0].elapsed_time(gks[j]) for j in range(1, len(gks))])
                 else:
                     out.append(gev[0].elapsed_time(gev[1]))
         else:
             if out is not None:
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
                 step_kernels(ev)
                 out.append(ev)
             else:
@@ -472,13 +502,11 @@ def run_epx(args):
         sampler.stop()
 
     if graph is None:   # cumulative times from each step's first event
-        rec_k = [[e[0].elapsed_time(e[j]) for j in (1, 2, 3)] for e in rec]
-        step_ms = [r[2] for r in rec_k]
+        rec_k = [[e[0].elapsed_time(e[j]) for j in range(1, len(e))] for e in rec]
+        step_ms = [r[-1] for r in rec_k]
     else:
         step_ms = rec
-    k_ms = {"layout": [r[0] for r in rec_k],
-            "dispatch_expand": [r[1] - r[0] for r in rec_k],
-            "combine_reduce": [r[2] - r[1] for r in rec_k]}
+    k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)
     value = whole_job_value(tot["T_real"] * args.steps, world, total_ms)
 
@@ -500,7 +528,9 @@ def run_epx(args):
         kernels[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
                          "alg_bytes": bytes_[name], "gbs": gbs, "frac": gbs / peak}
     dom = max(kernels, key=lambda n: kernels[n]["us"])
-    engine = {"dispatch_expand": "bulk" if args.dispatch_variant == 2 or
+    engine = {"combine_local": "two_stage_" + str(args.two_stage),
+              "combine_epilogue": "two_stage_" + str(args.two_stage),
+              "dispatch_expand": "bulk" if args.dispatch_variant == 2 or
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
               "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split"}
     traffic = committed_traffic(dom, args.workload, engine.get(dom))
@@ -519,7 +549,7 @@ def run_epx(args):
         "roofline": roofline,
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
         "kernels": kernels,
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": len(calls) * args.steps,
         "e2e": e2e,
     }
     if sampler:
