@@ -56,6 +56,8 @@ def _load():
     lib.orc_combine_local.restype = None
     lib.orc_combine_epilogue.argtypes = [P, I, P, P, I, I, I, P]
     lib.orc_combine_epilogue.restype = None
+    lib.orc_expand_index.argtypes = [P, I, P, P, I, I, I, I, P]
+    lib.orc_expand_index.restype = None
     lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
     lib.orc_bf16_from_double.restype = ctypes.c_uint16
     lib.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -188,3 +190,13 @@ def combine_epilogue(partial: np.ndarray, lay: dict, residual: np.ndarray = None
     _load().orc_combine_epilogue(_p(part), part_bits, _p(lay["recv_pos"]),
                                  _p(res) if res is not None else None, T, R, H, _p(out))
     return out
+
+
+def expand_index(lay: dict) -> np.ndarray:
+    """Row of `recv` that serves each expert-contiguous row, int32 [N_route]."""
+    idx = lay["idx"]
+    src = np.full(max(lay["N_route"], 1), -1, np.int32)
+    _load().orc_expand_index(_p(idx), 64 if idx.dtype == np.int64 else 32, _p(lay["pos"]),
+                             _p(lay["recv_pos"]), lay["T"], lay["k"], lay["E"], lay["R"],
+                             _p(src))
+    return src[:lay["N_route"]]

@@ -321,3 +321,27 @@ void orc_combine_epilogue(const void *partial, int part_bits, const int32_t *rec
             out[(size_t)t * H + h] = orc_bf16_from_double(acc);
         }
 }
+
+/* ------------------------------------------- dispatch without expand (NEXT) */
+
+/*
+ * Gather index for a consumer that reads the received rows directly instead
+ * of an expanded copy (DeepEP issue #760, Reproduction: dispatch with
+ * do_expand=False; issue #48, answer on the VRAM / performance tradeoff of
+ * expanding): the expert-contiguous row of route (t, j) is served by the row
+ * in which token t was received by the rank that owns expert e_j,
+ *   src[pos[t, j]] = recv_pos[t, rank(e_j)]   for every valid route.
+ * src has N_route entries.
+ */
+void orc_expand_index(const void *topk_idx, int idx_bits, const int32_t *pos,
+                      const int32_t *recv_pos, int T, int k, int E, int R, int32_t *src)
+{
+    const int epr = E / R;
+    for (int t = 0; t < T; t++)
+        for (int j = 0; j < k; j++) {
+            int32_t p = pos[(int64_t)t * k + j];
+            if (p < 0) continue;
+            int64_t e = read_idx(topk_idx, idx_bits, (int64_t)t * k + j);
+            src[p] = recv_pos[(int64_t)t * R + (int)(e / epr)];
+        }
+}

@@ -465,3 +465,22 @@ def test_epilogue_residual_add():
     out = wlmod.bf16_bits_to_f32(oracle.combine_epilogue(part, lay, residual=wl["x"]))
     want = wlmod.bf16_bits_to_f32(wl["x"]).astype(np.float64) + _closed_form(wl)
     assert np.all(np.abs(out - want) <= 2.0 ** -7 * np.abs(want) + 1e-30)
+
+
+# ------------------------------------------- dispatch without expand pins
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "dp_padded", "lowbatch2"])
+def test_expand_index_serves_every_expanded_row(name):
+    """Reading recv through the gather index gives exactly the expanded rows
+    (the copy a do_expand=False consumer avoids), and every index stays in the
+    owning rank's receive segment."""
+    wl = wlmod.make(name, seed=2)
+    lay = oracle.layout(wl["topk_idx"], wl["E"], wl["R"])
+    recv, expanded = oracle.dispatch_expand(wl["x"], lay)
+    src = oracle.expand_index(lay)
+    assert src.shape == (lay["N_route"],) and np.all(src >= 0)
+    np.testing.assert_array_equal(recv[src], expanded)
+    epr = wl["E"] // wl["R"]
+    expert_of_row = np.repeat(np.arange(wl["E"]), lay["cnt_e"])
+    rank_of_row = expert_of_row // epr
+    assert np.all(src >= lay["off_r"][rank_of_row]) and np.all(src < lay["off_r"][rank_of_row + 1])
