@@ -60,6 +60,10 @@ KERNEL_SOURCES = {
                        "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "layout": ["combine_ep_layout_07_b200/csrc/layout.cu",
                "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "dispatch": ["combine_ep_layout_07_b200/csrc/dispatch.cu",
+                 "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
+    "expand_index": ["combine_ep_layout_07_b200/csrc/gather.cu",
+                     "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "combine_local": ["combine_ep_layout_07_b200/csrc/combine_two_stage.cu",
                       "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "combine_epilogue": ["combine_ep_layout_07_b200/csrc/combine_two_stage.cu",
@@ -90,6 +94,10 @@ def parse_args(argv=None):
                     help="launch the three calls from Python each step instead of replaying "
                          "one captured CUDA graph per step")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-expand", action="store_true",
+                    help="dispatch writes recv rows only plus a gather index (the expert "
+                         "consumer reads recv through it); also times that consumer "
+                         "against the one reading the expanded copy")
     ap.add_argument("--two-stage", choices=["fp32", "bf16"], default=None,
                     help="combine as a per-(token, rank) local reduce with fp32 or bf16 "
                          "partials followed by the epilogue, instead of the fused reduce")
@@ -113,14 +121,21 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None):
+def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None,
+              no_expand=False):
     """Algorithmic HBM bytes per step of each kernel (each byte the definition
     must move once; no re-reads).  With part_bytes (4 or 2) the combine is the
-    two-stage form: local reduce + epilogue through N_recv partial rows."""
+    two-stage form: local reduce + epilogue through N_recv partial rows.  With
+    no_expand the dispatch writes recv rows only, plus the gather index."""
     row = H * 2
     layout = T * k * idx_bytes + T * k * 4 + T * R * 4
-    dispatch = T_real * row + (N_recv + N_route) * row + T * k * 4 + T * R * 4
-    out = dict(layout=layout, dispatch_expand=dispatch)
+    if no_expand:
+        out = dict(layout=layout,
+                   dispatch=T_real * row + N_recv * row + T * R * 4,
+                   expand_index=T * k * 4 + T * R * 4 + N_route * 4)
+    else:
+        out = dict(layout=layout,
+                   dispatch_expand=T_real * row + (N_recv + N_route) * row + T * k * 4 + T * R * 4)
     if part_bytes is None:
         out["combine_reduce"] = N_route * row + T * row + T * k * (4 + 4)
     else:
@@ -144,6 +159,8 @@ def committed_traffic(kernel, workload, engine=None):
     try:
         lines = open(TRAFFIC_FILE).read().splitlines()
     except OSError:
+        return None
+    if kernel not in KERNEL_SOURCES:
         return None
     want = sources_hash(kernel)
     for ln in lines:
@@ -336,7 +353,9 @@ def workload_config(wl, args, lay_totals, flush_desc=None):
            "R": wl["R"], "k": wl["k"], "seed": args.seed, "idx_bits": args.idx_bits,
            "T_real": int(lay_totals["T_real"]), "N_recv": int(lay_totals["N_recv"]),
            "N_route": int(lay_totals["N_route"]),
-           "timed": "layout + dispatch_expand + " + (
+           "timed": "layout + " + ("dispatch (recv only) + expand_index + "
+                                   if getattr(args, "no_expand", False)
+                                   else "dispatch_expand + ") + (
                "combine_reduce" if not getattr(args, "two_stage", None) else
                "combine_local_reduce (%s partials) + combine_epilogue" % args.two_stage),
            "parallelism": f"replicas x{dist_env()[1]}"}
@@ -386,11 +405,14 @@ def run_epx(args):
     if args.two_stage:
         part = torch.empty((lay.recv_cap, H), device=dev,
                            dtype=torch.float32 if args.two_stage == "fp32" else torch.bfloat16)
-    calls = [
-        ("layout", lambda st: epx.layout(idx, E, R, out=lay, stream=st)),
-        ("dispatch_expand", lambda st: epx.dispatch_expand(
-            x, lay, recv=recv, expanded=expanded, variant=args.dispatch_variant, stream=st)),
-    ]
+    src = torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev) if args.no_expand else None
+    calls = [("layout", lambda st: epx.layout(idx, E, R, out=lay, stream=st))]
+    if args.no_expand:
+        calls.append(("dispatch", lambda st: epx.dispatch(x, lay, recv=recv, stream=st)))
+        calls.append(("expand_index", lambda st: epx.expand_index(lay, src=src, stream=st)))
+    else:
+        calls.append(("dispatch_expand", lambda st: epx.dispatch_expand(
+            x, lay, recv=recv, expanded=expanded, variant=args.dispatch_variant, stream=st)))
     if part is None:
         calls.append(("combine_reduce", lambda st: epx.combine_reduce(
             y, w, lay, out=out, variant=args.combine_variant, stream=st)))
@@ -415,10 +437,14 @@ def run_epx(args):
         epx.dispatch_expand(x, lay, recv=recv, expanded=expanded, stream=stream)
         epx.standin_expert(expanded, lay, y=y, stream=stream)
     tot = epx.read_totals(lay, stream=stream)
+    consumer = None
+    if args.no_expand:
+        consumer = time_consumers(torch, epx, lay, recv, expanded, y, stream, dev, tot, H,
+                                  max(10, min(args.steps, 200)))
 
     bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
                        args.idx_bits // 8,
-                       None if part is None else part.element_size())
+                       None if part is None else part.element_size(), args.no_expand)
     working = bytes_["total"]
     flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
@@ -528,7 +554,8 @@ def run_epx(args):
         kernels[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
                          "alg_bytes": bytes_[name], "gbs": gbs, "frac": gbs / peak}
     dom = max(kernels, key=lambda n: kernels[n]["us"])
-    engine = {"combine_local": "two_stage_" + str(args.two_stage),
+    engine = {"dispatch": "recv_only", "expand_index": "gather_index",
+              "combine_local": "two_stage_" + str(args.two_stage),
               "combine_epilogue": "two_stage_" + str(args.two_stage),
               "dispatch_expand": "bulk" if args.dispatch_variant == 2 or
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
@@ -550,6 +577,7 @@ def run_epx(args):
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
         "kernels": kernels,
         "gpu_launches": len(calls) * args.steps,
+        **({"consumer": consumer} if consumer else {}),
         "e2e": e2e,
     }
     if sampler:
@@ -561,6 +589,33 @@ def run_epx(args):
     print(json.dumps(line), flush=True)
     finish(pg)
     return 0
+
+
+def time_consumers(torch, epx, lay, recv, expanded, y, stream, dev, tot, H, n):
+    """The stand-in expert reading the expanded copy vs reading recv through
+    the gather index (CUDA events, eager, n calls each)."""
+    src = epx.expand_index(lay, stream=stream)
+    res = {}
+    for name, fn in (("from_expanded", lambda: epx.standin_expert(expanded, lay, y=y,
+                                                                     stream=stream)),
+                     ("gather_from_recv", lambda: epx.standin_expert_gather(
+                         recv, lay, src, y=y, stream=stream))):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = {"us": e0.elapsed_time(e1) * 1e3 / n}
+    row = H * 2
+    res["from_expanded"]["alg_bytes"] = 2 * tot["N_route"] * row
+    res["gather_from_recv"]["alg_bytes"] = tot["N_recv"] * row + tot["N_route"] * (row + 4)
+    res["expanded_bytes_not_written"] = tot["N_route"] * row
+    return res
 
 
 def parity_summary(torch, lay, expanded, out, ores):

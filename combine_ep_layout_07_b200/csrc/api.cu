@@ -157,6 +157,78 @@ ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L, v
     return ep_dispatch_expand_variant(x, H, L, recv, recv_cap, expanded, exp_cap, 0, stream);
 }
 
+ep_status_t ep_dispatch(const void *x, int32_t H, const ep_layout_t *L, void *recv,
+                        int64_t recv_cap, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || recv_cap < 0) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!x || !recv) return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(recv, 16)) return EP_ERR_MISALIGNED;
+    DispatchParams p;
+    memset(&p, 0, sizeof p);
+    p.x = static_cast<const uint4 *>(x);
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.T = L->T;
+    p.k = L->k;
+    p.R = L->R;
+    p.V = H / 8;
+    p.recv = static_cast<uint4 *>(recv);
+    p.recv_cap = recv_cap;
+    p.expanded = nullptr;  // no expanded copy
+    p.exp_cap = 0;
+    p.err = L->totals + 3;
+    return from_cuda(launch_dispatch(p, 0, as_stream(stream)));
+}
+
+ep_status_t ep_expand_index(const ep_layout_t *L, int32_t *src_row, int64_t rows, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (rows < 0) return EP_ERR_INVALID_ARG;
+    if (L->T == 0 || rows == 0) return EP_OK;
+    if (!src_row) return EP_ERR_INVALID_ARG;
+    if (!aligned(src_row, 4)) return EP_ERR_MISALIGNED;
+    IndexParams p;
+    memset(&p, 0, sizeof p);
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.off_e = L->off_e;
+    p.T = L->T;
+    p.k = L->k;
+    p.R = L->R;
+    p.epr = L->E / L->R;
+    p.src = src_row;
+    p.rows = rows;
+    p.err = L->totals + 3;
+    return from_cuda(launch_expand_index(p, as_stream(stream)));
+}
+
+ep_status_t ep_standin_expert_gather(const void *recv, int64_t recv_rows, int32_t H,
+                                     const ep_layout_t *L, const int32_t *src_row, void *y,
+                                     int64_t rows, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || rows < 0 || recv_rows < 0) return EP_ERR_INVALID_ARG;
+    if (rows == 0 || L->T == 0) return EP_OK;
+    if (!recv || !src_row || !y) return EP_ERR_INVALID_ARG;
+    if (!aligned(recv, 16) || !aligned(y, 16) || !aligned(src_row, 4)) return EP_ERR_MISALIGNED;
+    GatherParams p;
+    memset(&p, 0, sizeof p);
+    p.recv = static_cast<const uint4 *>(recv);
+    p.recv_rows = recv_rows;
+    p.src = src_row;
+    p.off_e = L->off_e;
+    p.totals = L->totals;
+    p.E = L->E;
+    p.V = H / 8;
+    const int64_t cap = (int64_t)L->T * L->k;
+    p.rows = rows < cap ? rows : cap;
+    p.y = static_cast<uint4 *>(y);
+    p.err = L->totals + 3;
+    return from_cuda(launch_standin_gather(p, as_stream(stream)));
+}
+
 ep_status_t ep_standin_expert(const void *expanded, int32_t H, const ep_layout_t *L, void *y,
                               int64_t rows, void *stream)
 {

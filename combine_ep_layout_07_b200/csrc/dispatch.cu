@@ -24,8 +24,9 @@ namespace {
 constexpr int kMaxDst = EPX_MAX_TOPK + EPX_MAX_RANKS;
 
 // Warp-collective: compact the destination rows of token t into dst[0..n).
-// Expanded rows first (k order), then recv rows (rank order).  Rows beyond a
-// capacity are dropped and flagged.  Returns n on every lane.
+// Expanded rows first (k order; none when p.expanded is null), then recv rows
+// (rank order).  Rows beyond a capacity are dropped and flagged.  Returns n
+// on every lane.
 __device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
                                               uint4 **dst)
 {
@@ -33,7 +34,7 @@ __device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
     const unsigned lt = lanemask_lt();
     unsigned flag = 0;
     int n = 0;
-    {
+    if (p.expanded) {  // null: dispatch only (no expanded copy)
         int q = lane < p.k ? p.pos[(size_t)t * p.k + lane] : -1;
         bool over = q >= 0 && (int64_t)q >= p.exp_cap;
         bool ok = q >= 0 && !over;

@@ -77,6 +77,28 @@ struct EpilogueParams {
     int32_t *err;
 };
 
+struct IndexParams {
+    const int32_t *pos;
+    const int32_t *recv_pos;
+    const int32_t *off_e;
+    int T, k, R, epr;
+    int32_t *src;   // [rows] recv row serving each expanded row
+    int64_t rows;
+    int32_t *err;
+};
+
+struct GatherParams {
+    const uint4 *recv;
+    int64_t recv_rows;
+    const int32_t *src;
+    const int32_t *off_e;
+    const int32_t *totals;
+    int E, V, vpc;
+    int64_t rows;
+    uint4 *y;
+    int32_t *err;
+};
+
 struct StandinParams {
     const uint4 *ex;
     const int32_t *off_e;
@@ -96,6 +118,8 @@ cudaError_t launch_standin(const StandinParams &p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
 cudaError_t launch_local_reduce(const LocalParams &p, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueParams &p, cudaStream_t s);
+cudaError_t launch_expand_index(const IndexParams &p, cudaStream_t s);
+cudaError_t launch_standin_gather(const GatherParams &p, cudaStream_t s);
 
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;

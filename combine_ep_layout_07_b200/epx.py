@@ -22,6 +22,7 @@ import torch
 __all__ = [
     "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
     "combine_reduce", "combine_local_reduce", "combine_epilogue", "read_totals",
+    "dispatch", "expand_index", "standin_expert_gather",
     "roundtrip_host", "roundtrip_device_bytes",
     "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES",
     "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
@@ -77,6 +78,9 @@ def lib():
         "ep_standin_expert": ([P, I32, LP, P, I64, P], I32),
         "ep_combine_reduce": ([P, P, I32, LP, P, I64, P], I32),
         "ep_combine_reduce_variant": ([P, P, I32, LP, P, I64, I32, P], I32),
+        "ep_dispatch": ([P, I32, LP, P, I64, P], I32),
+        "ep_expand_index": ([LP, P, I64, P], I32),
+        "ep_standin_expert_gather": ([P, I64, I32, LP, P, P, I64, P], I32),
         "ep_combine_local_reduce": ([P, P, I32, LP, P, I64, I32, I64, P], I32),
         "ep_combine_epilogue": ([P, I32, I32, LP, I64, P, P, P], I32),
         "ep_layout_read_totals": ([LP, ctypes.POINTER(I64), ctypes.POINTER(I64),
@@ -192,6 +196,42 @@ def dispatch_expand(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None,
         _dev(expanded, "expanded", torch.bfloat16), expanded.shape[0], variant,
         _stream(stream)), "ep_dispatch_expand")
     return recv, expanded
+
+
+def dispatch(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None, stream=None):
+    """ep_dispatch: recv rows only (no expanded copy); returns recv [T*min(k,R), H]."""
+    if x.dim() != 2 or x.shape[0] != lay.T:
+        raise ValueError("x must be [T, H]")
+    H = x.shape[1]
+    if recv is None:
+        recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=x.device)
+    _check(lib().ep_dispatch(_dev(x, "x", torch.bfloat16), H, lay.ref,
+                             _dev(recv, "recv", torch.bfloat16), recv.shape[0], _stream(stream)),
+           "ep_dispatch")
+    return recv
+
+
+def expand_index(lay: Layout, src: torch.Tensor = None, stream=None):
+    """ep_expand_index: int32 [T*k] recv row serving each expanded row."""
+    if src is None:
+        src = torch.empty((lay.exp_cap,), dtype=torch.int32, device=lay.mem.device)
+    _check(lib().ep_expand_index(lay.ref, _dev(src, "src", torch.int32), src.shape[0],
+                                 _stream(stream)), "ep_expand_index")
+    return src
+
+
+def standin_expert_gather(recv: torch.Tensor, lay: Layout, src: torch.Tensor,
+                          y: torch.Tensor = None, stream=None):
+    """ep_standin_expert_gather: the stand-in expert reading recv[src[p]]."""
+    H = recv.shape[1]
+    if y is None:
+        y = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16, device=recv.device)
+    _check(lib().ep_standin_expert_gather(_dev(recv, "recv", torch.bfloat16), recv.shape[0], H,
+                                          lay.ref, _dev(src, "src", torch.int32),
+                                          _dev(y, "y", torch.bfloat16),
+                                          min(src.shape[0], y.shape[0]), _stream(stream)),
+           "ep_standin_expert_gather")
+    return y
 
 
 def standin_expert(expanded: torch.Tensor, lay: Layout, y: torch.Tensor = None, stream=None):

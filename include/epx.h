@@ -149,6 +149,36 @@ ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H,
                                        void *stream);
 
 /*
+ * Dispatch only (the pages' do_expand=False: DeepEP issue #760,
+ * Reproduction): recv[recv_pos[t, r]] = x[t] for every rank r the token
+ * reaches, and no expanded copy -- the VRAM side of the expand tradeoff
+ * (DeepEP issue #48, answer on VRAM vs performance).  Arguments as in
+ * ep_dispatch_expand.
+ */
+ep_status_t ep_dispatch(const void *x, int32_t H, const ep_layout_t *L, void *recv,
+                        int64_t recv_cap, void *stream);
+
+/*
+ * Gather index for a consumer that reads the received rows directly:
+ *   src_row[pos[t, j]] = recv_pos[t, rank(e_j)]   for every valid route,
+ * i.e. the recv row that holds expanded row p's data.  src_row: device int32
+ * [rows], rows >= N_route (worst case T*k); entries past N_route untouched;
+ * a pos >= rows is skipped and flagged (EP_DEVERR_EXP_CAP).
+ */
+ep_status_t ep_expand_index(const ep_layout_t *L, int32_t *src_row, int64_t rows,
+                            void *stream);
+
+/*
+ * The stand-in expert of ep_standin_expert reading recv[src_row[p]] in place
+ * of expanded[p] (identical results, no expanded buffer): the pattern of a
+ * grouped consumer of a dispatch without expand.  recv: device bf16
+ * [recv_rows, H]; src_row from ep_expand_index; y: device bf16 [rows, H].
+ */
+ep_status_t ep_standin_expert_gather(const void *recv, int64_t recv_rows, int32_t H,
+                                     const ep_layout_t *L, const int32_t *src_row,
+                                     void *y, int64_t rows, void *stream);
+
+/*
  * Deterministic stand-in for the expert FFN (test and benchmark helper):
  * y[p] = bf16_rn(float(expanded[p]) * (1 + e/E)) in IEEE fp32 for every row
  * p < N_route of expert e's segment.  expanded, y: device bf16 [rows, H],
