@@ -78,8 +78,7 @@ struct Smem {
     unsigned long long *hit;  // [tch] ranks each token reaches
     int32_t *tot;             // [E + R] CTA totals / chunk sums
     int32_t *base;            // [E + R] this CTA's first row per expert / rank
-    int32_t *acc_lo;          // [E + R + 2] sums of the lower CTAs' totals (cluster)
-    int32_t *acc_all;         // [E + R + 2] sums of all CTAs' totals, bad flag, real tokens
+    int32_t *all_tot;         // [csize][E + R + 2] every CTA's totals, bad flag, real tokens
     int32_t *misc;            // [2] bad flag, real tokens
     unsigned long long *scan; // [34] block-scan scratch
 };
@@ -144,12 +143,19 @@ __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const int wdt = p.wde + p.wdr, G = 1 << p.lg_g;
-    const int ta = min(n, lane * G), tb = min(n, ta + G);
+    const int ta = min(n, lane * G), cnt = min(n, ta + G) - ta;
     const int ca = col_of(ta, p.lg_g);
     for (int w = wid; w < wdt; w += nwarps) {
         uint32_t *row = sm.M + (size_t)w * p.ld + ca;
+        // lane sum: loads eight at a time, all in flight
         uint32_t sum = 0;
-        for (int t = 0; t < tb - ta; ++t) sum += row[t];
+        for (int c = 0; c < cnt; c += 8) {
+            uint32_t v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = c + i < cnt ? row[c + i] : 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += v[i];
+        }
         if (!__any_sync(kFull, sum != 0u)) {
             // nobody routed here: the zeroed row already is its own prefix
             if (lane == 0) {
@@ -168,11 +174,17 @@ __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
             const uint32_t v = __shfl_up_sync(kFull, inc, o);
             if (lane >= o) inc += v;
         }
+        // running prefix: each chunk is loaded whole before it is rewritten
         uint32_t run = inc - sum;
-        for (int t = 0; t < tb - ta; ++t) {
-            const uint32_t v = row[t];
-            row[t] = run;
-            run += v;
+        for (int c = 0; c < cnt; c += 8) {
+            uint32_t v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = c + i < cnt ? row[c + i] : 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (c + i < cnt) row[c + i] = run;
+                run += v[i];
+            }
         }
         const uint32_t total = __shfl_sync(kFull, inc, 31);
         if (lane == 0) {
@@ -315,9 +327,8 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     sm.codes = reinterpret_cast<int32_t *>(sm.scan + 34);
     sm.tot = sm.codes + (size_t)p.tch * p.k;
     sm.base = sm.tot + E + R;
-    sm.acc_lo = sm.base + E + R;
-    sm.acc_all = sm.acc_lo + W;
-    sm.misc = sm.acc_all + W;
+    sm.all_tot = sm.base + E + R;
+    sm.misc = sm.all_tot + (size_t)csize * W;
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
     const int c0 = min(T, crank * p.tpc);
@@ -328,16 +339,14 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 
     // prologue in shared memory only, so it may overlap the previous kernel
     if (tid < 2) sm.misc[tid] = 0;
-    if (CLUSTER)
-        for (int i = tid; i < 2 * W; i += blockDim.x) sm.acc_lo[i] = 0;  // acc_lo, acc_all
     if (nchunks <= 1) {
         zero_words(sm.M, wdt * p.ld);
     } else {
         for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
     }
     __syncthreads();
-    // peers add into this CTA's accumulators only after it zeroed them
-    if (CLUSTER) asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    // peers write into this CTA's shared memory only once every CTA runs
+    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     pdl_wait_previous();
 
     if (nchunks <= 1) {
@@ -351,65 +360,87 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     if (nreal) atomicAdd(&sm.misc[1], nreal);
     __syncthreads();
 
-    // ---- cluster exchange: add this CTA's totals into every peer's
-    // acc_all and into the acc_lo of the peers above it
-    const int32_t *glob = sm.tot;
-    const int32_t *lower = nullptr;
+    // ---- cluster exchange: push this CTA's totals into row crank of every
+    // CTA's table (distributed shared memory stores), then read locally
     if (CLUSTER) {
         cg::cluster_group cluster = cg::this_cluster();
-        asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+        asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
         for (int i = tid; i < W; i += blockDim.x) {
             const int v = i < E + R ? sm.tot[i] : sm.misc[i - E - R];
-            if (v == 0) continue;
-            for (int c = 0; c < csize; ++c) {
-                atomicAdd(cluster.map_shared_rank(sm.acc_all, c) + i, v);
-                if (c > crank) atomicAdd(cluster.map_shared_rank(sm.acc_lo, c) + i, v);
-            }
+            for (int c = 0; c < csize; ++c)
+                cluster.map_shared_rank(sm.all_tot, c)[(size_t)crank * W + i] = v;
         }
         cluster.sync();
-        glob = sm.acc_all;
-        lower = sm.acc_lo;
     }
 
     // ---- global exclusive scans (one packed 64-bit block scan), bases
     {
+        // this CTA's totals sum over the cluster: all CTAs (glob) and the
+        // CTAs below this one (lower), read from the local table
+        auto sums = [&](int i, int &g, int &lo) {
+            if (!CLUSTER) {
+                g = sm.tot[i];
+                lo = 0;
+                return;
+            }
+            g = 0;
+            lo = 0;
+            for (int c = 0; c < csize; ++c) {
+                const int v = sm.all_tot[(size_t)c * W + i];
+                g += v;
+                lo += c < crank ? v : 0;
+            }
+        };
         const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+        int glob[kMaxPer], lower[kMaxPer];
         unsigned int contrib_e = 0;
 #pragma unroll
         for (int q = 0; q < kMaxPer; ++q) {
             const int e = tid * per + q;
-            if (q < per && e < E) contrib_e += glob[e];
+            glob[q] = lower[q] = 0;
+            if (q < per && e < E) {
+                sums(e, glob[q], lower[q]);
+                contrib_e += glob[q];
+            }
         }
-        const unsigned int glob_r = tid < R ? (unsigned)glob[E + tid] : 0u;
+        int glob_r = 0, lower_r = 0;
+        if (tid < R) sums(E + tid, glob_r, lower_r);
         unsigned long long total;
         const unsigned long long ex = block_exclusive_scan64(
-            ((unsigned long long)contrib_e << 32) | glob_r, sm.scan, &total);
+            ((unsigned long long)contrib_e << 32) | (unsigned)glob_r, sm.scan, &total);
         unsigned int run = (unsigned int)(ex >> 32);
 #pragma unroll
         for (int q = 0; q < kMaxPer; ++q) {
             const int e = tid * per + q;
             if (q < per && e < E) {
-                sm.base[e] = (int)run + (lower ? lower[e] : 0);
+                sm.base[e] = (int)run + lower[q];
                 if (crank == 0) {
-                    p.cnt_e[e] = glob[e];
+                    p.cnt_e[e] = glob[q];
                     p.off_e[e] = (int)run;
                 }
-                run += glob[e];
+                run += glob[q];
             }
         }
         if (tid < R) {
             const int off_r = (int)(unsigned int)(ex & 0xffffffffull);
-            sm.base[E + tid] = off_r + (lower ? lower[E + tid] : 0);
+            sm.base[E + tid] = off_r + lower_r;
             if (crank == 0) {
-                p.cnt_r[tid] = glob[E + tid];
+                p.cnt_r[tid] = glob_r;
                 p.off_r[tid] = off_r;
             }
         }
         if (tid == 0 && crank == 0) {
             const int n_route = (int)(total >> 32);
             const int n_recv = (int)(total & 0xffffffffull);
-            const int errc = CLUSTER ? sm.acc_all[E + R] : sm.misc[0];
-            const int nr = CLUSTER ? sm.acc_all[E + R + 1] : sm.misc[1];
+            int errc = sm.misc[0], nr = sm.misc[1];
+            if (CLUSTER) {
+                errc = 0;
+                nr = 0;
+                for (int c = 0; c < csize; ++c) {
+                    errc |= sm.all_tot[(size_t)c * W + E + R];
+                    nr += sm.all_tot[(size_t)c * W + E + R + 1];
+                }
+            }
             p.off_e[E] = n_route;
             p.off_r[R] = n_recv;
             p.totals[0] = n_route;
@@ -449,10 +480,11 @@ struct Geometry {
     size_t smem;
 };
 
-size_t fixed_bytes(int E, int R)
+size_t fixed_bytes(int E, int R, int csize)
 {
-    // scan scratch, tot, base, acc_lo, acc_all, misc
-    return 34 * 8 + sizeof(int32_t) * (2 * (size_t)(E + R) + 2 * (size_t)(E + R + 2) + 2) + 16;
+    // scan scratch, tot, base, the cluster's totals table, misc
+    return 34 * 8 +
+           sizeof(int32_t) * (2 * (size_t)(E + R) + (size_t)csize * (E + R + 2) + 2) + 16;
 }
 
 // Cluster size and chunk width for a layout problem.
@@ -462,9 +494,14 @@ Geometry plan(int T, int k, int E, int R, int csize)
     g.wde = (E + 1) / 2;
     g.wdr = (R + 1) / 2;
     const int wdt = g.wde + g.wdr;
+    // the totals table grows with the cluster: shrink the cluster if the
+    // fixed part would leave room for fewer than 32 tokens per chunk
+    while (csize > 1 && fixed_bytes(E, R, csize) + ((size_t)wdt * 32 + 4) * 4 + 32 * 8 +
+                            (size_t)32 * k * 4 > (size_t)kMaxDynSmem)
+        csize >>= 1;
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
-    const size_t fixed = fixed_bytes(E, R);
+    const size_t fixed = fixed_bytes(E, R, csize);
     // shared memory for a chunk of w tokens: matrix (w + padding words per
     // row), rank masks, route codes
     auto bytes = [&](int w, int ld) {
