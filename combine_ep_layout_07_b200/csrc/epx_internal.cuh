@@ -18,9 +18,8 @@ struct LayoutParams {
     int T, k, E, R;
     float inv_epr;  // 1.0f / (E / R): rank of expert e = floor((e + 0.5) * inv_epr)
     int tpc;        // tokens per CTA of the cluster
-    int tch;        // tokens per chunk: 32 << lg_g, or fewer than 32 when shared memory is short
-    int lg_g;       // log2 of tokens per lane in the row scan (G = tch / 32)
-    int ld;         // count-matrix row length in words (tch plus padding)
+    int tch;        // tokens per chunk (columns of the count matrix)
+    int ld;         // count-matrix row length in words: odd, >= tch
     int wde, wdr;   // count-matrix rows (two 16-bit counts per 32-bit word) for experts / ranks
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };

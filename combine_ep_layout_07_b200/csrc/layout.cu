@@ -21,10 +21,9 @@
 //    memory -- counts are packed two 16-bit rows per 32-bit word, and the
 //    count seen before incrementing is the route's rank among equal experts
 //    of its own token;
-//  * row scan: each warp takes whole matrix rows; lane l owns a block of
-//    consecutive tokens, sums it, one shuffle scan over the lane sums gives
-//    each lane its start, and the lane writes its running prefix (packed
-//    16-bit halves add independently); the row sum is the CTA total;
+//  * row scan: one thread per matrix row walks its tokens and rewrites the
+//    counts as a running prefix (packed 16-bit halves add independently);
+//    the row sum is the CTA total;
 //  * cluster exchange: each CTA adds its totals into every peer's shared
 //    memory with distributed-shared-memory atomics -- into all peers' sums
 //    and into the "lower CTAs" sums of the peers above it -- so after one
@@ -66,14 +65,8 @@ __device__ __forceinline__ int div_small(int i, float inv)
 
 __device__ __forceinline__ uint32_t half16(uint32_t w, int sh) { return (w >> sh) & 0xffffu; }
 
-// Column of token u in a count-matrix row.  In the row scan lane l owns the
-// G = 2^lg_g consecutive tokens [l*G, l*G + G); with G even one padding word
-// after every G tokens makes lane l's block start at l*(G+1), an odd stride,
-// so the 32 lanes hit 32 different banks.
-__device__ __forceinline__ int col_of(int u, int lg_g) { return lg_g ? u + (u >> lg_g) : u; }
-
 struct Smem {
-    uint32_t *M;              // [wde + wdr][ld] counts, then in-chunk prefixes
+    uint32_t *M;              // [wde + wdr][ld] counts, then in-chunk prefixes (ld odd)
     int32_t *codes;           // [tch][k]
     unsigned long long *hit;  // [tch] ranks each token reaches
     int32_t *tot;             // [E + R] CTA totals / chunk sums
@@ -96,7 +89,6 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
     int nreal = 0;
     for (int u = threadIdx.x; u < n; u += blockDim.x) {
         const IdxT *row = idx + (size_t)(t0 + u) * k;
-        const int cu = col_of(u, p.lg_g);
         unsigned long long mask = 0ull;
         for (int j0 = 0; j0 < k; j0 += 8) {
             long long ev[8];
@@ -119,10 +111,10 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
                         if (first) atomicAdd(&sm.tot[E + r], 1);
                     } else {
                         const int sh = (ei & 1) * 16;
-                        uint32_t *cell = sm.M + (size_t)(ei >> 1) * ld + cu;
+                        uint32_t *cell = sm.M + (size_t)(ei >> 1) * ld + u;
                         const uint32_t w = *cell;
                         *cell = w + (1u << sh);
-                        if (first) sm.M[(size_t)(p.wde + (r >> 1)) * ld + cu] += 1u << ((r & 1) * 16);
+                        if (first) sm.M[(size_t)(p.wde + (r >> 1)) * ld + u] += 1u << ((r & 1) * 16);
                         code = ei | ((int)half16(w, sh) << 12);
                     }
                 }
@@ -135,66 +127,32 @@ __device__ int build_tokens(const LayoutParams &p, const IdxT *__restrict__ idx,
     return nreal;
 }
 
-// Exclusive prefix over the n tokens of every matrix row.  Warps take whole
-// rows; lane l owns tokens [l*G, l*G + G): it sums them, one shuffle scan over
-// the 32 lane sums gives every lane its start, and a second pass writes the
-// running prefix.  The row totals, unpacked, go to tot[E + R].
+// Exclusive prefix over the n tokens of every matrix row: one thread per row,
+// walking its tokens eight at a time (loads first, then the rewritten
+// prefixes); the row stride is odd, so the 32 rows of a warp sit in 32
+// different banks.  The row totals, unpacked, go to tot[E + R].
 __device__ void row_scan(const LayoutParams &p, const Smem &sm, int n)
 {
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const int wdt = p.wde + p.wdr, G = 1 << p.lg_g;
-    const int ta = min(n, lane * G), cnt = min(n, ta + G) - ta;
-    const int ca = col_of(ta, p.lg_g);
-    for (int w = wid; w < wdt; w += nwarps) {
-        uint32_t *row = sm.M + (size_t)w * p.ld + ca;
-        // lane sum: loads eight at a time, all in flight
-        uint32_t sum = 0;
-        for (int c = 0; c < cnt; c += 8) {
+    const int wdt = p.wde + p.wdr;
+    for (int w = threadIdx.x; w < wdt; w += blockDim.x) {
+        uint32_t *row = sm.M + (size_t)w * p.ld;
+        uint32_t run = 0;
+        for (int c = 0; c < n; c += 8) {
             uint32_t v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = c + i < cnt ? row[c + i] : 0u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) sum += v[i];
-        }
-        if (!__any_sync(kFull, sum != 0u)) {
-            // nobody routed here: the zeroed row already is its own prefix
-            if (lane == 0) {
-                const bool er = w < p.wde;
-                const int c0 = er ? 2 * w : 2 * (w - p.wde);
-                const int lim = er ? p.E : p.R;
-                int32_t *dst = er ? sm.tot : sm.tot + p.E;
-                dst[c0] = 0;
-                if (c0 + 1 < lim) dst[c0 + 1] = 0;
-            }
-            continue;
-        }
-        uint32_t inc = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(kFull, inc, o);
-            if (lane >= o) inc += v;
-        }
-        // running prefix: each chunk is loaded whole before it is rewritten
-        uint32_t run = inc - sum;
-        for (int c = 0; c < cnt; c += 8) {
-            uint32_t v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = c + i < cnt ? row[c + i] : 0u;
+            for (int i = 0; i < 8; ++i) v[i] = c + i < n ? row[c + i] : 0u;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                if (c + i < cnt) row[c + i] = run;
+                if (c + i < n) row[c + i] = run;
                 run += v[i];
             }
         }
-        const uint32_t total = __shfl_sync(kFull, inc, 31);
-        if (lane == 0) {
-            const bool er = w < p.wde;
-            const int c0 = er ? 2 * w : 2 * (w - p.wde);
-            const int lim = er ? p.E : p.R;
-            int32_t *dst = er ? sm.tot : sm.tot + p.E;
-            dst[c0] = (int32_t)(total & 0xffffu);
-            if (c0 + 1 < lim) dst[c0 + 1] = (int32_t)(total >> 16);
-        }
+        const bool er = w < p.wde;
+        const int c0 = er ? 2 * w : 2 * (w - p.wde);
+        const int lim = er ? p.E : p.R;
+        int32_t *dst = er ? sm.tot : sm.tot + p.E;
+        dst[c0] = (int32_t)(run & 0xffffu);
+        if (c0 + 1 < lim) dst[c0 + 1] = (int32_t)(run >> 16);
     }
 }
 
@@ -241,7 +199,7 @@ __device__ __forceinline__ int route_pos(const LayoutParams &p, const Smem &sm, 
     if (c < 0) return -1;
     const int e = code_e(c);
     return sm.base[e] +
-           (int)half16(sm.M[(size_t)(e >> 1) * p.ld + col_of(u, p.lg_g)], (e & 1) * 16) +
+           (int)half16(sm.M[(size_t)(e >> 1) * p.ld + u], (e & 1) * 16) +
            code_dup(c);
 }
 
@@ -249,7 +207,7 @@ __device__ __forceinline__ int pair_pos(const LayoutParams &p, const Smem &sm, i
 {
     if (!((sm.hit[u] >> r) & 1ull)) return -1;
     return sm.base[p.E + r] +
-           (int)half16(sm.M[(size_t)(p.wde + (r >> 1)) * p.ld + col_of(u, p.lg_g)], (r & 1) * 16);
+           (int)half16(sm.M[(size_t)(p.wde + (r >> 1)) * p.ld + u], (r & 1) * 16);
 }
 
 __device__ void place_tokens(const LayoutParams &p, const Smem &sm, int t0, int n)
@@ -476,7 +434,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 // ------------------------------------------------------------------- host
 
 struct Geometry {
-    int csize, tpc, tch, lg_g, ld, wde, wdr;
+    int csize, tpc, tch, ld, wde, wdr;
     size_t smem;
 };
 
@@ -502,30 +460,20 @@ Geometry plan(int T, int k, int E, int R, int csize)
     g.csize = csize;
     g.tpc = (T + csize - 1) / csize;
     const size_t fixed = fixed_bytes(E, R, csize);
-    // shared memory for a chunk of w tokens: matrix (w + padding words per
-    // row), rank masks, route codes
-    auto bytes = [&](int w, int ld) {
-        return ((size_t)wdt * ld + 4) * 4 + (size_t)w * 8 + (size_t)w * k * 4 + fixed;
+    // shared memory for a chunk of w tokens: matrix rows of an odd length
+    // >= w, rank masks, route codes
+    auto bytes = [&](int w) {
+        return ((size_t)wdt * (w | 1) + 4) * 4 + (size_t)w * 8 + (size_t)w * k * 4 + fixed;
     };
-    // tch = 32 * G with G a power of two: the smallest that holds the CTA's
-    // tokens, limited by shared memory, one token per thread and 16-bit counts
-    int lg = 0;
-    while ((32 << lg) < g.tpc && (32 << (lg + 1)) <= 1024 && (32 << (lg + 1)) * k <= 65535 &&
-           bytes(32 << (lg + 1), (32 << (lg + 1)) + 32) <= (size_t)kMaxDynSmem)
-        ++lg;
-    int tch = 32 << lg;
-    int ld = lg ? tch + 32 : tch;
-    if (bytes(tch, ld) > (size_t)kMaxDynSmem) {
-        // not even 32 tokens fit (very large E): smaller chunks, one per lane
-        lg = 0;
-        tch = 31;
-        while (tch > 1 && bytes(tch, tch) > (size_t)kMaxDynSmem) --tch;
-        ld = tch;
-    }
+    // the CTA's tokens in one chunk when they fit: at most one token per
+    // thread, 16-bit counts, shared memory
+    int tch = g.tpc < 1 ? 1 : g.tpc;
+    if (tch > 1024) tch = 1024;
+    if (tch > 65535 / k) tch = 65535 / k;
+    while (tch > 1 && bytes(tch) > (size_t)kMaxDynSmem) tch = tch > 64 ? tch - 32 : tch - 1;
     g.tch = tch;
-    g.lg_g = lg;
-    g.ld = ld;
-    g.smem = bytes(tch, ld);
+    g.ld = tch | 1;
+    g.smem = bytes(tch);
     return g;
 }
 
@@ -599,7 +547,6 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
         g = plan(p.T, p.k, p.E, p.R, g.csize > 8 ? 8 : g.csize >> 1);
     p.tpc = g.tpc;
     p.tch = g.tch;
-    p.lg_g = g.lg_g;
     p.ld = g.ld;
     p.wde = g.wde;
     p.wdr = g.wdr;
