@@ -135,12 +135,7 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
 {
     CombineParams p = p0;
     if (p.T == 0) return cudaSuccess;
-    int nsm = 148;
-    {
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int nsm = current_sm_count();
     const bool big_k = p.k > 8;
     if (variant == 1) {
         int blocks = (p.T + 3) / 4;

@@ -261,10 +261,7 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpilogueParams p)
 // chunks of a row so that a few tokens still spread over the SMs
 void split_rows(int T, int V, int &chunks, int &vpc, int &threads)
 {
-    int nsm = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const int nsm = current_sm_count();
     chunks = (4 * nsm + T - 1) / T;
     const int max_chunks = (V + 31) / 32;
     if (chunks > max_chunks) chunks = max_chunks;

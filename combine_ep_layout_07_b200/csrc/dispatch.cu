@@ -212,12 +212,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
 {
     DispatchParams p = p0;
     if (p.T == 0) return cudaSuccess;
-    int nsm = 148;
-    {
-        int dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess)
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    }
+    const int nsm = current_sm_count();
     const int gy = p.T < 65535 ? p.T : 65535;
     // automatic: TMA bulk copies for large batches (measured faster at 4096
     // rows of 14 KB), register copies for small ones (fewer fixed costs)
@@ -231,16 +226,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
         if (vpc > 2048) vpc = 2048;
         chunks = (p.V + vpc - 1) / vpc;
         p.vpc = vpc;
-        const size_t smem = (size_t)vpc * 16;
-        static int attr_set_mask = 0;
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (dev < 32 && !(attr_set_mask & (1 << dev))) {
-            cudaError_t e = cudaFuncSetAttribute(
-                dispatch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            if (e != cudaSuccess) return e;
-            attr_set_mask |= 1 << dev;
-        }
+        const size_t smem = (size_t)vpc * 16;  // <= 32 KB: no opt-in needed
         return launch_pdl(dispatch_bulk_kernel, dim3(chunks, gy), dim3(32), smem, s, p);
     }
     // vector engine: 128 threads x 2 vectors per pass

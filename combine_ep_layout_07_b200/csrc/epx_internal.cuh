@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "epx.h"
 
 namespace epx {
@@ -119,6 +122,36 @@ cudaError_t launch_local_reduce(const LocalParams &p, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueParams &p, cudaStream_t s);
 cudaError_t launch_expand_index(const IndexParams &p, cudaStream_t s);
 cudaError_t launch_standin_gather(const GatherParams &p, cudaStream_t s);
+
+// ------------------------------------------------- host-side caches
+// Launchers may be called from several host threads at once.
+
+// guards the launchers' small lookup tables
+inline std::mutex &launcher_mutex()
+{
+    static std::mutex m;
+    return m;
+}
+
+// multiprocessor count of device `dev`, queried once per device
+inline int sm_count(int dev)
+{
+    static std::atomic<int> cache[64];
+    int n = 0;
+    if (dev >= 0 && dev < 64) n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+inline int current_sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    return sm_count(dev);
+}
 
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;

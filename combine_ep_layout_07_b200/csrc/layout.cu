@@ -487,6 +487,7 @@ int max_clusters(int csize, size_t smem, int dev)
     };
     static Entry cache[64];
     static int n_cache = 0;
+    std::lock_guard<std::mutex> lock(launcher_mutex());
     for (int i = 0; i < n_cache; ++i)
         if (cache[i].dev == dev && cache[i].csize == csize && cache[i].smem == smem)
             return cache[i].result;
@@ -513,8 +514,8 @@ int max_clusters(int csize, size_t smem, int dev)
 template <typename IdxT>
 cudaError_t set_attributes_once(int dev)
 {
-    static unsigned done = 0;  // per device (up to 32)
-    if (dev < 32 && (done & (1u << dev))) return cudaSuccess;
+    static std::atomic<unsigned> done{0};  // per device (up to 32)
+    if (dev < 32 && (done.load() & (1u << dev))) return cudaSuccess;
     cudaError_t err = cudaFuncSetAttribute(layout_kernel<IdxT, false>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            kMaxDynSmem);
@@ -524,7 +525,7 @@ cudaError_t set_attributes_once(int dev)
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(layout_kernel<IdxT, true>,
                                    cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (err == cudaSuccess && dev < 32) done |= 1u << dev;
+    if (err == cudaSuccess && dev < 32) done.fetch_or(1u << dev);
     return err;
 }
 

@@ -1,0 +1,65 @@
+"""Host-side pieces of bench.py: algorithmic byte counts, the source-hash
+keyed DRAM traffic lookup and the clock-sample summary (no GPU)."""
+import os
+import sys
+import time
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_alg_bytes_prefill_numbers():
+    b = bench.alg_bytes(T=4096, T_real=4096, N_recv=25936, N_route=32768, H=7168, k=8, R=16,
+                        idx_bytes=8)
+    row = 7168 * 2
+    assert b["dispatch_expand"] == 4096 * row + (25936 + 32768) * row + 4096 * 8 * 4 + 4096 * 16 * 4
+    assert b["dispatch_expand"] == 900694016
+    assert b["combine_reduce"] == 32768 * row + 4096 * row + 4096 * 8 * 8
+    assert b["total"] == b["layout"] + b["dispatch_expand"] + b["combine_reduce"]
+
+
+def test_alg_bytes_variants():
+    two = bench.alg_bytes(128, 128, 833, 1024, 7168, 8, 16, 8, part_bytes=4)
+    assert set(two) == {"layout", "dispatch_expand", "combine_local", "combine_epilogue", "total"}
+    assert two["combine_local"] == 1024 * 14336 + 833 * 7168 * 4 + 128 * 8 * 8 + 128 * 16 * 4
+    ne = bench.alg_bytes(128, 128, 833, 1024, 7168, 8, 16, 8, no_expand=True)
+    assert "expand_index" in ne and ne["dispatch"] == 128 * 14336 + 833 * 14336 + 128 * 16 * 4
+
+
+def test_traffic_lookup_follows_source_and_engine(tmp_path, monkeypatch):
+    h = bench.sources_hash("dispatch_expand")
+    f = tmp_path / "traffic.txt"
+    f.write_text("# comment\n"
+                 f"kernel=dispatch_expand workload=prefill source={h} dram_bytes_per_launch=123 engine=bulk\n"
+                 "kernel=dispatch_expand workload=decode source=0000 dram_bytes_per_launch=9 engine=vec\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.committed_traffic("dispatch_expand", "prefill", "bulk") == 123.0
+    assert bench.committed_traffic("dispatch_expand", "prefill", "vec") is None
+    assert bench.committed_traffic("dispatch_expand", "decode", "vec") is None   # stale source
+    assert bench.committed_traffic("no_such_kernel", "prefill") is None
+
+
+def test_clock_summary_window_and_reasons(tmp_path):
+    s = bench.ClockSampler("GPU-x")
+    s.path = str(tmp_path / "clocks.csv")
+    t0 = time.time()
+    stamp = lambda t: time.strftime("%Y/%m/%d %H:%M:%S", time.localtime(t)) + ".000"  # noqa: E731
+    lines = []
+    for i, (mhz, pcap) in enumerate([(1965, "Not Active"), (1900, "Active"), (1965, "Not Active"),
+                                     (1950, "Not Active")]):
+        lines.append(f"{stamp(t0 + i)}, 0, {mhz}, 1965, 700.0, 0x0, Not Active, Not Active, "
+                     f"Not Active, {pcap}")
+    open(s.path, "w").write("\n".join(lines) + "\n")
+    out = s.summary(t0 - 1, t0 + 5)
+    assert out["samples"] == 4 and out["sm_max_mhz"] == 1965.0
+    assert out["sm_mhz"] == pytest.approx(1957.5)
+    assert out["reasons"] == ["sw_power_cap"] and out["window"] == "timed"
+
+
+def test_default_arguments_fit_the_contract():
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps > 0 and a.impl == "epx"
+    assert a.workload == "prefill"
