@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
     __shared__ int s_pos[EPX_MAX_TOPK];
     __shared__ float s_w[EPX_MAX_TOPK];
     __shared__ int s_n;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
             st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos, s_w, n, v));
         __syncthreads();
     }
+    pdl_launch_dependents();
 }
 
 template <int G>
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(128) combine_warp_per_token_kernel(CombinePara
     __shared__ int s_pos[4][EPX_MAX_TOPK];
     __shared__ float s_w[4][EPX_MAX_TOPK];
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.x * 4 + wid; t < p.T; t += gridDim.x * 4) {
         const int n = build_routes(p, t, s_pos[wid], s_w[wid]);
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(128) combine_warp_per_token_kernel(CombinePara
             st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos[wid], s_w[wid], n, v));
         __syncwarp();
     }
+    pdl_launch_dependents();
 }
 
 }  // namespace
@@ -140,6 +142,7 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     if (variant == 1) {
         int blocks = (p.T + 3) / 4;
         if (blocks > 65535 * 16) blocks = 65535 * 16;
+        p.early_pdl = early_trigger(blocks);
         if (big_k)
             return launch_pdl(combine_warp_per_token_kernel<16>, dim3(blocks), dim3(128), 0, s, p);
         return launch_pdl(combine_warp_per_token_kernel<8>, dim3(blocks), dim3(128), 0, s, p);
@@ -153,6 +156,7 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     chunks = (p.V + p.vpc - 1) / p.vpc;
     int threads = p.vpc < 128 ? ((p.vpc + 31) / 32) * 32 : 128;
     const int gy = p.T < 65535 ? p.T : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     if (big_k)
         return launch_pdl(combine_split_kernel<16>, dim3(chunks, gy), dim3(threads), 0, s, p);
     return launch_pdl(combine_split_kernel<8>, dim3(chunks, gy), dim3(threads), 0, s, p);

@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
     __shared__ float s_w[EPX_MAX_TOPK];
     __shared__ int64_t s_grow[EPX_MAX_TOPK];
     __shared__ int s_n, s_ng;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int i = threadIdx.x; i <= p.R; i += blockDim.x) s_bound[i] = p.off_e[i * p.epr];
     __syncthreads();
@@ -178,6 +178,7 @@ __global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
         }
         __syncthreads();
     }
+    pdl_launch_dependents();
 }
 
 // Warp 0: token t's partial rows in rank order.  Returns their number.
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpilogueParams p)
 {
     __shared__ int64_t s_row[EPX_MAX_RANKS];
     __shared__ int s_n;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
@@ -256,6 +257,7 @@ __global__ void __launch_bounds__(128) epilogue_kernel(EpilogueParams p)
         }
         __syncthreads();
     }
+    pdl_launch_dependents();
 }
 
 // chunks of a row so that a few tokens still spread over the SMs
@@ -280,6 +282,7 @@ cudaError_t launch_local_reduce(const LocalParams &p0, cudaStream_t s)
     int chunks, threads;
     split_rows(p.T, p.V, chunks, p.vpc, threads);
     const int gy = p.T < 65535 ? p.T : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     if (p.k > 8)
         return launch_pdl(local_reduce_kernel<16>, dim3(chunks, gy), dim3(threads), 0, s, p);
     return launch_pdl(local_reduce_kernel<8>, dim3(chunks, gy), dim3(threads), 0, s, p);
@@ -292,6 +295,7 @@ cudaError_t launch_epilogue(const EpilogueParams &p0, cudaStream_t s)
     int chunks, threads;
     split_rows(p.T, p.V, chunks, p.vpc, threads);
     const int gy = p.T < 65535 ? p.T : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     if (p.part_bits == 32)
         return launch_pdl(epilogue_kernel<4, 32>, dim3(chunks, gy), dim3(threads), 0, s, p);
     return launch_pdl(epilogue_kernel<8, 16>, dim3(chunks, gy), dim3(threads), 0, s, p);

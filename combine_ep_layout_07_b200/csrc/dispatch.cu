@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
 {
     __shared__ uint4 *s_dst[kMaxDst];
     __shared__ int s_n;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
         }
         __syncthreads();
     }
+    pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------ bulk
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
     __shared__ uint4 *s_dst[kMaxDst];
     __shared__ __align__(8) uint64_t bar;
     const int lane = threadIdx.x;
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     if (lane == 0) mbar_init(&bar, 1);
     __syncwarp();
     pdl_wait_previous();
@@ -204,6 +205,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
         bulk_commit_and_wait_read();  // sbuf and s_dst are reused next token
         __syncwarp();
     }
+    pdl_launch_dependents();
 }
 
 }  // namespace
@@ -227,6 +229,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
         chunks = (p.V + vpc - 1) / vpc;
         p.vpc = vpc;
         const size_t smem = (size_t)vpc * 16;  // <= 32 KB: no opt-in needed
+        p.early_pdl = early_trigger((long long)chunks * gy);
         return launch_pdl(dispatch_bulk_kernel, dim3(chunks, gy), dim3(32), smem, s, p);
     }
     // vector engine: 128 threads x 2 vectors per pass
@@ -236,6 +239,7 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
     if (chunks < 1) chunks = 1;
     p.vpc = (p.V + chunks - 1) / chunks;
     chunks = (p.V + p.vpc - 1) / p.vpc;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     return launch_pdl(dispatch_vec_kernel<2, false>, dim3(chunks, gy), dim3(128), 0, s, p);
 }
 

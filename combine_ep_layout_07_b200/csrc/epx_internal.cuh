@@ -39,6 +39,7 @@ struct DispatchParams {
     uint4 *expanded;
     int64_t exp_cap;
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct CombineParams {
@@ -51,6 +52,7 @@ struct CombineParams {
     int64_t y_rows;
     uint4 *out;
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct LocalParams {
@@ -66,6 +68,7 @@ struct LocalParams {
     int64_t part_cap;
     int part_bits;    // 32 or 16
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct EpilogueParams {
@@ -77,6 +80,7 @@ struct EpilogueParams {
     int64_t part_cap;
     uint4 *out;
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct IndexParams {
@@ -87,6 +91,7 @@ struct IndexParams {
     int32_t *src;   // [rows] recv row serving each expanded row
     int64_t rows;
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct GatherParams {
@@ -99,6 +104,7 @@ struct GatherParams {
     int64_t rows;
     uint4 *y;
     int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 struct StandinParams {
@@ -108,6 +114,7 @@ struct StandinParams {
     int E, V, vpc;
     int64_t rows;
     uint4 *y;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
 // ------------------------------------------------------------- launchers
@@ -153,6 +160,12 @@ inline int current_sm_count()
     return sm_count(dev);
 }
 
+// Programmatic-launch trigger policy: a grid that fits in about one wave
+// lets its dependents launch at once (their launch hides behind this grid);
+// a multi-wave grid triggers only after each CTA's main work, so waiting
+// dependent CTAs do not sit on the SMs through its later waves.
+inline int early_trigger(long long ctas) { return ctas <= 8LL * current_sm_count(); }
+
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;
 
@@ -188,10 +201,11 @@ cudaError_t launch_pdl(void (*kernel)(Params), dim3 grid, dim3 block, size_t sme
 // ----------------------------------------------------- device utilities
 
 // Programmatic dependent launch.  Every kernel of the path lets the next one
-// in its stream start launching right away (its prologue overlaps this
-// kernel), and waits for the previous one to finish -- with its memory
-// visible -- before it touches any global memory.  Without the launch
-// attribute both are no-ops.
+// in its stream start launching early (its launch and prologue overlap this
+// kernel: at once for one-wave grids, after the main work otherwise), and
+// waits for the previous one to finish -- with its memory visible -- before
+// it touches any global memory.  Without the launch attribute both are
+// no-ops.
 __device__ __forceinline__ void pdl_launch_dependents()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

@@ -32,7 +32,7 @@ __device__ __forceinline__ int rank_of_row(const int32_t *bound, int R, int q)
 __global__ void __launch_bounds__(256) expand_index_kernel(IndexParams p)
 {
     __shared__ int32_t s_bound[EPX_MAX_RANKS + 1];
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int i = threadIdx.x; i <= p.R; i += blockDim.x) s_bound[i] = p.off_e[i * p.epr];
     __syncthreads();
@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(256) expand_index_kernel(IndexParams p)
         const long long t = i / p.k;
         p.src[q] = p.recv_pos[t * p.R + rank_of_row(s_bound, p.R, q)];
     }
+    pdl_launch_dependents();
 }
 
 // expert owning expanded row q (largest e with off_e[e] <= q)
@@ -66,7 +67,7 @@ __device__ __forceinline__ int expert_of_row(const int32_t *off_e, int E, int q)
 
 __global__ void __launch_bounds__(128) standin_gather_kernel(GatherParams p)
 {
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     const int64_t n_route = p.totals[0];
     const int64_t rows = n_route < p.rows ? n_route : p.rows;
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(128) standin_gather_kernel(GatherParams p)
             st_v4(p.y + (size_t)row * p.V + v, make_uint4(o[0], o[1], o[2], o[3]));
         }
     }
+    pdl_launch_dependents();
 }
 
 }  // namespace
@@ -104,7 +106,9 @@ cudaError_t launch_expand_index(const IndexParams &p, cudaStream_t s)
     const long long n = (long long)p.T * p.k;
     long long blocks = (n + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    return launch_pdl(expand_index_kernel, dim3((unsigned)blocks), dim3(256), 0, s, p);
+    IndexParams q = p;
+    q.early_pdl = early_trigger(blocks);
+    return launch_pdl(expand_index_kernel, dim3((unsigned)blocks), dim3(256), 0, s, q);
 }
 
 cudaError_t launch_standin_gather(const GatherParams &p0, cudaStream_t s)
@@ -114,6 +118,7 @@ cudaError_t launch_standin_gather(const GatherParams &p0, cudaStream_t s)
     const int chunks = (p.V + 255) / 256;
     p.vpc = (p.V + chunks - 1) / chunks;
     const int64_t gy = p.rows < 65535 ? p.rows : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     return launch_pdl(standin_gather_kernel, dim3(chunks, (unsigned)gy), dim3(128), 0, s, p);
 }
 

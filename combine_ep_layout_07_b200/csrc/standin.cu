@@ -28,7 +28,7 @@ __device__ __forceinline__ int expert_of_row(const int32_t *off_e, int E, int p)
 
 __global__ void __launch_bounds__(128) standin_kernel(StandinParams p)
 {
-    pdl_launch_dependents();
+    if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     const int64_t n_route = p.totals[0];
     const int64_t rows = n_route < p.rows ? n_route : p.rows;
@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(128) standin_kernel(StandinParams p)
             st_v4(p.y + (size_t)row * p.V + v, make_uint4(o[0], o[1], o[2], o[3]));
         }
     }
+    pdl_launch_dependents();
 }
 
 }  // namespace
@@ -62,6 +63,7 @@ cudaError_t launch_standin(const StandinParams &p0, cudaStream_t s)
     const int chunks = (p.V + 255) / 256;
     p.vpc = (p.V + chunks - 1) / chunks;
     const int64_t gy = p.rows < 65535 ? p.rows : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
     return launch_pdl(standin_kernel, dim3(chunks, (unsigned)gy), dim3(128), 0, s, p);
 }
 
