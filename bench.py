@@ -82,6 +82,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["epx", "reference"], default="epx")
     ap.add_argument("--workload", choices=sorted(DESCRIBE), default="prefill")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layout-variant", type=int, default=0,
+                    help="0 automatic, 1 warp chunks, 2 count matrix")
     ap.add_argument("--dispatch-variant", type=int, default=0)
     ap.add_argument("--combine-variant", type=int, default=0)
     ap.add_argument("--idx-bits", type=int, choices=[32, 64], default=64)
@@ -406,7 +408,8 @@ def run_epx(args):
         part = torch.empty((lay.recv_cap, H), device=dev,
                            dtype=torch.float32 if args.two_stage == "fp32" else torch.bfloat16)
     src = torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev) if args.no_expand else None
-    calls = [("layout", lambda st: epx.layout(idx, E, R, out=lay, stream=st))]
+    calls = [("layout", lambda st: epx.layout(idx, E, R, out=lay, variant=args.layout_variant,
+                                              stream=st))]
     if args.no_expand:
         calls.append(("dispatch", lambda st: epx.dispatch(x, lay, recv=recv, stream=st)))
         calls.append(("expand_index", lambda st: epx.expand_index(lay, src=src, stream=st)))
@@ -433,7 +436,7 @@ def run_epx(args):
             events[len(calls)].record(st)
 
     with torch.cuda.stream(stream):
-        epx.layout(idx, E, R, out=lay, stream=stream)
+        epx.layout(idx, E, R, out=lay, variant=args.layout_variant, stream=stream)
         epx.dispatch_expand(x, lay, recv=recv, expanded=expanded, stream=stream)
         epx.standin_expert(expanded, lay, y=y, stream=stream)
     tot = epx.read_totals(lay, stream=stream)

@@ -101,9 +101,11 @@ ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E, int3
     return EP_OK;
 }
 
-ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
+ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L, int32_t variant,
+                              void *stream)
 {
     if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
     if (L->T > 0 && !topk_idx) return EP_ERR_INVALID_ARG;
     if (topk_idx && !aligned(topk_idx, (size_t)L->idx_bits / 8)) return EP_ERR_MISALIGNED;
     LayoutParams p;
@@ -121,7 +123,13 @@ ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
     p.pos = L->pos;
     p.recv_pos = L->recv_pos;
     p.totals = L->totals;
-    return from_cuda(launch_layout(p, L->idx_bits, as_stream(stream)));
+    const cudaError_t e = launch_layout(p, L->idx_bits, variant, as_stream(stream));
+    return e == cudaErrorNotSupported ? EP_ERR_UNSUPPORTED : from_cuda(e);
+}
+
+ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
+{
+    return ep_layout_variant(topk_idx, L, 0, stream);
 }
 
 ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout_t *L,

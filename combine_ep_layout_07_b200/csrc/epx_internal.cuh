@@ -24,6 +24,10 @@ struct LayoutParams {
     int tch;        // tokens per chunk (columns of the count matrix)
     int ld;         // count-matrix row length in words: odd, >= tch
     int wde, wdr;   // count-matrix rows (two 16-bit counts per 32-bit word) for experts / ranks
+    int tpw;        // warp-chunk schedule: whole tokens per warp, floor(32 / k)
+    int tstr;       // warp-chunk schedule: table row length in 16-bit counts (even, >= E + R)
+    float inv_k;    // 1.0f / k
+    int bits_e, bits_r;  // bits of the largest expert / rank
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
 };
 
@@ -121,7 +125,7 @@ struct StandinParams {
 // Each returns cudaSuccess or the launch error; arguments are already
 // validated by the C-ABI layer.
 
-cudaError_t launch_layout(const LayoutParams &p, int idx_bits, cudaStream_t s);
+cudaError_t launch_layout(const LayoutParams &p, int idx_bits, int variant, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchParams &p, int variant, cudaStream_t s);
 cudaError_t launch_standin(const StandinParams &p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);

@@ -261,63 +261,15 @@ __host__ __device__ size_t matrix_words(int wdt, int ld)
     return ((size_t)wdt * ld + 3) & ~(size_t)3;
 }
 
-template <typename IdxT, bool CLUSTER>
-__global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
+// Cluster exchange of the CTA totals in sm.tot (and sm.misc), then one packed
+// 64-bit block scan: writes cnt / off / totals (CTA 0) and this CTA's first
+// row per expert and rank into sm.base.  Ends without a barrier.
+template <bool CLUSTER>
+__device__ void global_offsets(const LayoutParams &p, const Smem &sm, int crank, int csize)
 {
-    extern __shared__ __align__(16) int32_t smem[];
     const int tid = threadIdx.x;
-    const int E = p.E, R = p.R, T = p.T;
-    pdl_launch_dependents();
-
-    int crank = 0, csize = 1;
-    if (CLUSTER) {
-        cg::cluster_group cluster = cg::this_cluster();
-        crank = (int)cluster.block_rank();
-        csize = (int)cluster.num_blocks();
-    }
-
+    const int E = p.E, R = p.R;
     const int W = E + R + 2;
-    const int wdt = p.wde + p.wdr;
-    Smem sm;
-    sm.M = reinterpret_cast<uint32_t *>(smem);
-    sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.ld));
-    sm.scan = sm.hit + p.tch;
-    sm.codes = reinterpret_cast<int32_t *>(sm.scan + 34);
-    sm.tot = sm.codes + (size_t)p.tch * p.k;
-    sm.base = sm.tot + E + R;
-    sm.all_tot = sm.base + E + R;
-    sm.misc = sm.all_tot + (size_t)csize * W;
-
-    const IdxT *idx = static_cast<const IdxT *>(p.idx);
-    const int c0 = min(T, crank * p.tpc);
-    const int nt = min(T, c0 + p.tpc) - c0;
-    const int nchunks = (nt + p.tch - 1) / p.tch;
-    bool bad = false;
-    int nreal = 0;
-
-    // prologue in shared memory only, so it may overlap the previous kernel
-    if (tid < 2) sm.misc[tid] = 0;
-    if (nchunks <= 1) {
-        zero_words(sm.M, wdt * p.ld);
-    } else {
-        for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
-    }
-    __syncthreads();
-    // peers write into this CTA's shared memory only once every CTA runs
-    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-    pdl_wait_previous();
-
-    if (nchunks <= 1) {
-        nreal = build_tokens(p, idx, c0, nt, sm, false, &bad);
-        __syncthreads();
-        row_scan(p, sm, nt);
-    } else {
-        nreal = build_tokens(p, idx, c0, nt, sm, true, &bad);
-    }
-    if (__any_sync(kFull, bad) && (tid & 31) == 0) atomicOr(&sm.misc[0], 1);
-    if (nreal) atomicAdd(&sm.misc[1], nreal);
-    __syncthreads();
-
     // ---- cluster exchange: push this CTA's totals into row crank of every
     // CTA's table (distributed shared memory stores), then read locally
     if (CLUSTER) {
@@ -407,6 +359,66 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
             p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
         }
     }
+}
+
+template <typename IdxT, bool CLUSTER>
+__global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
+{
+    extern __shared__ __align__(16) int32_t smem[];
+    const int tid = threadIdx.x;
+    const int E = p.E, R = p.R, T = p.T;
+    pdl_launch_dependents();
+
+    int crank = 0, csize = 1;
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        crank = (int)cluster.block_rank();
+        csize = (int)cluster.num_blocks();
+    }
+
+    const int W = E + R + 2;
+    const int wdt = p.wde + p.wdr;
+    Smem sm;
+    sm.M = reinterpret_cast<uint32_t *>(smem);
+    sm.hit = reinterpret_cast<unsigned long long *>(smem + matrix_words(wdt, p.ld));
+    sm.scan = sm.hit + p.tch;
+    sm.codes = reinterpret_cast<int32_t *>(sm.scan + 34);
+    sm.tot = sm.codes + (size_t)p.tch * p.k;
+    sm.base = sm.tot + E + R;
+    sm.all_tot = sm.base + E + R;
+    sm.misc = sm.all_tot + (size_t)csize * W;
+
+    const IdxT *idx = static_cast<const IdxT *>(p.idx);
+    const int c0 = min(T, crank * p.tpc);
+    const int nt = min(T, c0 + p.tpc) - c0;
+    const int nchunks = (nt + p.tch - 1) / p.tch;
+    bool bad = false;
+    int nreal = 0;
+
+    // prologue in shared memory only, so it may overlap the previous kernel
+    if (tid < 2) sm.misc[tid] = 0;
+    if (nchunks <= 1) {
+        zero_words(sm.M, wdt * p.ld);
+    } else {
+        for (int i = tid; i < E + R; i += blockDim.x) sm.tot[i] = 0;
+    }
+    __syncthreads();
+    // peers write into this CTA's shared memory only once every CTA runs
+    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pdl_wait_previous();
+
+    if (nchunks <= 1) {
+        nreal = build_tokens(p, idx, c0, nt, sm, false, &bad);
+        __syncthreads();
+        row_scan(p, sm, nt);
+    } else {
+        nreal = build_tokens(p, idx, c0, nt, sm, true, &bad);
+    }
+    if (__any_sync(kFull, bad) && (tid & 31) == 0) atomicOr(&sm.misc[0], 1);
+    if (nreal) atomicAdd(&sm.misc[1], nreal);
+    __syncthreads();
+
+    global_offsets<CLUSTER>(p, sm, crank, csize);
     __syncthreads();
 
     // ---- positions
@@ -428,6 +440,175 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
         __syncthreads();
         for (int i = tid; i < E + R; i += blockDim.x) sm.base[i] += sm.tot[i];
         __syncthreads();
+    }
+}
+
+// ------------------------------------------------------ warp-chunk schedule
+//
+// A warp takes tpw = floor(32 / k) whole tokens, one lane per route in
+// (token, slot) order, so the warp's routes form one chunk of the CTA's
+// tokens.  Inside the warp, lanes with equal experts are found with one
+// ballot per bit of the expert (match_bits): a route's rank among the warp's
+// earlier routes to its expert (from earlier tokens and from earlier slots of
+// its own token alike) is the population count of its group below its lane,
+// and the group's lowest lane stores the group size into the warp's row of a
+// chunk x (expert | rank) count table of 16-bit counts.  The same on the
+// rank marks the first route of each (token, rank) pair (no lower lane of
+// its token has its rank) and ranks those first routes.  One thread per
+// table word (two 16-bit columns) then rewrites its column as an exclusive
+// prefix over the chunks, so that
+//     pos = base[e] + prefix[chunk][e] + rank in warp
+// and the same for recv_pos with the rank columns; base comes from the
+// cluster exchange and global scan shared with the count-matrix schedule.
+// Each lane keeps its routes in registers (one per pass of the CTA's warps
+// over its tokens), so nothing walks the tokens serially.  The CTA has as
+// few warps as keep the passes at four or fewer: the phases are short and
+// separated by barriers, and every barrier and every shared-memory phase is
+// cheaper with fewer warps.
+
+// Lanes of the warp whose `key` equals this lane's, among `active` lanes;
+// `bits` covers every key value.  One ballot per bit (match.any is a slow
+// instruction on this part).
+__device__ __forceinline__ unsigned match_bits(unsigned key, int bits, unsigned active)
+{
+    unsigned m = active;
+    for (int b = 0; b < bits; ++b) {
+        const bool set = (key >> b) & 1u;
+        const unsigned bb = __ballot_sync(kFull, set);
+        m &= set ? bb : ~bb;
+    }
+    return m;
+}
+
+__host__ __device__ size_t warp_table_words(int nch, int wt)
+{
+    return ((size_t)nch * wt + 3) & ~(size_t)3;
+}
+
+template <typename IdxT, bool CLUSTER, int PASSES>
+__global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
+{
+    extern __shared__ __align__(16) int32_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int NW = blockDim.x >> 5;
+    const int E = p.E, R = p.R, T = p.T, k = p.k, tpw = p.tpw;
+    pdl_launch_dependents();
+
+    int crank = 0, csize = 1;
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        crank = (int)cluster.block_rank();
+        csize = (int)cluster.num_blocks();
+    }
+    const int W = E + R + 2;
+    const int wt = p.tstr >> 1;  // table row length in 32-bit words
+    const int nch_max = (p.tpc + tpw - 1) / tpw;
+
+    uint32_t *tab = reinterpret_cast<uint32_t *>(smem);  // [chunks][wt]
+    Smem sm;
+    sm.M = nullptr;
+    sm.codes = nullptr;
+    sm.hit = nullptr;
+    sm.scan = reinterpret_cast<unsigned long long *>(smem + warp_table_words(nch_max, wt));
+    sm.tot = reinterpret_cast<int32_t *>(sm.scan + 34);
+    sm.base = sm.tot + E + R;
+    sm.all_tot = sm.base + E + R;
+    sm.misc = sm.all_tot + (size_t)csize * W;
+
+    const IdxT *idx = static_cast<const IdxT *>(p.idx);
+    const int c0 = min(T, crank * p.tpc);
+    const int nt = min(T, c0 + p.tpc) - c0;
+    const int nuse = (nt + tpw - 1) / tpw;  // chunks holding tokens
+
+    // prologue in shared memory only, so it may overlap the previous kernel
+    if (tid < 2) sm.misc[tid] = 0;
+    zero_words(tab, nuse * wt);
+    __syncthreads();
+    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pdl_wait_previous();
+
+    const int tl = div_small(lane, p.inv_k);  // token of this lane within its chunk
+    const int j = lane - tl * k;              // slot
+    const unsigned lt = lanemask_lt();
+    IdxT raw[PASSES];
+#pragma unroll
+    for (int q = 0; q < PASSES; ++q) {
+        const int u = (q * NW + wid) * tpw + tl;
+        raw[q] = (tl < tpw && u < nt) ? idx[(size_t)(c0 + u) * k + j] : (IdxT)-1;
+    }
+    // (token, rank) pairs nobody reaches read -1: fill this CTA's rows first
+    if ((R & 3) == 0) {
+        int4 *dst = reinterpret_cast<int4 *>(p.recv_pos + (size_t)c0 * R);
+        for (int i = tid; i < (nt * R) >> 2; i += blockDim.x) dst[i] = make_int4(-1, -1, -1, -1);
+    } else {
+        for (int i = tid; i < nt * R; i += blockDim.x) p.recv_pos[(size_t)c0 * R + i] = -1;
+    }
+
+    bool bad = false;
+    int nreal = 0;
+    int re_e[PASSES], re_r[PASSES], rk[PASSES], ex[PASSES];
+    const unsigned kmask = k == 32 ? kFull : ((1u << k) - 1u);
+    const unsigned tokmask = tl < tpw ? kmask << (tl * k) : 0u;  // lanes of this lane's token
+#pragma unroll
+    for (int q = 0; q < PASSES; ++q) {
+        const int c = q * NW + wid;
+        const long long ev = (long long)raw[q];
+        bad |= (ev < -1 || ev >= E);
+        const bool v = ev >= 0 && ev < E;
+        const int e = v ? (int)ev : 0;
+        const int r = v ? rank_of(e, p.inv_epr) : 0;
+        const unsigned vb = __ballot_sync(kFull, v);
+        const unsigned pe = match_bits((unsigned)e, p.bits_e, vb);
+        const unsigned pr = match_bits((unsigned)r, p.bits_r, vb);
+        const bool first = v && !(pr & tokmask & lt);
+        const unsigned pf = pr & __ballot_sync(kFull, first);
+        uint16_t *row = reinterpret_cast<uint16_t *>(tab + (size_t)c * wt);
+        if (v && !(pe & lt)) row[e] = (uint16_t)__popc(pe);
+        if (first && !(pf & lt)) row[E + r] = (uint16_t)__popc(pf);
+        nreal += j == 0 && (vb & tokmask) != 0u;
+        ex[q] = v ? e : -1;
+        re_e[q] = __popc(pe & lt);
+        rk[q] = first ? r : -1;
+        re_r[q] = __popc(pf & lt);
+    }
+    __syncthreads();
+
+    // exclusive prefix of every table column over the chunks (two packed
+    // 16-bit columns per word add independently); the sums are the CTA totals
+    for (int w = tid; w < wt; w += blockDim.x) {
+        uint32_t run = 0;
+        for (int c = 0; c < nuse; c += 8) {
+            uint32_t v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = c + i < nuse ? tab[(size_t)(c + i) * wt + w] : 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (c + i < nuse) tab[(size_t)(c + i) * wt + w] = run;
+                run += v[i];
+            }
+        }
+        if (2 * w < E + R) sm.tot[2 * w] = (int32_t)(run & 0xffffu);
+        if (2 * w + 1 < E + R) sm.tot[2 * w + 1] = (int32_t)(run >> 16);
+    }
+    if (__any_sync(kFull, bad) && lane == 0) atomicOr(&sm.misc[0], 1);
+    if (nreal) atomicAdd(&sm.misc[1], nreal);
+    __syncthreads();
+
+    global_offsets<CLUSTER>(p, sm, crank, csize);
+    __syncthreads();
+
+#pragma unroll
+    for (int q = 0; q < PASSES; ++q) {
+        const int c = q * NW + wid;
+        const int u = c * tpw + tl;
+        if (tl < tpw && u < nt) {
+            const uint16_t *row = reinterpret_cast<const uint16_t *>(tab + (size_t)c * wt);
+            const int e = ex[q];
+            p.pos[(size_t)(c0 + u) * k + j] = e < 0 ? -1 : sm.base[e] + (int)row[e] + re_e[q];
+            const int r = rk[q];
+            if (r >= 0)
+                p.recv_pos[(size_t)(c0 + u) * R + r] = sm.base[E + r] + (int)row[E + r] + re_r[q];
+        }
     }
 }
 
@@ -477,23 +658,75 @@ Geometry plan(int T, int k, int E, int R, int csize)
     return g;
 }
 
-template <typename IdxT>
-int max_clusters(int csize, size_t smem, int dev)
+// Warp-chunk geometry: tokens per warp and per CTA, passes, table row
+// length, shared memory; false when the table does not fit or more than
+// four passes would be needed (the count-matrix schedule covers those).
+struct WarpGeometry {
+    int csize, tpc, tpw, passes, threads, tstr;
+    size_t smem;
+};
+
+int bits_for(int n)  // bits of the largest value below n (at least 1)
+{
+    int b = 1;
+    while ((1 << b) < n) ++b;
+    return b;
+}
+
+bool plan_warp(int T, int k, int E, int R, int csize, WarpGeometry *g)
+{
+    g->tpw = 32 / k;
+    g->tstr = (E + R + 1) & ~1;
+    // the global scan gives each thread at most four experts, and one rank
+    int min_threads = (E + 3) / 4 > R ? (E + 3) / 4 : R;
+    min_threads = ((min_threads + 31) / 32) * 32;
+    for (;; csize >>= 1) {
+        g->csize = csize;
+        g->tpc = (T + csize - 1) / csize;
+        const int nch = (g->tpc + g->tpw - 1) / g->tpw;
+        // fewest warps (of 8, 16 or 32) that need no more than four passes
+        int warps = 8;
+        while (warps < 32 && nch > 4 * warps) warps *= 2;
+        if (warps * 32 < min_threads) warps = (min_threads + 31) / 32;
+        const int passes = (nch + warps - 1) / warps;
+        g->threads = warps * 32;
+        g->passes = passes <= 1 ? 1 : passes <= 2 ? 2 : 4;
+        g->smem = warp_table_words(nch, g->tstr >> 1) * 4 + fixed_bytes(E, R, csize);
+        if (passes <= 4 && g->smem <= (size_t)kMaxDynSmem) return true;
+        if (csize == 1 || passes > 4) return false;
+    }
+}
+
+using LayoutKernel = void (*)(LayoutParams);
+
+template <typename IdxT, bool CLUSTER>
+LayoutKernel warp_kernel(int passes)
+{
+    return passes == 1   ? layout_warp_kernel<IdxT, CLUSTER, 1>
+           : passes == 2 ? layout_warp_kernel<IdxT, CLUSTER, 2>
+                         : layout_warp_kernel<IdxT, CLUSTER, 4>;
+}
+
+// largest number of co-resident clusters of `csize` CTAs of `fn` (0 when a
+// cluster of that size with that much shared memory cannot be placed)
+int max_clusters(LayoutKernel fn, int csize, int threads, size_t smem, int dev)
 {
     struct Entry {
-        int dev, csize;
+        LayoutKernel fn;
+        int dev, csize, threads;
         size_t smem;
         int result;
     };
-    static Entry cache[64];
+    static Entry cache[128];
     static int n_cache = 0;
     std::lock_guard<std::mutex> lock(launcher_mutex());
     for (int i = 0; i < n_cache; ++i)
-        if (cache[i].dev == dev && cache[i].csize == csize && cache[i].smem == smem)
+        if (cache[i].fn == fn && cache[i].dev == dev && cache[i].csize == csize &&
+            cache[i].threads == threads && cache[i].smem == smem)
             return cache[i].result;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(csize, 1, 1);
-    cfg.blockDim = dim3(1024, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -503,11 +736,11 @@ int max_clusters(int csize, size_t smem, int dev)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, layout_kernel<IdxT, true>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
-    if (n_cache < 64) cache[n_cache++] = Entry{dev, csize, smem, n};
+    if (n_cache < 128) cache[n_cache++] = Entry{fn, dev, csize, threads, smem, n};
     return n;
 }
 
@@ -516,21 +749,31 @@ cudaError_t set_attributes_once(int dev)
 {
     static std::atomic<unsigned> done{0};  // per device (up to 32)
     if (dev < 32 && (done.load() & (1u << dev))) return cudaSuccess;
-    cudaError_t err = cudaFuncSetAttribute(layout_kernel<IdxT, false>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kMaxDynSmem);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(layout_kernel<IdxT, true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(layout_kernel<IdxT, true>,
-                                   cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    const LayoutKernel single[] = {layout_kernel<IdxT, false>, warp_kernel<IdxT, false>(1),
+                                   warp_kernel<IdxT, false>(2), warp_kernel<IdxT, false>(4)};
+    const LayoutKernel clustered[] = {layout_kernel<IdxT, true>, warp_kernel<IdxT, true>(1),
+                                      warp_kernel<IdxT, true>(2), warp_kernel<IdxT, true>(4)};
+    cudaError_t err = cudaSuccess;
+    for (LayoutKernel fn : single)
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxDynSmem);
+    for (LayoutKernel fn : clustered) {
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxDynSmem);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    }
     if (err == cudaSuccess && dev < 32) done.fetch_or(1u << dev);
     return err;
 }
 
+// variant: 0 = warp chunks where they fit, else the count matrix;
+// 1 = warp chunks (cudaErrorNotSupported where they do not fit);
+// 2 = count matrix
 template <typename IdxT>
-cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
+cudaError_t launch_layout_t(const LayoutParams &p0, int variant, cudaStream_t s)
 {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -543,8 +786,33 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
     // one CTA up to ~2K routes, then a cluster of up to 16 CTAs
     int csize = (int)((routes + 2047) / 2048);
     csize = csize < 1 ? 1 : (csize > 16 ? 16 : csize);
+
+    if (variant != 2) {
+        WarpGeometry g;
+        bool ok = plan_warp(p.T, p.k, p.E, p.R, csize, &g);
+        while (ok && g.csize > 1 &&
+               max_clusters(warp_kernel<IdxT, true>(g.passes), g.csize, g.threads, g.smem,
+                            dev) == 0)
+            ok = plan_warp(p.T, p.k, p.E, p.R, g.csize > 8 ? 8 : g.csize >> 1, &g);
+        if (ok) {
+            p.tpc = g.tpc;
+            p.tpw = g.tpw;
+            p.tstr = g.tstr;
+            p.inv_k = 1.0f / (float)p.k;
+            p.bits_e = bits_for(p.E);
+            p.bits_r = bits_for(p.R);
+            if (g.csize == 1)
+                return launch_pdl(warp_kernel<IdxT, false>(g.passes), dim3(1), dim3(g.threads),
+                                  g.smem, s, p);
+            return launch_pdl(warp_kernel<IdxT, true>(g.passes), dim3(g.csize), dim3(g.threads),
+                              g.smem, s, p, g.csize);
+        }
+        if (variant == 1) return cudaErrorNotSupported;
+    }
+
     Geometry g = plan(p.T, p.k, p.E, p.R, csize);
-    while (g.csize > 1 && max_clusters<IdxT>(g.csize, g.smem, dev) == 0)
+    while (g.csize > 1 &&
+           max_clusters(layout_kernel<IdxT, true>, g.csize, 1024, g.smem, dev) == 0)
         g = plan(p.T, p.k, p.E, p.R, g.csize > 8 ? 8 : g.csize >> 1);
     p.tpc = g.tpc;
     p.tch = g.tch;
@@ -559,9 +827,10 @@ cudaError_t launch_layout_t(const LayoutParams &p0, cudaStream_t s)
 
 }  // namespace
 
-cudaError_t launch_layout(const LayoutParams &p, int idx_bits, cudaStream_t s)
+cudaError_t launch_layout(const LayoutParams &p, int idx_bits, int variant, cudaStream_t s)
 {
-    return idx_bits == 64 ? launch_layout_t<long long>(p, s) : launch_layout_t<int>(p, s);
+    return idx_bits == 64 ? launch_layout_t<long long>(p, variant, s)
+                          : launch_layout_t<int>(p, variant, s);
 }
 
 }  // namespace epx

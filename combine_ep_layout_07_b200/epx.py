@@ -73,6 +73,7 @@ def lib():
         "ep_layout_bytes": ([I32, I32, I32, I32], SZ),
         "ep_layout_init": ([LP, I32, I32, I32, I32, I32, P, SZ], I32),
         "ep_layout": ([P, LP, P], I32),
+        "ep_layout_variant": ([P, LP, I32, P], I32),
         "ep_dispatch_expand": ([P, I32, LP, P, I64, P, I64, P], I32),
         "ep_dispatch_expand_variant": ([P, I32, LP, P, I64, P, I64, I32, P], I32),
         "ep_standin_expert": ([P, I32, LP, P, I64, P], I32),
@@ -159,8 +160,9 @@ class Layout:
 
 
 def layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, out: Layout = None,
-           stream=None) -> Layout:
-    """ep_layout: routing layout of topk_idx (int32 or int64 [T, k], -1 = none)."""
+           variant: int = 0, stream=None) -> Layout:
+    """ep_layout: routing layout of topk_idx (int32 or int64 [T, k], -1 = none).
+    variant: 0 automatic, 1 warp chunks, 2 count matrix (same results)."""
     if topk_idx.dim() != 2:
         raise ValueError("topk_idx must be [T, k]")
     T, k = topk_idx.shape
@@ -172,7 +174,7 @@ def layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, out: Layout
                                              device=topk_idx.device)
     if (lay.T, lay.k, lay.E, lay.R, lay.idx_bits) != (T, k, num_experts, num_ranks, bits):
         raise ValueError("layout buffer does not match the sizes")
-    _check(lib().ep_layout(ptr, lay.ref, _stream(stream)), "ep_layout")
+    _check(lib().ep_layout_variant(ptr, lay.ref, variant, _stream(stream)), "ep_layout")
     return lay
 
 

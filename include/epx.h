@@ -59,7 +59,8 @@ typedef enum ep_status {
     EP_ERR_CAPACITY = 3,    /* device: a destination row exceeded a capacity  */
     EP_ERR_BAD_INDEX = 4,   /* device: a topk index < -1 or >= E was skipped  */
     EP_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed           */
-    EP_ERR_UNSUPPORTED = 6  /* size beyond a documented EPX_MAX_* limit       */
+    EP_ERR_UNSUPPORTED = 6  /* size beyond a documented limit (EPX_MAX_*, or  */
+                            /* of a schedule chosen by a *_variant call)      */
 } ep_status_t;
 
 /* bits of the device error word, totals[3] */
@@ -124,6 +125,15 @@ ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E,
  * cluster whose CTAs share histograms through distributed shared memory).
  */
 ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream);
+
+/* Same, choosing the schedule: 0 = automatic, 1 = warp chunks (each warp
+ * takes whole tokens, one lane per route, and ranks routes with warp match
+ * instructions; EP_ERR_UNSUPPORTED when its per-warp count table does not
+ * fit in shared memory or the CTA's tokens need more than four passes of
+ * its warps), 2 = count matrix (one thread per token; any valid size).
+ * Results are identical. */
+ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
+                              int32_t variant, void *stream);
 
 /*
  * Dispatch + expand.  x: device bf16 [T, H] row-major (16-byte aligned,

@@ -35,9 +35,10 @@ def gpu_inputs(wl, idx_dtype=torch.int64):
     return x, idx, w
 
 
-def run_gpu(wl, idx_dtype=torch.int64, dispatch_variant=0, combine_variant=0, y_override=None):
+def run_gpu(wl, idx_dtype=torch.int64, dispatch_variant=0, combine_variant=0, y_override=None,
+            layout_variant=0):
     x, idx, w = gpu_inputs(wl, idx_dtype)
-    lay = epx.layout(idx, wl["E"], wl["R"])
+    lay = epx.layout(idx, wl["E"], wl["R"], variant=layout_variant)
     recv, expanded = epx.dispatch_expand(x, lay, variant=dispatch_variant)
     y = epx.standin_expert(expanded, lay)
     y_in = y if y_override is None else y_override
@@ -47,7 +48,7 @@ def run_gpu(wl, idx_dtype=torch.int64, dispatch_variant=0, combine_variant=0, y_
 
 
 def assert_layout_equal(g, o):
-    lay = g["layout"] if "layout" in g else g
+    lay = g["layout"] if isinstance(g, dict) else g
     np.testing.assert_array_equal(lay.cnt_e.cpu().numpy(), o["cnt_e"])
     np.testing.assert_array_equal(lay.off_e.cpu().numpy(), o["off_e"])
     np.testing.assert_array_equal(lay.cnt_r.cpu().numpy(), o["cnt_r"])

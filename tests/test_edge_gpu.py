@@ -8,7 +8,8 @@ import oracle
 from combine_ep_layout_07_b200 import epx
 from combine_ep_layout_07_b200 import workloads as wlmod
 
-from gpu_helpers import assert_all_equal, assert_combine_close, run_gpu, torch_to_bits
+from gpu_helpers import (assert_all_equal, assert_combine_close, assert_layout_equal, run_gpu,
+                         torch_to_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -52,6 +53,51 @@ def test_random_shapes(case, dv):
     wl = _random_wl(seed=case["T"] + case["E"], p_pad=0.2, **case)
     for cv in (1, 2):
         _check(wl, dispatch_variant=dv, combine_variant=cv)
+
+
+# shapes for both layout schedules: k not dividing 32 (idle lanes), k = 32,
+# R not a multiple of 4 (scalar -1 fill), several passes of the warps, a
+# cluster with a ragged last CTA, duplicates and bad indices in one batch
+LAYOUT_CASES = [
+    dict(T=1, H=8, E=1, R=1, k=1),
+    dict(T=33, H=8, E=12, R=3, k=3),
+    dict(T=300, H=8, E=60, R=6, k=6),
+    dict(T=77, H=8, E=64, R=4, k=32),
+    dict(T=3000, H=8, E=70, R=7, k=7),
+    dict(T=5, H=8, E=8, R=8, k=1),
+    dict(T=960, H=8, E=256, R=16, k=8),
+    dict(T=8192, H=8, E=256, R=16, k=8),
+]
+
+
+@pytest.mark.parametrize("case", LAYOUT_CASES, ids=lambda c: "T{T}k{k}E{E}R{R}".format(**c))
+@pytest.mark.parametrize("lv", [1, 2])
+def test_layout_schedules_shapes(case, lv):
+    wl = _random_wl(seed=case["T"] * 3 + case["k"], p_pad=0.2, distinct=False, **case)
+    idx = wl["topk_idx"]
+    if case["T"] > 3:
+        idx[2, 0] = case["E"] + 5      # bad index: dropped and flagged
+        idx[3, :] = -1                 # all-padding row
+    if case["T"] > 1 and case["k"] > 1:
+        idx[1, 1] = idx[1, 0]          # same expert twice in one token
+    lay_o = oracle.layout(idx, case["E"], case["R"])
+    lay = epx.layout(torch.from_numpy(idx).cuda(), case["E"], case["R"], variant=lv)
+    torch.cuda.synchronize()
+    assert_layout_equal(lay, lay_o)
+
+
+def test_layout_warp_schedule_unsupported_shape():
+    # the per-warp count table of E = 4096, R = 64 for 129 tokens of top-5
+    # does not fit in shared memory: variant 1 refuses, auto and 2 agree
+    wl = _random_wl(T=129, H=8, E=4096, R=64, k=5, seed=9)
+    idx = torch.from_numpy(wl["topk_idx"]).cuda()
+    with pytest.raises(RuntimeError, match="UNSUPPORTED|unsupported"):
+        epx.layout(idx, 4096, 64, variant=1)
+    lay_o = oracle.layout(wl["topk_idx"], 4096, 64)
+    for lv in (0, 2):
+        lay = epx.layout(idx, 4096, 64, variant=lv)
+        torch.cuda.synchronize()
+        assert_layout_equal(lay, lay_o)
 
 
 def test_duplicates_within_row():

@@ -3,8 +3,8 @@
 Layout, recv, expanded and the stand-in expert output are compared bit for
 bit; the combine output elementwise within |gpu - oracle| <= 2^-7 |oracle| + 1e-3.
 All five workloads (the low-batch one at T = 1, 2, 4, 8; the DP batch compact
-and padded) at their full sizes, seeds 0-2, both index widths, both copy
-engines and both combine schedules.
+and padded) at their full sizes, seeds 0-2, both index widths, both layout
+schedules, both copy engines and both combine schedules.
 """
 import numpy as np
 import pytest
@@ -43,6 +43,20 @@ def test_other_seeds(name, seed):
 def test_int32_indices(name):
     wl, o = oracle_run(name, 0)
     assert_all_equal(run_gpu(wl, idx_dtype=torch.int32), o)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("name", ALL)
+def test_layout_schedules(name, variant):
+    wl, o = oracle_run(name, 0)
+    assert_all_equal(run_gpu(wl, layout_variant=variant), o)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("name", ["decode", "prefill", "lowbatch8"])
+def test_layout_schedules_int32(name, variant):
+    wl, o = oracle_run(name, 1)
+    assert_all_equal(run_gpu(wl, idx_dtype=torch.int32, layout_variant=variant), o)
 
 
 @pytest.mark.parametrize("variant", [1, 2])
