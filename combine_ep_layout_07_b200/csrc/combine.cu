@@ -152,6 +152,11 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     const int max_chunks = (p.V + 31) / 32;
     if (chunks > max_chunks) chunks = max_chunks;
     if (chunks < 1) chunks = 1;
+    // when one vector per thread fits in one wave (seven 128-thread CTAs
+    // per SM at this kernel's register count), take it: a thread's second
+    // vector would wait for its first one's loads
+    const int one_each = (p.V + 127) / 128;
+    if (chunks < one_each && (long long)p.T * one_each <= 7ll * nsm) chunks = one_each;
     p.vpc = (p.V + chunks - 1) / chunks;
     chunks = (p.V + p.vpc - 1) / p.vpc;
     int threads = p.vpc < 128 ? ((p.vpc + 31) / 32) * 32 : 128;
