@@ -161,7 +161,7 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     chunks = (p.V + p.vpc - 1) / p.vpc;
     int threads = p.vpc < 128 ? ((p.vpc + 31) / 32) * 32 : 128;
     const int gy = p.T < 65535 ? p.T : 65535;
-    p.early_pdl = early_trigger((long long)chunks * gy);
+    p.early_pdl = early_trigger((long long)chunks * gy, 1024 / threads > 16 ? 16 : 1024 / threads);
     if (big_k)
         return launch_pdl(combine_split_kernel<16>, dim3(chunks, gy), dim3(threads), 0, s, p);
     return launch_pdl(combine_split_kernel<8>, dim3(chunks, gy), dim3(threads), 0, s, p);

@@ -232,15 +232,19 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
         p.early_pdl = early_trigger((long long)chunks * gy);
         return launch_pdl(dispatch_bulk_kernel, dim3(chunks, gy), dim3(32), smem, s, p);
     }
-    // vector engine: 128 threads x 2 vectors per pass
-    int chunks = (4 * nsm + p.T - 1) / p.T;
-    const int max_chunks = (p.V + 255) / 256;
+    // vector engine: up to 128 threads x 2 vectors per pass.  Small batches
+    // split the row into chunks of down to 64 vectors (one warp) so that the
+    // stores of a few tokens spread over ~16 CTAs per SM rather than a few SMs
+    int chunks = (16 * nsm + p.T - 1) / p.T;
+    const int max_chunks = (p.V + 63) / 64;
     if (chunks > max_chunks) chunks = max_chunks;
     if (chunks < 1) chunks = 1;
     p.vpc = (p.V + chunks - 1) / chunks;
     chunks = (p.V + p.vpc - 1) / p.vpc;
-    p.early_pdl = early_trigger((long long)chunks * gy);
-    return launch_pdl(dispatch_vec_kernel<2, false>, dim3(chunks, gy), dim3(128), 0, s, p);
+    int threads = ((p.vpc + 1) / 2 + 31) / 32 * 32;
+    if (threads > 128) threads = 128;
+    p.early_pdl = early_trigger((long long)chunks * gy, 1024 / threads > 16 ? 16 : 1024 / threads);
+    return launch_pdl(dispatch_vec_kernel<2, false>, dim3(chunks, gy), dim3(threads), 0, s, p);
 }
 
 }  // namespace epx

@@ -167,8 +167,13 @@ inline int current_sm_count()
 // Programmatic-launch trigger policy: a grid that fits in about one wave
 // lets its dependents launch at once (their launch hides behind this grid);
 // a multi-wave grid triggers only after each CTA's main work, so waiting
-// dependent CTAs do not sit on the SMs through its later waves.
-inline int early_trigger(long long ctas) { return ctas <= 8LL * current_sm_count(); }
+// dependent CTAs do not sit on the SMs through its later waves.  per_sm is
+// how many of the grid's CTAs count as one wave's share of an SM (8 for
+// 128-thread CTAs; more for smaller CTAs that shared memory does not limit).
+inline int early_trigger(long long ctas, int per_sm = 8)
+{
+    return ctas <= (long long)per_sm * current_sm_count();
+}
 
 // maximum dynamic shared memory per block that the layout kernel may use
 constexpr int kMaxDynSmem = 227 * 1024;
