@@ -562,7 +562,8 @@ def run_epx(args):
               "combine_epilogue": "two_stage_" + str(args.two_stage),
               "dispatch_expand": "bulk" if args.dispatch_variant == 2 or
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
-              "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split"}
+              "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split",
+              "layout": "count_matrix" if args.layout_variant == 2 else "warp_chunks"}
     traffic = committed_traffic(dom, args.workload, engine.get(dom))
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
