@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -272,6 +273,27 @@ def slice_workload(wl, n):
     return out
 
 
+def host_cpu():
+    """CPU model and logical core count of this host (for the oracle's timing)."""
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
+def step_stats(step_ms):
+    """Median and 10th / 90th percentiles of the per-step times, in µs."""
+    a = np.sort(np.asarray(step_ms, dtype=np.float64)) * 1e3
+    pick = lambda q: float(a[min(len(a) - 1, int(round(q * (len(a) - 1))))])
+    return {"median": pick(0.5), "p10": pick(0.1), "p90": pick(0.9)}
+
+
 def cpu_baseline(wl, budget_s, idx_bits):
     """Oracle, as it stands, over the full workload repeated for ~budget_s."""
     import oracle
@@ -289,7 +311,7 @@ def cpu_baseline(wl, budget_s, idx_bits):
         if el >= budget_s:
             break
     value = lay["T_real"] * passes / el
-    return dict(value=value, unit=UNIT, cores=1, kind="oracle",
+    return dict(value=value, unit=UNIT, cores=1, kind="oracle", host=host_cpu(),
                 sample=f"{passes} full pass(es) of the {wl['name']} workload "
                        f"({lay['T_real']} effective tokens each) in {el:.1f} s, "
                        f"single-threaded C, layout+dispatch/expand+combine"), \
@@ -343,7 +365,7 @@ def run_reference(args):
         "data": "synthetic", "config": dict(workload_config(wl, args, slay),
                                             launch="host CPU, single thread"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -451,8 +473,13 @@ def run_epx(args):
     working = bytes_["total"]
     flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
-    flush_desc = ("L2 flushed between steps (256 MiB write, outside the timed events)" if flush
-                  else f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)")
+    if flush:
+        flush_desc = "L2 flushed between steps (256 MiB write, outside the timed events)"
+    elif working >= 2 * L2_BYTES:
+        flush_desc = f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)"
+    else:
+        flush_desc = (f"hot L2: no flush between steps ({working / 1e6:.0f} MB moved per step, "
+                      f"below 2x L2)")
 
     graph = graph_k = None
     gev = gks = None
@@ -579,6 +606,7 @@ def run_epx(args):
         "config": workload_config(wl, args, tot, flush_desc),
         "roofline": roofline,
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
+        "step_us": step_stats(step_ms),
         "kernels": kernels,
         "gpu_launches": len(calls) * args.steps,
         **({"consumer": consumer} if consumer else {}),

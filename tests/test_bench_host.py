@@ -63,3 +63,16 @@ def test_default_arguments_fit_the_contract():
     a = bench.parse_args([])
     assert a.gpus == 1 and a.warmup >= 3 and a.steps > 0 and a.impl == "epx"
     assert a.workload == "prefill"
+
+
+def test_step_stats_percentiles():
+    # 1..101 ms: median 51, p10 11, p90 91 (nearest rank), reported in µs
+    st = bench.step_stats([float(i) for i in range(101, 0, -1)])
+    assert st == {"median": 51000.0, "p10": 11000.0, "p90": 91000.0}
+    assert bench.step_stats([0.25]) == {"median": 250.0, "p10": 250.0, "p90": 250.0}
+
+
+def test_host_cpu_reports_model_and_cores():
+    h = bench.host_cpu()
+    assert isinstance(h["model"], str)
+    assert h["nproc"] == os.cpu_count()

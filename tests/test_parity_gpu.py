@@ -121,3 +121,26 @@ def test_deterministic_across_runs(name):
         np.testing.assert_array_equal(g["layout"].recv_pos.cpu().numpy(), rp0)
         for k, n in rows.items():
             np.testing.assert_array_equal(torch_to_bits(g[k][:n]), ref[k])
+
+
+@pytest.mark.parametrize("layout_variant", [0, 2])
+def test_dp_compact_and_padded_agree_on_gpu(layout_variant):
+    # the same 127 real tokens laid out compact (127 rows) and padded (960
+    # rows, group g at rows 120g...): identical totals and copies, identical
+    # real output rows, +0.0 padding rows
+    c = run_gpu(wlmod.make("dp_compact", seed=0), layout_variant=layout_variant)
+    p = run_gpu(wlmod.make("dp_padded", seed=0), layout_variant=layout_variant)
+    for key in ("N_route", "N_recv", "T_real"):
+        assert c["totals"][key] == p["totals"][key]
+    np.testing.assert_array_equal(c["layout"].cnt_e.cpu().numpy(), p["layout"].cnt_e.cpu().numpy())
+    n_route, n_recv = c["totals"]["N_route"], c["totals"]["N_recv"]
+    np.testing.assert_array_equal(torch_to_bits(c["expanded"][:n_route]),
+                                  torch_to_bits(p["expanded"][:n_route]))
+    np.testing.assert_array_equal(torch_to_bits(c["recv"][:n_recv]),
+                                  torch_to_bits(p["recv"][:n_recv]))
+    rows = np.concatenate([np.arange(120), 120 * np.arange(1, 8)])
+    out_c, out_p = torch_to_bits(c["out"]), torch_to_bits(p["out"])
+    np.testing.assert_array_equal(out_p[rows], out_c)
+    mask = np.ones(960, bool)
+    mask[rows] = False
+    assert np.all(out_p[mask] == 0)
