@@ -461,8 +461,8 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
 // and the same for recv_pos with the rank columns; base comes from the
 // cluster exchange and global scan shared with the count-matrix schedule.
 // Each lane keeps its routes in registers (one per pass of the CTA's warps
-// over its tokens), so nothing walks the tokens serially.  The CTA has as
-// few warps as keep the passes at four or fewer: the phases are short and
+// over its tokens), so nothing walks the tokens serially.  The CTA has few
+// warps (8 or 16, 32 only beyond 64 chunks): the phases are short and
 // separated by barriers, and every barrier and every shared-memory phase is
 // cheaper with fewer warps.
 
@@ -684,8 +684,11 @@ bool plan_warp(int T, int k, int E, int R, int csize, WarpGeometry *g)
         g->csize = csize;
         g->tpc = (T + csize - 1) / csize;
         const int nch = (g->tpc + g->tpw - 1) / g->tpw;
-        // fewest warps (of 8, 16 or 32) that need no more than four passes
+        // warps (8, 16 or 32): at most two passes up to 16 warps, then at
+        // most four (measured: decode's 32 chunks run faster as 16 warps x 2
+        // passes than as 8 x 4; prefill's 64 faster as 16 x 4 than 32 x 2)
         int warps = 8;
+        while (warps < 16 && nch > 2 * warps) warps *= 2;
         while (warps < 32 && nch > 4 * warps) warps *= 2;
         if (warps * 32 < min_threads) warps = (min_threads + 31) / 32;
         const int passes = (nch + warps - 1) / warps;
