@@ -665,34 +665,42 @@ def parity_summary(torch, lay, expanded, out, ores):
             "combine_within_tol": ok}
 
 
+E2E_STREAMS = 3
+
+
 def run_e2e(torch, epx, wl, args, dev, stream, pg, world, T_real):
     """The metric through ep_roundtrip_host with pinned host buffers: every
     step copies its inputs host -> device, runs layout, dispatch/expand, the
-    stand-in expert and combine, and copies the output back.  Steps alternate
-    between two streams with their own device scratch and output buffer, so
-    one step's upload overlaps the other's compute and download (the link is
-    full duplex) -- what a caller pipelining the public call gets."""
+    stand-in expert and combine, and copies the output back.  Steps rotate
+    over E2E_STREAMS streams with their own device scratch and output buffer,
+    so one step's upload overlaps the others' compute and download (the link
+    is full duplex; with three streams an upload is always queued while a
+    stream's own download runs) -- what a caller pipelining the public call
+    gets."""
     T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
     itype = torch.int64 if args.idx_bits == 64 else torch.int32
     x_h = torch.from_numpy(wl["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
     i_h = torch.from_numpy(wl["topk_idx"]).to(itype).pin_memory()
     w_h = torch.from_numpy(wl["topk_weights"]).pin_memory()
     nbytes = epx.roundtrip_device_bytes(T, H, k, E, R, args.idx_bits)
-    streams = [stream, torch.cuda.Stream(device=dev)]
+    streams = [stream] + [torch.cuda.Stream(device=dev) for _ in range(E2E_STREAMS - 1)]
     dmem = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in streams]
     out_h = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in streams]
     n = max(1, args.e2e_steps)
-    for i in range(4):
-        epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem[i % 2], out_h[i % 2], stream=streams[i % 2])
+    ns = len(streams)
+    for i in range(2 * ns):
+        epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem[i % ns], out_h[i % ns],
+                           stream=streams[i % ns])
     torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     ends = [torch.cuda.Event(enable_timing=True) for _ in streams]
     e0.record(streams[0])
-    streams[1].wait_event(e0)
+    for st in streams[1:]:
+        st.wait_event(e0)
     for i in range(n):
-        s = i % 2
+        s = i % ns
         epx.roundtrip_host(x_h, i_h, w_h, E, R, dmem[s], out_h[s], stream=streams[s])
     for s, ev in zip(streams, ends):
         ev.record(s)
@@ -704,7 +712,7 @@ def run_e2e(torch, epx, wl, args, dev, stream, pg, world, T_real):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "path": "ep_roundtrip_host per step (pinned host -> device, layout, "
                     "dispatch/expand, stand-in expert, combine, device -> host), steps "
-                    "alternating over two streams"}
+                    f"rotating over {ns} streams"}
 
 
 def reduce_max(pg, value: float, device) -> float:
