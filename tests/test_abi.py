@@ -95,6 +95,11 @@ def test_calls_reject_bad_arguments_before_launching(lib):
     assert lib.ep_standin_expert(fake, 16, ctypes.byref(c), fake + 4, 8, None) == 2
     # misaligned 64-bit indices
     assert lib.ep_layout(fake + 4, ctypes.byref(c), None) == 2
+    # unknown layout schedule or combine schedule
+    assert lib.ep_layout_variant(fake, ctypes.byref(c), 3, None) == 1
+    assert lib.ep_layout_variant(fake, ctypes.byref(c), -1, None) == 1
+    assert lib.ep_layout_variant(fake + 4, ctypes.byref(c), 1, None) == 2
+    assert lib.ep_combine_reduce_variant(fake, fake, 16, ctypes.byref(c), fake, 8, 3, None) == 1
 
 
 def test_roundtrip_sizes(lib):
