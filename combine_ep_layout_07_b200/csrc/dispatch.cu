@@ -14,8 +14,8 @@
 //  * bulk: the row (or a chunk of it) is staged in shared memory by one TMA
 //    bulk load (cp.async.bulk, completion on an mbarrier) and written out by
 //    one TMA bulk store per destination row, issued by the warp's lanes in
-//    parallel.  No multicast: every copy is a plain global<->shared::cta
-//    bulk copy on this GPU.
+//    parallel.  Every copy is a plain global<->shared::cta bulk copy of
+//    this GPU's own memory, issued by the CTA that uses it.
 #include "epx_internal.cuh"
 
 namespace epx {
