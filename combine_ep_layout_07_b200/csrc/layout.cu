@@ -11,8 +11,10 @@
 // A route's row is off_e[e] + (routes to e from earlier tokens) + (earlier
 // slots of its own token with the same expert); a (token, rank) pair's row
 // is off_r[r] + (earlier tokens that reach r).  Both middle terms are prefix
-// sums over tokens of a (expert | rank) x token count matrix, so they are
-// computed here without any ordering primitive:
+// sums over tokens, computed without any ordering primitive by one of two
+// schedules with identical results: the warp-chunk schedule (the default
+// wherever its per-warp table fits; described at layout_warp_kernel below)
+// and the count-matrix schedule, which handles every valid size:
 //  * one launch of one CTA, or of one thread-block cluster of up to 16 CTAs
 //    of 1024 threads; CTA c owns a contiguous range of tokens;
 //  * build: one thread per token loads its k indices, validates them,
@@ -24,11 +26,10 @@
 //  * row scan: one thread per matrix row walks its tokens and rewrites the
 //    counts as a running prefix (packed 16-bit halves add independently);
 //    the row sum is the CTA total;
-//  * cluster exchange: each CTA adds its totals into every peer's shared
-//    memory with distributed-shared-memory atomics -- into all peers' sums
-//    and into the "lower CTAs" sums of the peers above it -- so after one
-//    cluster barrier each CTA reads two values per expert; a single CTA
-//    skips this;
+//  * cluster exchange: each CTA stores its totals into its own row of every
+//    peer's totals table (distributed-shared-memory stores); after one
+//    cluster barrier each CTA sums the table locally, over all CTAs and over
+//    the CTAs below it; a single CTA skips this;
 //  * global scan: one packed 64-bit block scan of the (expert, rank) totals
 //    gives both exclusive scans, plus this CTA's base per expert / rank;
 //  * placement: one thread per four routes, then per four (token, rank)
