@@ -152,6 +152,10 @@ cudaError_t launch_combine(const CombineParams &p0, int variant, cudaStream_t s)
     const int max_chunks = (p.V + 31) / 32;
     if (chunks > max_chunks) chunks = max_chunks;
     if (chunks < 1) chunks = 1;
+    // at large batch still two chunks per row: CTAs half as long give the
+    // grid a shorter ragged tail (measured 1.4 us off a 241 us prefill step on
+    // two boxes; four or seven chunks per row were no better)
+    if (chunks < 2 && p.V >= 256) chunks = 2;
     // when one vector per thread fits in one wave (seven 128-thread CTAs
     // per SM at this kernel's register count), take it: a thread's second
     // vector would wait for its first one's loads
