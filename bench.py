@@ -55,6 +55,8 @@ DESCRIBE = {
 
 # sources whose hash keys the committed ncu DRAM traffic figure
 KERNEL_SOURCES = {
+    "layout_dispatch_expand": ["combine_ep_layout_07_b200/csrc/fused.cu",
+                               "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "dispatch_expand": ["combine_ep_layout_07_b200/csrc/dispatch.cu",
                         "combine_ep_layout_07_b200/csrc/epx_internal.cuh"],
     "combine_reduce": ["combine_ep_layout_07_b200/csrc/combine.cu",
@@ -101,6 +103,13 @@ def parse_args(argv=None):
                     help="dispatch writes recv rows only plus a gather index (the expert "
                          "consumer reads recv through it); also times that consumer "
                          "against the one reading the expanded copy")
+    ap.add_argument("--step-calls", choices=["auto", "separate", "fused"], default="auto",
+                    help="layout and dispatch/expand as one call (one launch, small batches), "
+                         "as two calls, or automatic (one launch up to "
+                         "EPX_FUSED_AUTO_ROUTES routes, as the library's automatic choice)")
+    ap.add_argument("--small-steps", type=int, default=1500,
+                    help="steps of each small-batch workload measured beside the headline "
+                         "(0 skips them)")
     ap.add_argument("--two-stage", choices=["fp32", "bf16"], default=None,
                     help="combine as a per-(token, rank) local reduce with fp32 or bf16 "
                          "partials followed by the epilogue, instead of the fused reduce")
@@ -125,14 +134,18 @@ def load_peaks():
 
 
 def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None,
-              no_expand=False):
+              no_expand=False, fused=False):
     """Algorithmic HBM bytes per step of each kernel (each byte the definition
     must move once; no re-reads).  With part_bytes (4 or 2) the combine is the
     two-stage form: local reduce + epilogue through N_recv partial rows.  With
-    no_expand the dispatch writes recv rows only, plus the gather index."""
+    no_expand the dispatch writes recv rows only, plus the gather index.  With
+    fused the layout and dispatch/expand are one kernel (their bytes add; the
+    layout's own pos / recv_pos stores replace the dispatch's loads of them)."""
     row = H * 2
     layout = T * k * idx_bytes + T * k * 4 + T * R * 4
-    if no_expand:
+    if fused:
+        out = dict(layout_dispatch_expand=layout + T_real * row + (N_recv + N_route) * row)
+    elif no_expand:
         out = dict(layout=layout,
                    dispatch=T_real * row + N_recv * row + T * R * 4,
                    expand_index=T * k * 4 + T * R * 4 + N_route * 4)
@@ -294,24 +307,51 @@ def step_stats(step_ms):
     return {"median": pick(0.5), "p10": pick(0.1), "p90": pick(0.9)}
 
 
+class PinnedToOneCore:
+    """Runs the enclosed code on one host core (the oracle is single-threaded;
+    pinning keeps its timing from migrating between cores).  Restores the
+    previous affinity; a no-op where affinity cannot be set."""
+
+    def __enter__(self):
+        self.prev = None
+        try:
+            self.prev = os.sched_getaffinity(0)
+            self.core = min(self.prev)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            self.core = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            try:
+                os.sched_setaffinity(0, self.prev)
+            except OSError:
+                pass
+        return False
+
+
 def cpu_baseline(wl, budget_s, idx_bits):
-    """Oracle, as it stands, over the full workload repeated for ~budget_s."""
+    """Oracle, as it stands, over the full workload repeated for ~budget_s,
+    pinned to one host core."""
     import oracle
     oracle.build()
     idx = wl["topk_idx"].astype(np.int64 if idx_bits == 64 else np.int32)
     lay = oracle.layout(idx, wl["E"], wl["R"])
     _, expanded = oracle.dispatch_expand(wl["x"], lay)
     y = oracle.standin(expanded, lay)
-    passes, t0 = 0, time.perf_counter()
     out = None
-    while True:
-        out, _ = oracle_pass(oracle, wl, y, idx)
-        passes += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
+    with PinnedToOneCore() as pin:
+        passes, t0 = 0, time.perf_counter()
+        while True:
+            out, _ = oracle_pass(oracle, wl, y, idx)
+            passes += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
     value = lay["T_real"] * passes / el
     return dict(value=value, unit=UNIT, cores=1, kind="oracle", host=host_cpu(),
+                pinned_core=pin.core,
                 sample=f"{passes} full pass(es) of the {wl['name']} workload "
                        f"({lay['T_real']} effective tokens each) in {el:.1f} s, "
                        f"single-threaded C, layout+dispatch/expand+combine"), \
@@ -347,12 +387,13 @@ def run_reference(args):
     slay = oracle.layout(sidx, wl["E"], wl["R"])
     _, sex = oracle.dispatch_expand(sub["x"], slay)
     sy = oracle.standin(sex, slay)
-    for _ in range(args.warmup):
-        oracle_pass(oracle, sub, sy, sidx)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_pass(oracle, sub, sy, sidx)
-    el = time.perf_counter() - t0
+    with PinnedToOneCore() as pin:
+        for _ in range(args.warmup):
+            oracle_pass(oracle, sub, sy, sidx)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_pass(oracle, sub, sy, sidx)
+        el = time.perf_counter() - t0
     units = slay["T_real"] * args.steps
     value = units / el
     sample = (f"first {n} of {wl['T']} rows of the {wl['name']} workload "
@@ -365,21 +406,31 @@ def run_reference(args):
         "data": "synthetic", "config": dict(workload_config(wl, args, slay),
                                             launch="host CPU, single thread"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample, "host": host_cpu()},
+                         "sample": sample, "host": host_cpu(), "pinned_core": pin.core},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def workload_config(wl, args, lay_totals, flush_desc=None):
+def fused_step(args, T, k):
+    """Whether the step runs layout + dispatch/expand as one launch."""
+    if getattr(args, "no_expand", False) or args.step_calls == "separate":
+        return False
+    if args.step_calls == "fused":
+        return True
+    from combine_ep_layout_07_b200 import epx
+    return T * k <= epx.FUSED_AUTO_ROUTES
+
+
+def workload_config(wl, args, lay_totals, flush_desc=None, fused=False):
     cfg = {"workload": DESCRIBE[args.workload], "T": wl["T"], "H": wl["H"], "E": wl["E"],
            "R": wl["R"], "k": wl["k"], "seed": args.seed, "idx_bits": args.idx_bits,
            "T_real": int(lay_totals["T_real"]), "N_recv": int(lay_totals["N_recv"]),
            "N_route": int(lay_totals["N_route"]),
-           "timed": "layout + " + ("dispatch (recv only) + expand_index + "
-                                   if getattr(args, "no_expand", False)
-                                   else "dispatch_expand + ") + (
+           "timed": ("layout_dispatch_expand (one launch) + " if fused else "layout + " + (
+               "dispatch (recv only) + expand_index + " if getattr(args, "no_expand", False)
+               else "dispatch_expand + ")) + (
                "combine_reduce" if not getattr(args, "two_stage", None) else
                "combine_local_reduce (%s partials) + combine_epilogue" % args.two_stage),
            "parallelism": f"replicas x{dist_env()[1]}"}
@@ -390,6 +441,216 @@ def workload_config(wl, args, lay_totals, flush_desc=None):
                      "launch; per-kernel split from a second run of the same steps with "
                      "events between kernels")
     return cfg
+
+
+class Step:
+    """Device buffers and the calls of one step of the path on one workload."""
+
+    def __init__(self, torch, epx, wl, args, dev, fused, two_stage=None, no_expand=False):
+        self.torch, self.epx, self.wl = torch, epx, wl
+        T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
+        itype = torch.int64 if args.idx_bits == 64 else torch.int32
+        self.x = x = torch.from_numpy(wl["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+        self.idx = idx = torch.from_numpy(wl["topk_idx"]).to(itype).to(dev)
+        self.w = w = torch.from_numpy(wl["topk_weights"]).to(dev)
+        self.lay = lay = epx.Layout(T, k, E, R, args.idx_bits, device=dev)
+        self.recv = recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=dev)
+        self.expanded = expanded = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16,
+                                               device=dev)
+        self.y = y = torch.empty_like(expanded)
+        self.out = out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+        self.part = part = None
+        if two_stage:
+            self.part = part = torch.empty(
+                (lay.recv_cap, H), device=dev,
+                dtype=torch.float32 if two_stage == "fp32" else torch.bfloat16)
+        self.src = src = (torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev)
+                          if no_expand else None)
+        self.fused, self.no_expand = fused, no_expand
+        calls = []
+        if fused:
+            calls.append(("layout_dispatch_expand", lambda st: epx.layout_dispatch_expand(
+                idx, x, E, R, out=lay, recv=recv, expanded=expanded, variant=1, stream=st)))
+        else:
+            calls.append(("layout", lambda st: epx.layout(
+                idx, E, R, out=lay, variant=args.layout_variant, stream=st)))
+            if no_expand:
+                calls.append(("dispatch", lambda st: epx.dispatch(x, lay, recv=recv, stream=st)))
+                calls.append(("expand_index", lambda st: epx.expand_index(lay, src=src,
+                                                                          stream=st)))
+            else:
+                calls.append(("dispatch_expand", lambda st: epx.dispatch_expand(
+                    x, lay, recv=recv, expanded=expanded, variant=args.dispatch_variant,
+                    stream=st)))
+        if part is None:
+            calls.append(("combine_reduce", lambda st: epx.combine_reduce(
+                y, w, lay, out=out, variant=args.combine_variant, stream=st)))
+        else:
+            calls.append(("combine_local", lambda st: epx.combine_local_reduce(
+                y, w, lay, partial=part, stream=st)))
+            calls.append(("combine_epilogue", lambda st: epx.combine_epilogue(
+                part, lay, out=out, stream=st)))
+        self.calls = calls
+        self.names = [n for n, _ in calls]
+
+    def prepare(self, stream):
+        """The stand-in expert's output that combine reads (made once,
+        outside the timed steps) and the layout totals."""
+        torch, epx = self.torch, self.epx
+        with torch.cuda.stream(stream):
+            epx.layout(self.idx, self.wl["E"], self.wl["R"], out=self.lay, stream=stream)
+            epx.dispatch_expand(self.x, self.lay, recv=self.recv, expanded=self.expanded,
+                                stream=stream)
+            epx.standin_expert(self.expanded, self.lay, y=self.y, stream=stream)
+        self.tot = epx.read_totals(self.lay, stream=stream)
+        return self.tot
+
+    def launch(self, st, events=None):
+        for i, (_, fn) in enumerate(self.calls):
+            if events is not None:
+                events[i].record(st)
+            fn(st)
+        if events is not None:
+            events[len(self.calls)].record(st)
+
+
+class L2Flush:
+    """Evicts L2 between steps by READING a buffer of twice its size (outside
+    the timed events): lines the previous step left dirty are written back
+    during the flush, and the step starts with its inputs in DRAM and no
+    dirty lines of anyone else's to write back."""
+
+    def __init__(self, torch, dev):
+        self.buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int64, device=dev)
+        self.torch = torch
+
+    def __call__(self):
+        self.torch.sum(self.buf, dim=0, dtype=self.torch.int64, out=self.sink)
+
+    DESC = "L2 flushed between steps (256 MiB read, outside the timed events)"
+
+
+def time_step(torch, launch, n_calls, stream, dev, steps, warmup, flush=None, eager=False,
+              split=True, pg=None):
+    """Times `steps` steps of `launch(st, events=None)` with CUDA events on
+    `stream`.  Graph mode (default): the step is captured once with events at
+    its ends only (programmatic-launch overlaps kept) and, when split, once
+    more with events between its calls for the per-call split.  Returns
+    (per-step ms, per-step cumulative split ms or None, wall-clock window)."""
+    graph = graph_k = None
+    if not eager:
+        with torch.cuda.stream(stream):
+            launch(stream)          # launchers set their function attributes here
+        torch.cuda.synchronize(dev)
+        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            cs = torch.cuda.current_stream()
+            gev[0].record(cs)
+            launch(cs)
+            gev[1].record(cs)
+        if split:
+            gks = [torch.cuda.Event(enable_timing=True, external=True)
+                   for _ in range(n_calls + 1)]
+            graph_k = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_k, stream=stream):
+                launch(torch.cuda.current_stream(), gks)
+        torch.cuda.synchronize(dev)
+
+    def one(rec=None, use_split=False):
+        if flush is not None:
+            flush()
+        if graph is not None:
+            (graph_k if use_split else graph).replay()
+            if rec is not None:
+                torch.cuda.current_stream().synchronize()
+                if use_split:
+                    rec.append([gks[0].elapsed_time(gks[j]) for j in range(1, len(gks))])
+                else:
+                    rec.append(gev[0].elapsed_time(gev[1]))
+        else:
+            if rec is not None:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)]
+                launch(torch.cuda.current_stream(), ev)
+                rec.append(ev)
+            else:
+                launch(torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one()
+            if graph_k is not None:
+                one(use_split=True)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    rec, rec_k = [], []
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    t_lo = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            one(rec)
+    torch.cuda.synchronize(dev)
+    t_hi = time.time()
+    if pg:
+        pg.barrier()
+    if graph_k is not None:
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                one(rec_k, use_split=True)
+        torch.cuda.synchronize(dev)
+    if graph is None:   # cumulative times from each step's first event
+        rec_k = [[e[0].elapsed_time(e[j]) for j in range(1, len(e))] for e in rec]
+        step_ms = [r[-1] for r in rec_k]
+    else:
+        step_ms = rec
+    del graph, graph_k
+    return step_ms, (rec_k if (split or eager) else None), (t_lo, t_hi)
+
+
+def time_floor(torch, epx, stream, dev, n_kernels, steps, warmup, flush):
+    """ep_latency_floor chain of n_kernels, timed exactly like a step."""
+    buf = torch.zeros(64 * (2 * n_kernels + 2), dtype=torch.int32, device=dev)
+    ms, _, _ = time_step(torch, lambda st, ev=None: epx.latency_floor(buf, n_kernels, stream=st),
+                         1, stream, dev, steps, warmup, flush=flush, split=False)
+    return step_stats(ms)
+
+
+SMALL_WORKLOADS = ("decode", "dp_compact", "dp_padded", "lowbatch1")
+
+
+def measure_small(torch, epx, wlmod, args, dev, stream, peak, flush, floors):
+    """Step time of each small-batch workload in the same run (graph mode, L2
+    flushed by a read between steps, automatic layout/dispatch choice)."""
+    res = {}
+    for name in SMALL_WORKLOADS:
+        if name == args.workload:
+            continue
+        wl = wlmod.make(name, seed=args.seed)
+        fused = fused_step(args, wl["T"], wl["k"])
+        st = Step(torch, epx, wl, args, dev, fused)
+        tot = st.prepare(stream)
+        ms, rec_k, _ = time_step(torch, st.launch, len(st.calls), stream, dev, args.small_steps,
+                                 max(3, args.warmup), flush=flush)
+        stats = step_stats(ms)
+        b = alg_bytes(wl["T"], tot["T_real"], tot["N_recv"], tot["N_route"], wl["H"], wl["k"],
+                      wl["R"], args.idx_bits // 8, fused=fused)
+        kern = {n: statistics.median([r[i] - (r[i - 1] if i else 0.0) for r in rec_k]) * 1e3
+                for i, n in enumerate(st.names)}
+        floor = floors.get(len(st.calls))
+        res[name] = {
+            "workload": DESCRIBE[name], "T_real": int(tot["T_real"]),
+            "step_us": stats, "tokens_per_s": tot["T_real"] / (stats["median"] / 1e6),
+            "alg_bytes": b["total"],
+            "hbm_frac": b["total"] / (stats["median"] / 1e6) / 1e9 / peak,
+            "launches": len(st.calls), "calls": st.names,
+            "kernel_us_median_split": kern,
+            "x_floor": (stats["median"] / floor["median"]) if floor else None,
+        }
+    return res
 
 
 # ---------------------------------------------------------------- epx arm
@@ -414,54 +675,12 @@ def run_epx(args):
 
     wl = wlmod.make(args.workload, seed=args.seed + rank)
     T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
-    itype = torch.int64 if args.idx_bits == 64 else torch.int32
-    x = torch.from_numpy(wl["x"].view(np.int16)).view(torch.bfloat16).to(dev)
-    idx = torch.from_numpy(wl["topk_idx"]).to(itype).to(dev)
-    w = torch.from_numpy(wl["topk_weights"]).to(dev)
     stream = torch.cuda.Stream(device=dev)
-    lay = epx.Layout(T, k, E, R, args.idx_bits, device=dev)
-    recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=dev)
-    expanded = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16, device=dev)
-    y = torch.empty_like(expanded)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-
-    part = None
-    if args.two_stage:
-        part = torch.empty((lay.recv_cap, H), device=dev,
-                           dtype=torch.float32 if args.two_stage == "fp32" else torch.bfloat16)
-    src = torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev) if args.no_expand else None
-    calls = [("layout", lambda st: epx.layout(idx, E, R, out=lay, variant=args.layout_variant,
-                                              stream=st))]
-    if args.no_expand:
-        calls.append(("dispatch", lambda st: epx.dispatch(x, lay, recv=recv, stream=st)))
-        calls.append(("expand_index", lambda st: epx.expand_index(lay, src=src, stream=st)))
-    else:
-        calls.append(("dispatch_expand", lambda st: epx.dispatch_expand(
-            x, lay, recv=recv, expanded=expanded, variant=args.dispatch_variant, stream=st)))
-    if part is None:
-        calls.append(("combine_reduce", lambda st: epx.combine_reduce(
-            y, w, lay, out=out, variant=args.combine_variant, stream=st)))
-    else:
-        calls.append(("combine_local", lambda st: epx.combine_local_reduce(
-            y, w, lay, partial=part, stream=st)))
-        calls.append(("combine_epilogue", lambda st: epx.combine_epilogue(
-            part, lay, out=out, stream=st)))
-    names = [n for n, _ in calls]
-
-    def step_kernels(events=None, st=None):
-        st = stream if st is None else st
-        for i, (_, fn) in enumerate(calls):
-            if events is not None:
-                events[i].record(st)
-            fn(st)
-        if events is not None:
-            events[len(calls)].record(st)
-
-    with torch.cuda.stream(stream):
-        epx.layout(idx, E, R, out=lay, variant=args.layout_variant, stream=stream)
-        epx.dispatch_expand(x, lay, recv=recv, expanded=expanded, stream=stream)
-        epx.standin_expert(expanded, lay, y=y, stream=stream)
-    tot = epx.read_totals(lay, stream=stream)
+    fused = fused_step(args, T, k)
+    step = Step(torch, epx, wl, args, dev, fused, two_stage=args.two_stage,
+                no_expand=args.no_expand)
+    tot = step.prepare(stream)
+    lay, recv, expanded, y, out = step.lay, step.recv, step.expanded, step.y, step.out
     consumer = None
     if args.no_expand:
         consumer = time_consumers(torch, epx, lay, recv, expanded, y, stream, dev, tot, H,
@@ -469,99 +688,28 @@ def run_epx(args):
 
     bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
                        args.idx_bits // 8,
-                       None if part is None else part.element_size(), args.no_expand)
+                       None if step.part is None else step.part.element_size(), args.no_expand,
+                       fused=fused)
     working = bytes_["total"]
-    flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
-    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev) if flush else None
-    if flush:
-        flush_desc = "L2 flushed between steps (256 MiB write, outside the timed events)"
+    do_flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
+    l2flush = L2Flush(torch, dev)
+    if do_flush:
+        flush_desc = L2Flush.DESC
     elif working >= 2 * L2_BYTES:
         flush_desc = f"inputs larger than L2 ({working / 1e6:.0f} MB moved per step, no flush)"
     else:
         flush_desc = (f"hot L2: no flush between steps ({working / 1e6:.0f} MB moved per step, "
                       f"below 2x L2)")
 
-    graph = graph_k = None
-    gev = gks = None
-    if not args.eager:
-        # Two captured graphs of one step: `graph` has timing events only at
-        # its ends, so consecutive kernels overlap their launches
-        # (programmatic dependent launch); `graph_k` also has events between
-        # the kernels (which serialises them) for the per-kernel split.
-        with torch.cuda.stream(stream):
-            step_kernels()          # launchers set their function attributes here
-        torch.cuda.synchronize(dev)
-        gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
-            cs = torch.cuda.current_stream()
-            gev[0].record(cs)
-            step_kernels(st=cs)
-            gev[1].record(cs)
-        gks = [torch.cuda.Event(enable_timing=True, external=True)
-               for _ in range(len(calls) + 1)]
-        graph_k = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph_k, stream=stream):
-            step_kernels(gks, st=torch.cuda.current_stream())
-        torch.cuda.synchronize(dev)
-
-    def run_step(out=None, split=False):
-        if flush:
-            flush_buf.add_(1)
-        if graph is not None:
-            (graph_k if split else graph).replay()
-            if out is not None:
-                torch.cuda.current_stream().synchronize()
-                if split:
-                    out.append([gks[0].elapsed_time(gks[j]) for j in range(1, len(gks))])
-                else:
-                    out.append(gev[0].elapsed_time(gev[1]))
-        else:
-            if out is not None:
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
-                step_kernels(ev)
-                out.append(ev)
-            else:
-                step_kernels()
-
-    # warm-up
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            run_step()
-            if graph_k is not None:
-                run_step(split=True)
-    torch.cuda.synchronize(dev)
-    if pg:
-        pg.barrier()
-
     sampler = ClockSampler(gpu_uuid(torch, local)) if rank == 0 else None
     if sampler:
         sampler.start()
-    rec, rec_k = [], []
-    torch.cuda.synchronize(dev)
-    if pg:
-        pg.barrier()
-    t_lo = time.time()
-    with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            run_step(rec)
-    torch.cuda.synchronize(dev)
-    t_hi = time.time()
-    if pg:
-        pg.barrier()
-    if graph_k is not None:
-        with torch.cuda.stream(stream):
-            for i in range(args.steps):
-                run_step(rec_k, split=True)
-        torch.cuda.synchronize(dev)
+    step_ms, rec_k, (t_lo, t_hi) = time_step(
+        torch, step.launch, len(step.calls), stream, dev, args.steps, args.warmup,
+        flush=l2flush if do_flush else None, eager=args.eager, split=True, pg=pg)
     if sampler:
         sampler.stop()
-
-    if graph is None:   # cumulative times from each step's first event
-        rec_k = [[e[0].elapsed_time(e[j]) for j in range(1, len(e))] for e in rec]
-        step_ms = [r[-1] for r in rec_k]
-    else:
-        step_ms = rec
+    names = step.names
     k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)
     value = whole_job_value(tot["T_real"] * args.steps, world, total_ms)
@@ -569,14 +717,21 @@ def run_epx(args):
     # ---- e2e through the host-buffer C-ABI call
     e2e = None if args.no_e2e else run_e2e(torch, epx, wl, args, dev, stream, pg, world,
                                            tot["T_real"])
-    if graph is not None:
-        del graph, graph_k
+
+    peak, peak_kind = load_peaks()
+    # ---- latency floor and the small-batch workloads, same run, same protocol
+    floors, small = {}, None
+    if args.small_steps > 0 and rank == 0:
+        n_floor = max(3, min(args.small_steps, 1000))
+        for n in (2, 3):
+            floors[n] = time_floor(torch, epx, stream, dev, n, n_floor, max(3, args.warmup),
+                                   l2flush)
+        small = measure_small(torch, epx, wlmod, args, dev, stream, peak, l2flush, floors)
 
     if rank != 0:
         finish(pg)
         return 0
 
-    peak, peak_kind = load_peaks()
     kernels = {}
     for name, ms in k_ms.items():
         avg_s = statistics.fmean(ms) / 1e3
@@ -587,10 +742,12 @@ def run_epx(args):
     engine = {"dispatch": "recv_only", "expand_index": "gather_index",
               "combine_local": "two_stage_" + str(args.two_stage),
               "combine_epilogue": "two_stage_" + str(args.two_stage),
+              "layout_dispatch_expand": "one_launch",
               "dispatch_expand": "bulk" if args.dispatch_variant == 2 or
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
               "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split",
-              "layout": "count_matrix" if args.layout_variant == 2 else "warp_chunks"}
+              "layout": {1: "warp_chunks", 2: "count_matrix", 3: "grid"}.get(
+                  args.layout_variant, "grid" if T * k > 8192 else "warp_chunks")}
     traffic = committed_traffic(dom, args.workload, engine.get(dom))
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
@@ -603,15 +760,23 @@ def run_epx(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(wl, args, tot, flush_desc),
+        "config": workload_config(wl, args, tot, flush_desc, fused),
         "roofline": roofline,
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
         "step_us": step_stats(step_ms),
         "kernels": kernels,
-        "gpu_launches": len(calls) * args.steps,
+        "gpu_launches": len(step.calls) * args.steps,
         **({"consumer": consumer} if consumer else {}),
         "e2e": e2e,
     }
+    if floors:
+        line["floor_us"] = {
+            str(n): dict(v, what=f"{n} chained one-warp launches (programmatic dependent launch),"
+                                 " one global load each after its wait, graph-timed like the "
+                                 "step, L2 flushed by a read")
+            for n, v in floors.items()}
+    if small:
+        line["small_batch"] = small
     if sampler:
         line["clocks"] = sampler.summary(t_lo, t_hi)
     if world == 1 and not args.no_cpu_baseline:

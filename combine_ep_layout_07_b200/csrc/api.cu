@@ -28,7 +28,8 @@ bool layout_ok(const ep_layout_t *L)
     if (!L) return false;
     if (!sizes_ok(L->T, L->k, L->E, L->R)) return false;
     if (L->idx_bits != 32 && L->idx_bits != 64) return false;
-    return L->cnt_e && L->off_e && L->cnt_r && L->off_r && L->pos && L->recv_pos && L->totals;
+    return L->cnt_e && L->off_e && L->cnt_r && L->off_r && L->pos && L->recv_pos && L->totals &&
+           L->work;
 }
 
 ep_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
@@ -64,6 +65,7 @@ size_t ep_layout_bytes(int32_t T, int32_t k, int32_t E, int32_t R)
     n += round_up(sizeof(int32_t) * (size_t)T * k, 16);
     n += round_up(sizeof(int32_t) * (size_t)T * R, 16);
     n += round_up(sizeof(int32_t) * 4, 16);
+    n += round_up(grid_work_bytes(T, k, E, R), 16);
     return n;
 }
 
@@ -97,6 +99,7 @@ ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E, int3
     l.pos = take((size_t)T * k);
     l.recv_pos = take((size_t)T * R);
     l.totals = take(4);
+    l.work = reinterpret_cast<int32_t *>(p);
     *L = l;
     return EP_OK;
 }
@@ -105,7 +108,7 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L, int32_
                               void *stream)
 {
     if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
-    if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
+    if (variant < 0 || variant > 3) return EP_ERR_INVALID_ARG;
     if (L->T > 0 && !topk_idx) return EP_ERR_INVALID_ARG;
     if (topk_idx && !aligned(topk_idx, (size_t)L->idx_bits / 8)) return EP_ERR_MISALIGNED;
     LayoutParams p;
@@ -123,6 +126,7 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L, int32_
     p.pos = L->pos;
     p.recv_pos = L->recv_pos;
     p.totals = L->totals;
+    p.work = L->work;
     const cudaError_t e = launch_layout(p, L->idx_bits, variant, as_stream(stream));
     return e == cudaErrorNotSupported ? EP_ERR_UNSUPPORTED : from_cuda(e);
 }
@@ -140,7 +144,8 @@ ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout
     if (H <= 0 || H % 8 != 0 || recv_cap < 0 || exp_cap < 0) return EP_ERR_INVALID_ARG;
     if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
     if (L->T == 0) return EP_OK;
-    if (!x || !recv || !expanded) return EP_ERR_INVALID_ARG;
+    // recv may be NULL with recv_cap 0: expanded rows only
+    if (!x || !expanded || (!recv && recv_cap != 0)) return EP_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(recv, 16) || !aligned(expanded, 16)) return EP_ERR_MISALIGNED;
     DispatchParams p;
     memset(&p, 0, sizeof p);
@@ -163,6 +168,61 @@ ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L, v
                                int64_t recv_cap, void *expanded, int64_t exp_cap, void *stream)
 {
     return ep_dispatch_expand_variant(x, H, L, recv, recv_cap, expanded, exp_cap, 0, stream);
+}
+
+ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_layout_t *L,
+                                              const void *x, int32_t H, void *recv,
+                                              int64_t recv_cap, void *expanded, int64_t exp_cap,
+                                              int32_t variant, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || recv_cap < 0 || exp_cap < 0) return EP_ERR_INVALID_ARG;
+    if (variant < 0 || variant > 2) return EP_ERR_INVALID_ARG;
+    if (L->T > 0 && (!topk_idx || !x || !recv || !expanded)) return EP_ERR_INVALID_ARG;
+    if (topk_idx && !aligned(topk_idx, (size_t)L->idx_bits / 8)) return EP_ERR_MISALIGNED;
+    if (L->T > 0 && (!aligned(x, 16) || !aligned(recv, 16) || !aligned(expanded, 16)))
+        return EP_ERR_MISALIGNED;
+    const long long routes = (long long)L->T * L->k;
+    // automatic: one launch while each CTA's count over all routes stays
+    // cheap (measured on B200), else the layout and dispatch kernels
+    if (variant == 0) variant = routes <= kFusedAutoRoutes ? 1 : 2;
+    if (variant == 2) {
+        ep_status_t st = ep_layout(topk_idx, L, stream);
+        if (st != EP_OK || L->T == 0) return st;
+        return ep_dispatch_expand(x, H, L, recv, recv_cap, expanded, exp_cap, stream);
+    }
+    if (routes > kFusedMaxRoutes) return EP_ERR_UNSUPPORTED;
+    FusedParams p;
+    memset(&p, 0, sizeof p);
+    p.idx = topk_idx;
+    p.x = static_cast<const uint4 *>(x);
+    p.T = L->T;
+    p.k = L->k;
+    p.E = L->E;
+    p.R = L->R;
+    p.V = H / 8;
+    p.inv_epr = 1.0f / (float)(L->E / L->R);
+    p.recv = static_cast<uint4 *>(recv);
+    p.recv_cap = recv_cap;
+    p.expanded = static_cast<uint4 *>(expanded);
+    p.exp_cap = exp_cap;
+    p.cnt_e = L->cnt_e;
+    p.off_e = L->off_e;
+    p.cnt_r = L->cnt_r;
+    p.off_r = L->off_r;
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.totals = L->totals;
+    const cudaError_t e = launch_layout_dispatch(p, L->idx_bits, as_stream(stream));
+    return e == cudaErrorNotSupported ? EP_ERR_UNSUPPORTED : from_cuda(e);
+}
+
+ep_status_t ep_layout_dispatch_expand(const void *topk_idx, const ep_layout_t *L, const void *x,
+                                      int32_t H, void *recv, int64_t recv_cap, void *expanded,
+                                      int64_t exp_cap, void *stream)
+{
+    return ep_layout_dispatch_expand_variant(topk_idx, L, x, H, recv, recv_cap, expanded, exp_cap,
+                                             0, stream);
 }
 
 ep_status_t ep_dispatch(const void *x, int32_t H, const ep_layout_t *L, void *recv,
@@ -188,6 +248,33 @@ ep_status_t ep_dispatch(const void *x, int32_t H, const ep_layout_t *L, void *re
     p.exp_cap = 0;
     p.err = L->totals + 3;
     return from_cuda(launch_dispatch(p, 0, as_stream(stream)));
+}
+
+ep_status_t ep_route_meta(const void *topk_idx, const float *topk_weights, const ep_layout_t *L,
+                          int32_t *meta_idx, float *meta_w, int64_t rows, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (rows < 0) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!topk_idx || !topk_weights || !meta_idx || !meta_w) return EP_ERR_INVALID_ARG;
+    if (!aligned(topk_idx, (size_t)L->idx_bits / 8) || !aligned(topk_weights, 4) ||
+        !aligned(meta_idx, 4) || !aligned(meta_w, 4))
+        return EP_ERR_MISALIGNED;
+    MetaParams p;
+    memset(&p, 0, sizeof p);
+    p.idx = topk_idx;
+    p.w = topk_weights;
+    p.recv_pos = L->recv_pos;
+    p.T = L->T;
+    p.k = L->k;
+    p.E = L->E;
+    p.R = L->R;
+    p.inv_epr = 1.0f / (float)(L->E / L->R);
+    p.meta_idx = meta_idx;
+    p.meta_w = meta_w;
+    p.rows = rows;
+    p.err = L->totals + 3;
+    return from_cuda(launch_route_meta(p, L->idx_bits, as_stream(stream)));
 }
 
 ep_status_t ep_expand_index(const ep_layout_t *L, int32_t *src_row, int64_t rows, void *stream)
@@ -412,7 +499,7 @@ size_t ep_roundtrip_device_bytes(int32_t T, int32_t H, int32_t k, int32_t E, int
 ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
                               const float *topk_weights_host, int32_t T, int32_t H, int32_t k,
                               int32_t E, int32_t R, int32_t idx_bits, void *dev_mem, size_t bytes,
-                              void *out_host, void *stream)
+                              void *out_host, int32_t *dev_err_host, void *stream)
 {
     RoundtripCarve c;
     if (!roundtrip_carve(T, H, k, E, R, idx_bits, &c)) return EP_ERR_INVALID_ARG;
@@ -428,6 +515,10 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
     ep_layout_t L;
     ep_status_t st = ep_layout_init(&L, T, k, E, R, idx_bits, d + c.lay, ep_layout_bytes(T, k, E, R));
     if (st != EP_OK) return st;
+    // the grid layout's barrier words must start at zero (the scratch may
+    // hold anything from an earlier call)
+    if (cudaMemsetAsync(L.work, 0, sizeof(int32_t) * kGridHeaderWords, s) != cudaSuccess)
+        return EP_ERR_CUDA;
     if (T > 0) {
         cudaError_t e;
         e = cudaMemcpyAsync(d + c.x, x_host, (size_t)T * row, cudaMemcpyHostToDevice, s);
@@ -438,18 +529,30 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
         e = cudaMemcpyAsync(d + c.w, topk_weights_host, (size_t)T * k * 4, cudaMemcpyHostToDevice, s);
         if (e != cudaSuccess) return EP_ERR_CUDA;
     }
-    st = ep_layout(d + c.idx, &L, stream);
+    st = ep_layout_dispatch_expand(d + c.idx, &L, d + c.x, H, d + c.recv, cap_recv, d + c.exp,
+                                   cap_exp, stream);
     if (st != EP_OK) return st;
-    if (T == 0) return EP_OK;
-    st = ep_dispatch_expand(d + c.x, H, &L, d + c.recv, cap_recv, d + c.exp, cap_exp, stream);
-    if (st != EP_OK) return st;
-    st = ep_standin_expert(d + c.exp, H, &L, d + c.y, cap_exp, stream);
-    if (st != EP_OK) return st;
-    st = ep_combine_reduce(d + c.y, reinterpret_cast<const float *>(d + c.w), H, &L, d + c.out,
-                           cap_exp, stream);
-    if (st != EP_OK) return st;
-    cudaError_t e = cudaMemcpyAsync(out_host, d + c.out, (size_t)T * row, cudaMemcpyDeviceToHost, s);
-    return from_cuda(e);
+    if (T > 0) {
+        st = ep_standin_expert(d + c.exp, H, &L, d + c.y, cap_exp, stream);
+        if (st != EP_OK) return st;
+        st = ep_combine_reduce(d + c.y, reinterpret_cast<const float *>(d + c.w), H, &L,
+                               d + c.out, cap_exp, stream);
+        if (st != EP_OK) return st;
+        const cudaError_t e =
+            cudaMemcpyAsync(out_host, d + c.out, (size_t)T * row, cudaMemcpyDeviceToHost, s);
+        if (e != cudaSuccess) return EP_ERR_CUDA;
+    }
+    // the layout's device error word (dropped routes / rows) for the caller
+    if (dev_err_host &&
+        cudaMemcpyAsync(dev_err_host, L.totals + 3, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess)
+        return EP_ERR_CUDA;
+    return EP_OK;
+}
+
+void ep_debug_dispatch_first_wait_limit(int64_t limit)
+{
+    dispatch_first_wait_limit.store(limit, std::memory_order_relaxed);
 }
 
 }  // extern "C"

@@ -25,7 +25,7 @@ constexpr int kMaxDst = EPX_MAX_TOPK + EPX_MAX_RANKS;
 
 // Warp-collective: compact the destination rows of token t into dst[0..n).
 // Expanded rows first (k order; none when p.expanded is null), then recv rows
-// (rank order).  Rows beyond a capacity are dropped and flagged.  Returns n
+// (rank order; none when p.recv is null).  Rows beyond a capacity are dropped and flagged.  Returns n
 // on every lane.
 __device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
                                               uint4 **dst)
@@ -43,7 +43,8 @@ __device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
         if (ok) dst[__popc(m & lt)] = p.expanded + (size_t)q * p.V;
         n = __popc(m);
     }
-    for (int r0 = 0; r0 < p.R; r0 += 32) {
+    // null: expand only (no recv copy)
+    for (int r0 = 0; p.recv && r0 < p.R; r0 += 32) {
         const int r = r0 + lane;
         int q = r < p.R ? p.recv_pos[(size_t)t * p.R + r] : -1;
         bool over = q >= 0 && (int64_t)q >= p.recv_cap;
@@ -126,8 +127,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes)
                  : "memory");
 }
 
-// bounded wait for phase `parity` of the barrier; false if the limit ran out
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, long long limit)
+// Warp-collective bounded wait for phase `parity` of the barrier.  Every
+// lane polls, and the warp leaves the loop together once every lane has
+// seen the phase complete, so all lanes return the same answer after the
+// same number of polls; false if `limit` polls ran out.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, unsigned parity, long long limit)
 {
     const uint32_t a = smem_addr(bar);
     for (long long i = 0; i < limit; ++i) {
@@ -139,7 +143,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity, long l
             : "=r"(done)
             : "r"(a), "r"(parity)
             : "memory");
-        if (done) return true;
+        if (__all_sync(kFull, done != 0u)) return true;
     }
     return false;
 }
@@ -171,6 +175,12 @@ __device__ __forceinline__ void bulk_commit_and_wait_read()
 // bound is far above any real completion time while still ending.
 constexpr long long kWaitLimit = 1ll << 22;
 
+}  // namespace
+
+std::atomic<long long> dispatch_first_wait_limit{-1};
+
+namespace {
+
 // One warp per CTA; the CTA handles chunk blockIdx.x (vpc vectors) of token t.
 __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
 {
@@ -183,6 +193,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
     __syncwarp();
     pdl_wait_previous();
     unsigned phase = 0;
+    bool first = true;
     const int v0 = blockIdx.x * p.vpc;
     const int nv = min(p.V, v0 + p.vpc) - v0;
     if (nv <= 0) return;
@@ -194,10 +205,15 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
             mbar_expect_tx(&bar, bytes);
             bulk_g2s(sbuf, p.x + (size_t)t * p.V + v0, bytes, &bar);
         }
-        if (!mbar_wait(&bar, phase, kWaitLimit)) {
+        // the first wait of the CTA may take a shorter limit (a test setting;
+        // kWaitLimit unless changed)
+        const long long limit = first ? p.first_wait_limit : kWaitLimit;
+        first = false;
+        if (!mbar_wait_warp(&bar, phase, limit)) {
             if (lane == 0) atomicOr(p.err, (int)EP_DEVERR_TIMEOUT);
-            // give the copy in flight a second bounded chance before leaving
-            mbar_wait(&bar, phase, kWaitLimit);
+            // leave only once the copy in flight has landed in shared memory
+            // (again a bounded wait)
+            mbar_wait_warp(&bar, phase, kWaitLimit);
             return;
         }
         phase ^= 1u;
@@ -230,6 +246,8 @@ cudaError_t launch_dispatch(const DispatchParams &p0, int variant, cudaStream_t 
         p.vpc = vpc;
         const size_t smem = (size_t)vpc * 16;  // <= 32 KB: no opt-in needed
         p.early_pdl = early_trigger((long long)chunks * gy);
+        const long long fw = dispatch_first_wait_limit.load(std::memory_order_relaxed);
+        p.first_wait_limit = fw < 0 ? kWaitLimit : fw;
         return launch_pdl(dispatch_bulk_kernel, dim3(chunks, gy), dim3(32), smem, s, p);
     }
     // vector engine: up to 128 threads x 2 vectors per pass.  Small batches

@@ -28,8 +28,33 @@ struct LayoutParams {
     int tstr;       // warp-chunk schedule: table row length in 16-bit counts (even, >= E + R)
     float inv_k;    // 1.0f / k
     int bits_e, bits_r;  // bits of the largest expert / rank
+    int hs;              // grid schedule: workspace row length in words
     int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
+    int32_t *work;       // grid schedule workspace (header + one row per CTA), or null
 };
+
+// Grid schedule of the layout: one CTA per this many routes, at most
+// kGridMaxCtas CTAs (and never more than the SMs); its workspace holds a
+// header and one row of packed 16-bit (expert | rank) counts per CTA.
+constexpr int kGridRoutesPerCta = 256;
+constexpr int kGridMaxCtas = 256;
+constexpr int kGridHeaderWords = 16;
+// the automatic layout choice takes the grid schedule above this many routes
+constexpr int kGridAutoRoutes = 8192;
+
+inline int grid_row_words(int E, int R) { return (((E + R + 1) / 2) + 3) & ~3; }
+
+inline int grid_max_ctas(long long routes)
+{
+    long long n = (routes + kGridRoutesPerCta - 1) / kGridRoutesPerCta;
+    return (int)(n < kGridMaxCtas ? n : kGridMaxCtas);
+}
+
+inline size_t grid_work_bytes(int T, int k, int E, int R)
+{
+    return sizeof(int32_t) *
+           ((size_t)kGridHeaderWords + (size_t)grid_max_ctas((long long)T * k) * grid_row_words(E, R));
+}
 
 struct DispatchParams {
     const uint4 *x;
@@ -42,6 +67,43 @@ struct DispatchParams {
     int64_t recv_cap;
     uint4 *expanded;
     int64_t exp_cap;
+    int32_t *err;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
+    long long first_wait_limit;  // bulk engine: polls allowed by a CTA's first bounded wait
+};
+
+// layout + dispatch/expand in one launch (small batches)
+struct FusedParams {
+    const void *idx;
+    const uint4 *x;
+    int T, k, E, R;
+    int V;       // 16-byte vectors per row (H / 8)
+    int vpc;     // vectors per CTA chunk
+    int chunks;  // CTAs per token
+    float inv_epr;
+    uint4 *recv;
+    int64_t recv_cap;
+    uint4 *expanded;
+    int64_t exp_cap;
+    int32_t *cnt_e, *off_e, *cnt_r, *off_r, *pos, *recv_pos, *totals;
+    int early_pdl;  // trigger dependents at start (grid fits in one wave)
+};
+
+// the one-launch layout + dispatch handles at most this many routes (T*k)
+constexpr int kFusedMaxRoutes = EPX_FUSED_MAX_ROUTES;
+// ... and is the automatic choice up to this many
+constexpr int kFusedAutoRoutes = EPX_FUSED_AUTO_ROUTES;
+
+// routing that travels with each row of a multi-GPU dispatch
+struct MetaParams {
+    const void *idx;
+    const float *w;
+    const int32_t *recv_pos;
+    int T, k, E, R;
+    float inv_epr;
+    int32_t *meta_idx;  // [rows, k]
+    float *meta_w;      // [rows, k]
+    int64_t rows;
     int32_t *err;
     int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
@@ -128,11 +190,19 @@ struct StandinParams {
 cudaError_t launch_layout(const LayoutParams &p, int idx_bits, int variant, cudaStream_t s);
 cudaError_t launch_dispatch(const DispatchParams &p, int variant, cudaStream_t s);
 cudaError_t launch_standin(const StandinParams &p, cudaStream_t s);
+// cudaErrorNotSupported when T*k > kFusedMaxRoutes
+cudaError_t launch_layout_dispatch(const FusedParams &p, int idx_bits, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
+cudaError_t launch_route_meta(const MetaParams &p, int idx_bits, cudaStream_t s);
 cudaError_t launch_local_reduce(const LocalParams &p, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueParams &p, cudaStream_t s);
 cudaError_t launch_expand_index(const IndexParams &p, cudaStream_t s);
 cudaError_t launch_standin_gather(const GatherParams &p, cudaStream_t s);
+
+// Test setting: polls allowed by the first bounded wait of every CTA of the
+// bulk copy engine (< 0: the normal limit).  Set by
+// ep_debug_dispatch_first_wait_limit.
+extern std::atomic<long long> dispatch_first_wait_limit;
 
 // ------------------------------------------------- host-side caches
 // Launchers may be called from several host threads at once.

@@ -1,0 +1,400 @@
+// Routing layout and dispatch + expand in one launch, for small batches.
+//
+// What is computed is exactly ep_layout followed by ep_dispatch_expand: the
+// layout ("handle") of DeepEP issue #760's Reproduction (dispatch returns
+// it, combine takes it back) and the copies of DeepEP issue #48 (a token is
+// received once per destination rank, then duplicated once per expert).  At
+// a handful of tokens -- the regime of the issue #760 report -- the separate
+// layout launch is a chain of dependent steps (load, count, exchange, scan,
+// place) that the dispatch must wait for; here that chain is removed:
+//
+//  * CTA (token t, chunk c) loads its chunk of x[t] into registers first, so
+//    the DRAM latency of x overlaps everything below;
+//  * it then derives its own token's rows by counting over all T*k routes
+//    (topk_idx is a few KB and stays in L2 after the first CTA reads it).
+//    In (expert, token, slot) order the row of route (t, j) with expert e is
+//    the number of valid routes before it:
+//        pos[t, j] = #{(t', j') : e' < e, or e' == e and t' < t}
+//                  + #{j' < j : e_{t, j'} == e}.
+//    With key K' = 2 e' + [t' >= t] and query Q = 2 e, the first term counts
+//    routes with K' <= Q, one compare per (route, slot).  Likewise a
+//    (token, rank) pair's row is the number of pairs (t', r') with r' < r,
+//    or r' == r and t' < t: popcount(M' & lowmask(r + [t' < t])) summed over
+//    tokens t', M' being t''s set of ranks;
+//  * the per-thread counts are summed with warp reductions, and the CTA
+//    stores its chunk to every destination row;
+//  * chunk 0 of token t writes pos[t, :] and recv_pos[t, :];
+//  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
+//    counts and exclusive scans, the totals and the error word.
+//
+// No CTA waits for another, so there is no grid-wide barrier.  The work per
+// CTA grows with T*k, so the launcher takes this kernel only for small
+// batches (routes per CTA bounded) and otherwise runs the two kernels.
+// Rows beyond a caller's capacity are skipped; the summary CTA flags them
+// (a row beyond the capacity exists exactly when the total exceeds it).
+#include "epx_internal.cuh"
+
+namespace epx {
+namespace {
+
+constexpr int kFusedThreads = 128;
+constexpr int kFusedWarps = kFusedThreads / 32;
+
+__device__ __forceinline__ int rank_of_e(int e, float inv_epr)
+{
+    // floor(e / epr), exact for e < 2^22 ((e + 1/2) / epr is at least
+    // 1/(2 epr) away from an integer, more than two fp32 roundings move it)
+    return __float2int_rd(__fmul_rn(__fadd_rn((float)e, 0.5f), inv_epr));
+}
+
+__device__ __forceinline__ unsigned long long lowmask64(int n)
+{
+    return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+}
+
+template <typename IdxT>
+__device__ __forceinline__ int load_expert(const IdxT *idx, size_t i, int E, bool *bad)
+{
+    const long long e = (long long)idx[i];
+    *bad |= (e < -1 || e >= E);
+    return (e >= 0 && e < E) ? (int)e : -1;
+}
+
+// ----------------------------------------------------------- summary CTA
+// cnt_e / off_e / cnt_r / off_r / totals for the whole batch.  Expert counts
+// are 16-bit halves of 32-bit shared words (a count is at most T*k, which the
+// launcher keeps below 2^16).
+template <typename IdxT, int KM>
+__device__ void summary_cta(const FusedParams &p, uint32_t *smem)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int E = p.E, R = p.R, k = p.k;
+    const int wde = (E + 1) >> 1;
+    uint32_t *he = smem;                  // [wde] packed 16-bit expert counts
+    int *hr = reinterpret_cast<int *>(smem + wde);  // [R] rank counts
+    int *misc = hr + R;                   // [0] bad flag, [1] real tokens
+    unsigned long long *scan = reinterpret_cast<unsigned long long *>(
+        smem + (((size_t)wde + R + 2 + 1) & ~(size_t)1));  // [kFusedWarps + 1]
+    for (int i = tid; i < wde; i += kFusedThreads) he[i] = 0u;
+    for (int i = tid; i < R; i += kFusedThreads) hr[i] = 0;
+    if (tid < 2) misc[tid] = 0;
+    __syncthreads();
+
+    const IdxT *idx = static_cast<const IdxT *>(p.idx);
+    bool bad = false;
+    int nreal = 0;
+    for (int u = tid; u < p.T; u += kFusedThreads) {
+        unsigned long long m = 0ull;
+        int ev[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j) ev[j] = j < k ? load_expert(idx, (size_t)u * k + j, E, &bad) : -1;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            const int e = ev[j];
+            if (e < 0) continue;
+            atomicAdd(&he[e >> 1], 1u << ((e & 1) * 16));
+            m |= 1ull << rank_of_e(e, p.inv_epr);
+        }
+        nreal += m != 0ull;
+        while (m) {
+            atomicAdd(&hr[__ffsll((long long)m) - 1], 1);
+            m &= m - 1ull;
+        }
+    }
+    if (__any_sync(kFull, bad) && lane == 0) atomicOr(&misc[0], 1);
+    const int wr = __reduce_add_sync(kFull, nreal);
+    if (lane == 0 && wr) atomicAdd(&misc[1], wr);
+    __syncthreads();
+
+    // one packed 64-bit exclusive scan: experts (a contiguous run per
+    // thread) in the high half, ranks (one per thread) in the low half
+    const int per = (E + kFusedThreads - 1) / kFusedThreads;
+    const int e0 = tid * per;
+    unsigned int run_e = 0;
+    for (int q = 0; q < per; ++q) {
+        const int e = e0 + q;
+        if (e < E) run_e += (he[e >> 1] >> ((e & 1) * 16)) & 0xffffu;
+    }
+    const unsigned int cr = tid < R ? (unsigned)hr[tid] : 0u;
+    // a rank beyond the first 128 threads cannot occur: R <= 64
+    const unsigned long long v = ((unsigned long long)run_e << 32) | cr;
+    unsigned long long inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long n = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) scan[wid] = inc;
+    __syncthreads();
+    if (tid == 0) {
+        unsigned long long s = 0ull;
+        for (int w = 0; w < kFusedWarps; ++w) {
+            const unsigned long long x = scan[w];
+            scan[w] = s;
+            s += x;
+        }
+        scan[kFusedWarps] = s;
+    }
+    __syncthreads();
+    const unsigned long long ex = scan[wid] + inc - v;
+    const unsigned long long total = scan[kFusedWarps];
+    unsigned int off = (unsigned int)(ex >> 32);
+    for (int q = 0; q < per; ++q) {
+        const int e = e0 + q;
+        if (e < E) {
+            const int c = (int)((he[e >> 1] >> ((e & 1) * 16)) & 0xffffu);
+            p.cnt_e[e] = c;
+            p.off_e[e] = (int)off;
+            off += c;
+        }
+    }
+    if (tid < R) {
+        p.cnt_r[tid] = (int)cr;
+        p.off_r[tid] = (int)(unsigned int)(ex & 0xffffffffull);
+    }
+    if (tid == 0) {
+        const int n_route = (int)(total >> 32);
+        const int n_recv = (int)(total & 0xffffffffull);
+        p.off_e[E] = n_route;
+        p.off_r[R] = n_recv;
+        p.totals[0] = n_route;
+        p.totals[1] = n_recv;
+        p.totals[2] = misc[1];
+        int err = misc[0] ? (int)EP_DEVERR_BAD_INDEX : 0;
+        if ((int64_t)n_recv > p.recv_cap) err |= (int)EP_DEVERR_RECV_CAP;
+        if ((int64_t)n_route > p.exp_cap) err |= (int)EP_DEVERR_EXP_CAP;
+        p.totals[3] = err;
+    }
+}
+
+// ------------------------------------------------------------ token CTAs
+
+template <typename IdxT, int KM, int VPT>
+__global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedParams p)
+{
+    extern __shared__ __align__(16) uint32_t fsmem[];
+    __shared__ int s_part[kFusedWarps][2 * KM];
+    __shared__ int s_rrow[KM];
+    __shared__ uint4 *s_dst[2 * KM];
+    __shared__ int s_n;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (p.early_pdl) pdl_launch_dependents();
+    pdl_wait_previous();
+    if (blockIdx.x == 0) {
+        summary_cta<IdxT, KM>(p, fsmem);
+        return;
+    }
+    const int b = (int)blockIdx.x - 1;
+    const int t = b / p.chunks;
+    const int c = b - t * p.chunks;
+    const int k = p.k, E = p.E, R = p.R;
+    const IdxT *idx = static_cast<const IdxT *>(p.idx);
+
+    // this token's routes (the same k values in every thread)
+    bool bad = false;
+    int q_own[KM];
+    unsigned long long m_own = 0ull;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        q_own[j] = -1;
+        if (j < k) {
+            const int e = load_expert(idx, (size_t)t * k + j, E, &bad);
+            if (e >= 0) {
+                q_own[j] = 2 * e;
+                m_own |= 1ull << rank_of_e(e, p.inv_epr);
+            }
+        }
+    }
+    if (m_own == 0ull) {  // no valid route: nothing to copy, rows of -1
+        if (c == 0) {
+            for (int j = tid; j < k; j += kFusedThreads) p.pos[(size_t)t * k + j] = -1;
+            for (int r = tid; r < R; r += kFusedThreads) p.recv_pos[(size_t)t * R + r] = -1;
+        }
+        return;
+    }
+
+    // this CTA's chunk of x[t], in flight while the rows are counted
+    const int v0 = c * p.vpc;
+    const int v1 = min(p.V, v0 + p.vpc);
+    const uint4 *src = p.x + (size_t)t * p.V;
+    uint4 val[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        const int v = v0 + tid + u * kFusedThreads;
+        if (v < v1) val[u] = ld_nc_v4(src + v);
+    }
+
+    // the token's ranks in increasing order
+    const int nr = __popcll((long long)m_own);
+    int r_own[KM];
+    {
+        unsigned long long m = m_own;
+#pragma unroll
+        for (int q = 0; q < KM; ++q) {
+            r_own[q] = 64;
+            if (m) {
+                r_own[q] = __ffsll((long long)m) - 1;
+                m &= m - 1ull;
+            }
+        }
+    }
+
+    // count routes (t', j') with 2 e' + [t' >= t] <= 2 e_j, and pairs
+    // (t', r') with r' < r_q + [t' < t]
+    int cnt[KM], cpr[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) cnt[j] = cpr[j] = 0;
+    for (int u = tid; u < p.T; u += kFusedThreads) {
+        const int after = u >= t;
+        // all k loads of the token first, so they are in flight together
+        long long ev[KM];
+#pragma unroll
+        for (int j2 = 0; j2 < KM; ++j2) ev[j2] = j2 < k ? (long long)idx[(size_t)u * k + j2] : -1;
+        unsigned long long m = 0ull;
+#pragma unroll
+        for (int j2 = 0; j2 < KM; ++j2) {
+            if (ev[j2] < 0 || ev[j2] >= E) continue;
+            const int e = (int)ev[j2];
+            const int key = 2 * e + after;
+#pragma unroll
+            for (int j = 0; j < KM; ++j) cnt[j] += key <= q_own[j];
+            m |= 1ull << rank_of_e(e, p.inv_epr);
+        }
+        if (m) {
+            const int before = 1 - after;
+#pragma unroll
+            for (int q = 0; q < KM; ++q)
+                if (q < nr) cpr[q] += __popcll((long long)(m & lowmask64(r_own[q] + before)));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        if (j < k) {
+            const int s = __reduce_add_sync(kFull, cnt[j]);
+            if (lane == 0) s_part[wid][j] = s;
+        }
+        if (j < nr) {
+            const int s = __reduce_add_sync(kFull, cpr[j]);
+            if (lane == 0) s_part[wid][KM + j] = s;
+        }
+    }
+    __syncthreads();
+
+    // warp 0: rows of the token's routes and pairs, destination list
+    if (wid == 0) {
+        const unsigned lt = lanemask_lt();
+        int e_mine = -1;
+        if (lane < k) {
+            bool b2 = false;
+            e_mine = load_expert(idx, (size_t)t * k + lane, E, &b2);
+        }
+        int dup = 0;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            const int ej = __shfl_sync(kFull, e_mine, j);
+            dup += (j < lane && ej == e_mine) ? 1 : 0;
+        }
+        int row = -1;
+        if (lane < k && e_mine >= 0) {
+            row = dup;
+#pragma unroll
+            for (int w = 0; w < kFusedWarps; ++w) row += s_part[w][lane];
+        }
+        int rrow = -1;
+        if (lane < nr) {
+            rrow = 0;
+#pragma unroll
+            for (int w = 0; w < kFusedWarps; ++w) rrow += s_part[w][KM + lane];
+            s_rrow[lane] = rrow;
+        }
+        const bool ok_e = row >= 0 && (int64_t)row < p.exp_cap;
+        const unsigned me = __ballot_sync(kFull, ok_e);
+        if (ok_e) s_dst[__popc(me & lt)] = p.expanded + (size_t)row * p.V;
+        const int ne = __popc(me);
+        const bool ok_r = rrow >= 0 && (int64_t)rrow < p.recv_cap;
+        const unsigned mr = __ballot_sync(kFull, ok_r);
+        if (ok_r) s_dst[ne + __popc(mr & lt)] = p.recv + (size_t)rrow * p.V;
+        if (lane == 0) s_n = ne + __popc(mr);
+        if (c == 0 && lane < k) p.pos[(size_t)t * k + lane] = row;
+        __syncwarp();
+        if (c == 0) {
+            for (int r = lane; r < R; r += 32) {
+                int v = -1;
+                if ((m_own >> r) & 1ull) v = s_rrow[__popcll((long long)(m_own & lowmask64(r)))];
+                p.recv_pos[(size_t)t * R + r] = v;
+            }
+        }
+    }
+    __syncthreads();
+
+    const int n = s_n;
+    for (int i = 0; i < n; ++i) {
+        uint4 *d = s_dst[i];
+#pragma unroll
+        for (int u = 0; u < VPT; ++u) {
+            const int v = v0 + tid + u * kFusedThreads;
+            if (v < v1) st_v4(d + v, val[u]);
+        }
+    }
+}
+
+template <typename IdxT, int KM>
+cudaError_t launch_km(const FusedParams &p, int vpt, dim3 grid, size_t smem, cudaStream_t s)
+{
+    switch (vpt) {
+    case 1: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 1>, grid, dim3(kFusedThreads), smem, s, p);
+    case 2: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 2>, grid, dim3(kFusedThreads), smem, s, p);
+    default: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 4>, grid, dim3(kFusedThreads), smem, s, p);
+    }
+}
+
+template <typename IdxT>
+cudaError_t launch_t(const FusedParams &p, int vpt, dim3 grid, size_t smem, cudaStream_t s)
+{
+    if (p.k <= 4) return launch_km<IdxT, 4>(p, vpt, grid, smem, s);
+    if (p.k <= 8) return launch_km<IdxT, 8>(p, vpt, grid, smem, s);
+    if (p.k <= 16) return launch_km<IdxT, 16>(p, vpt, grid, smem, s);
+    return launch_km<IdxT, 32>(p, vpt, grid, smem, s);
+}
+
+}  // namespace
+
+#ifndef EPX_FUSED_CTAS_PER_SM
+#define EPX_FUSED_CTAS_PER_SM 4
+#endif
+
+cudaError_t launch_layout_dispatch(const FusedParams &p0, int idx_bits, cudaStream_t s)
+{
+    FusedParams p = p0;
+    // per-CTA counting reads every route: small batches only (this also keeps
+    // the summary CTA's 16-bit expert counts below 2^16)
+    if ((long long)p.T * p.k > kFusedMaxRoutes) return cudaErrorNotSupported;
+    const int nsm = current_sm_count();
+    int chunks = 1, vpt = 1;
+    if (p.T > 0) {
+        // about EPX_FUSED_CTAS_PER_SM CTAs per SM, chunks of >= 32 vectors,
+        // at most four vectors per thread
+        chunks = (EPX_FUSED_CTAS_PER_SM * nsm + p.T - 1) / p.T;
+        const int max_chunks = (p.V + 31) / 32;
+        if (chunks > max_chunks) chunks = max_chunks;
+        const int min_chunks = (p.V + 4 * kFusedThreads - 1) / (4 * kFusedThreads);
+        if (chunks < min_chunks) chunks = min_chunks;
+        if (chunks < 1) chunks = 1;
+        p.vpc = (p.V + chunks - 1) / chunks;
+        chunks = (p.V + p.vpc - 1) / p.vpc;
+        vpt = (p.vpc + kFusedThreads - 1) / kFusedThreads;
+        vpt = vpt <= 1 ? 1 : vpt <= 2 ? 2 : 4;
+    }
+    p.chunks = chunks;
+    const long long ctas = 1 + (long long)p.T * chunks;
+    if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;
+    // summary CTA: packed expert counts, rank counts, flags, scan scratch
+    const size_t smem = (((size_t)(p.E + 1) / 2 + p.R + 2 + 1) & ~(size_t)1) * 4 +
+                        (kFusedWarps + 1) * 8;
+    p.early_pdl = early_trigger(ctas);
+    const dim3 grid((unsigned)ctas);
+    return idx_bits == 64 ? launch_t<long long>(p, vpt, grid, smem, s)
+                          : launch_t<int>(p, vpt, grid, smem, s);
+}
+
+}  // namespace epx

@@ -73,7 +73,9 @@ struct Smem {
     int32_t *tot;             // [E + R] CTA totals / chunk sums
     int32_t *base;            // [E + R] this CTA's first row per expert / rank
     int32_t *all_tot;         // [csize][E + R + 2] every CTA's totals, bad flag, real tokens
+                              // (grid schedule: partial column sums)
     int32_t *misc;            // [2] bad flag, real tokens
+    int32_t *low;             // grid schedule: [E + R] totals of the CTAs below this one
     unsigned long long *scan; // [34] block-scan scratch
 };
 
@@ -262,12 +264,19 @@ __host__ __device__ size_t matrix_words(int wdt, int ld)
     return ((size_t)wdt * ld + 3) & ~(size_t)3;
 }
 
+// How CTA totals reach the global scan: one CTA; a thread-block cluster
+// (distributed shared memory); a grid (sums already in sm.tot / sm.low).
+constexpr int kModeSingle = 0, kModeCluster = 1, kModeGrid = 2;
+
 // Cluster exchange of the CTA totals in sm.tot (and sm.misc), then one packed
 // 64-bit block scan: writes cnt / off / totals (CTA 0) and this CTA's first
-// row per expert and rank into sm.base.  Ends without a barrier.
-template <bool CLUSTER>
+// row per expert and rank into sm.base.  In grid mode sm.tot already holds
+// the grid totals and sm.low the totals of the CTAs below this one, and
+// totals[2..3] are left to the grid's last CTA.  Ends without a barrier.
+template <int MODE>
 __device__ void global_offsets(const LayoutParams &p, const Smem &sm, int crank, int csize)
 {
+    constexpr bool CLUSTER = MODE == kModeCluster;
     const int tid = threadIdx.x;
     const int E = p.E, R = p.R;
     const int W = E + R + 2;
@@ -289,6 +298,11 @@ __device__ void global_offsets(const LayoutParams &p, const Smem &sm, int crank,
         // this CTA's totals sum over the cluster: all CTAs (glob) and the
         // CTAs below this one (lower), read from the local table
         auto sums = [&](int i, int &g, int &lo) {
+            if (MODE == kModeGrid) {
+                g = sm.tot[i];
+                lo = sm.low[i];
+                return;
+            }
             if (!CLUSTER) {
                 g = sm.tot[i];
                 lo = 0;
@@ -356,8 +370,10 @@ __device__ void global_offsets(const LayoutParams &p, const Smem &sm, int crank,
             p.off_r[R] = n_recv;
             p.totals[0] = n_route;
             p.totals[1] = n_recv;
-            p.totals[2] = nr;
-            p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
+            if (MODE != kModeGrid) {
+                p.totals[2] = nr;
+                p.totals[3] = errc ? (int32_t)EP_DEVERR_BAD_INDEX : 0;
+            }
         }
     }
 }
@@ -419,7 +435,7 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     if (nreal) atomicAdd(&sm.misc[1], nreal);
     __syncthreads();
 
-    global_offsets<CLUSTER>(p, sm, crank, csize);
+    global_offsets<CLUSTER ? kModeCluster : kModeSingle>(p, sm, crank, csize);
     __syncthreads();
 
     // ---- positions
@@ -486,50 +502,39 @@ __host__ __device__ size_t warp_table_words(int nch, int wt)
     return ((size_t)nch * wt + 3) & ~(size_t)3;
 }
 
-template <typename IdxT, bool CLUSTER, int PASSES>
-__global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
+// Per-lane state of the warp-chunk schedule, one entry per pass of the
+// CTA's warps over its tokens.
+template <int PASSES>
+struct WarpRoutes {
+    int ex[PASSES];    // expert of the route, -1 for none
+    int re_e[PASSES];  // rank among the warp's earlier routes to that expert
+    int rk[PASSES];    // rank of the (token, rank) pair this route opens, -1 if none
+    int re_r[PASSES];  // rank among the warp's earlier pairs of that rank
+    int tl, j;         // token within the warp's chunk, slot
+};
+
+// Count phase of the warp-chunk schedule over tokens [c0, c0 + nt) (the
+// table `tab` is zero, sm.misc cleared, and the previous kernel waited for):
+// fills this CTA's recv_pos rows with -1, matches routes within each warp,
+// writes the chunk x (expert | rank) table, turns every column into its
+// exclusive prefix over chunks and leaves the CTA totals in sm.tot[E + R],
+// the bad-index flag in sm.misc[0] and the real-token count in sm.misc[1].
+// Ends with a barrier.
+template <typename IdxT, int PASSES>
+__device__ __forceinline__ void warp_count(const LayoutParams &p, uint32_t *tab, const Smem &sm,
+                                           int c0, int nt, WarpRoutes<PASSES> &wr)
 {
-    extern __shared__ __align__(16) int32_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int NW = blockDim.x >> 5;
-    const int E = p.E, R = p.R, T = p.T, k = p.k, tpw = p.tpw;
-    pdl_launch_dependents();
-
-    int crank = 0, csize = 1;
-    if (CLUSTER) {
-        cg::cluster_group cluster = cg::this_cluster();
-        crank = (int)cluster.block_rank();
-        csize = (int)cluster.num_blocks();
-    }
-    const int W = E + R + 2;
-    const int wt = p.tstr >> 1;  // table row length in 32-bit words
-    const int nch_max = (p.tpc + tpw - 1) / tpw;
-
-    uint32_t *tab = reinterpret_cast<uint32_t *>(smem);  // [chunks][wt]
-    Smem sm;
-    sm.M = nullptr;
-    sm.codes = nullptr;
-    sm.hit = nullptr;
-    sm.scan = reinterpret_cast<unsigned long long *>(smem + warp_table_words(nch_max, wt));
-    sm.tot = reinterpret_cast<int32_t *>(sm.scan + 34);
-    sm.base = sm.tot + E + R;
-    sm.all_tot = sm.base + E + R;
-    sm.misc = sm.all_tot + (size_t)csize * W;
-
-    const IdxT *idx = static_cast<const IdxT *>(p.idx);
-    const int c0 = min(T, crank * p.tpc);
-    const int nt = min(T, c0 + p.tpc) - c0;
+    const int E = p.E, R = p.R, k = p.k, tpw = p.tpw;
+    const int wt = p.tstr >> 1;
     const int nuse = (nt + tpw - 1) / tpw;  // chunks holding tokens
-
-    // prologue in shared memory only, so it may overlap the previous kernel
-    if (tid < 2) sm.misc[tid] = 0;
-    zero_words(tab, nuse * wt);
-    __syncthreads();
-    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-    pdl_wait_previous();
+    const IdxT *idx = static_cast<const IdxT *>(p.idx);
 
     const int tl = div_small(lane, p.inv_k);  // token of this lane within its chunk
     const int j = lane - tl * k;              // slot
+    wr.tl = tl;
+    wr.j = j;
     const unsigned lt = lanemask_lt();
     IdxT raw[PASSES];
 #pragma unroll
@@ -547,7 +552,6 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
 
     bool bad = false;
     int nreal = 0;
-    int re_e[PASSES], re_r[PASSES], rk[PASSES], ex[PASSES];
     const unsigned kmask = k == 32 ? kFull : ((1u << k) - 1u);
     const unsigned tokmask = tl < tpw ? kmask << (tl * k) : 0u;  // lanes of this lane's token
 #pragma unroll
@@ -567,10 +571,10 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
         if (v && !(pe & lt)) row[e] = (uint16_t)__popc(pe);
         if (first && !(pf & lt)) row[E + r] = (uint16_t)__popc(pf);
         nreal += j == 0 && (vb & tokmask) != 0u;
-        ex[q] = v ? e : -1;
-        re_e[q] = __popc(pe & lt);
-        rk[q] = first ? r : -1;
-        re_r[q] = __popc(pf & lt);
+        wr.ex[q] = v ? e : -1;
+        wr.re_e[q] = __popc(pe & lt);
+        wr.rk[q] = first ? r : -1;
+        wr.re_r[q] = __popc(pf & lt);
     }
     __syncthreads();
 
@@ -594,23 +598,256 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
     if (__any_sync(kFull, bad) && lane == 0) atomicOr(&sm.misc[0], 1);
     if (nreal) atomicAdd(&sm.misc[1], nreal);
     __syncthreads();
+}
 
-    global_offsets<CLUSTER>(p, sm, crank, csize);
-    __syncthreads();
-
+// Placement phase: pos and recv_pos of every route this lane holds, from the
+// bases in sm.base, the chunk prefixes in `tab` and the in-warp ranks.
+template <int PASSES>
+__device__ __forceinline__ void warp_place(const LayoutParams &p, const uint32_t *tab,
+                                           const Smem &sm, int c0, int nt,
+                                           const WarpRoutes<PASSES> &wr)
+{
+    const int wid = threadIdx.x >> 5;
+    const int NW = blockDim.x >> 5;
+    const int E = p.E, R = p.R, k = p.k, tpw = p.tpw;
+    const int wt = p.tstr >> 1;
 #pragma unroll
     for (int q = 0; q < PASSES; ++q) {
         const int c = q * NW + wid;
-        const int u = c * tpw + tl;
-        if (tl < tpw && u < nt) {
+        const int u = c * tpw + wr.tl;
+        if (wr.tl < tpw && u < nt) {
             const uint16_t *row = reinterpret_cast<const uint16_t *>(tab + (size_t)c * wt);
-            const int e = ex[q];
-            p.pos[(size_t)(c0 + u) * k + j] = e < 0 ? -1 : sm.base[e] + (int)row[e] + re_e[q];
-            const int r = rk[q];
+            const int e = wr.ex[q];
+            p.pos[(size_t)(c0 + u) * k + wr.j] =
+                e < 0 ? -1 : sm.base[e] + (int)row[e] + wr.re_e[q];
+            const int r = wr.rk[q];
             if (r >= 0)
-                p.recv_pos[(size_t)(c0 + u) * R + r] = sm.base[E + r] + (int)row[E + r] + re_r[q];
+                p.recv_pos[(size_t)(c0 + u) * R + r] =
+                    sm.base[E + r] + (int)row[E + r] + wr.re_r[q];
         }
     }
+}
+
+template <typename IdxT, bool CLUSTER, int PASSES>
+__global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
+{
+    extern __shared__ __align__(16) int32_t smem[];
+    const int tid = threadIdx.x;
+    const int E = p.E, R = p.R, T = p.T, tpw = p.tpw;
+    pdl_launch_dependents();
+
+    int crank = 0, csize = 1;
+    if (CLUSTER) {
+        cg::cluster_group cluster = cg::this_cluster();
+        crank = (int)cluster.block_rank();
+        csize = (int)cluster.num_blocks();
+    }
+    const int W = E + R + 2;
+    const int wt = p.tstr >> 1;  // table row length in 32-bit words
+    const int nch_max = (p.tpc + tpw - 1) / tpw;
+
+    uint32_t *tab = reinterpret_cast<uint32_t *>(smem);  // [chunks][wt]
+    Smem sm;
+    sm.M = nullptr;
+    sm.codes = nullptr;
+    sm.hit = nullptr;
+    sm.low = nullptr;
+    sm.scan = reinterpret_cast<unsigned long long *>(smem + warp_table_words(nch_max, wt));
+    sm.tot = reinterpret_cast<int32_t *>(sm.scan + 34);
+    sm.base = sm.tot + E + R;
+    sm.all_tot = sm.base + E + R;
+    sm.misc = sm.all_tot + (size_t)csize * W;
+
+    const int c0 = min(T, crank * p.tpc);
+    const int nt = min(T, c0 + p.tpc) - c0;
+    const int nuse = (nt + tpw - 1) / tpw;  // chunks holding tokens
+
+    // prologue in shared memory only, so it may overlap the previous kernel
+    if (tid < 2) sm.misc[tid] = 0;
+    zero_words(tab, nuse * wt);
+    __syncthreads();
+    if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    pdl_wait_previous();
+
+    WarpRoutes<PASSES> wr;
+    warp_count<IdxT, PASSES>(p, tab, sm, c0, nt, wr);
+    global_offsets<CLUSTER ? kModeCluster : kModeSingle>(p, sm, crank, csize);
+    __syncthreads();
+    warp_place<PASSES>(p, tab, sm, c0, nt, wr);
+}
+
+// --------------------------------------------------------- grid schedule
+//
+// For large batches the warp-chunk schedule spreads over many CTAs of one
+// ordinary grid -- up to one per SM, each with a few hundred routes -- in
+// place of one cluster of at most 16.  CTA totals cannot go through
+// distributed shared memory across a grid, so they go through a workspace
+// in global memory:
+//  * count phase as above, then the CTA's (expert | rank) totals are stored
+//    as one row of packed 16-bit counts;
+//  * one grid barrier: every CTA adds one to an arrival counter and waits
+//    (bounded: after kGridWaitLimit polls it flags EP_DEVERR_TIMEOUT and goes
+//    on) until all have arrived.  The grid never has more CTAs than SMs, and
+//    programmatic launch lets dependent grids start only once every CTA of
+//    this one has started, so all CTAs are resident together;
+//  * every CTA sums the rows -- over all CTAs (the totals) and over the CTAs
+//    below it (its bases) -- with many 16-byte loads in flight per thread,
+//    then runs the packed block scan and places its routes;
+//  * bad-index and real-token counts go into two more header words, and the
+//    last CTA to leave writes them to totals[2..3] and zeroes the header, so
+//    the workspace is clean after every call (it must be zero before the
+//    first one).
+constexpr int kGridHeader = kGridHeaderWords;  // workspace header words (first four used)
+constexpr long long kGridWaitLimit = 1ll << 21;
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+constexpr int kGridMaxThreads = 512;
+
+template <typename IdxT, int PASSES>
+__global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutParams p)
+{
+    // no static shared memory: the dynamic part may take the whole 227 KB
+    extern __shared__ __align__(16) int32_t smem[];
+    const int tid = threadIdx.x;
+    const int E = p.E, R = p.R, T = p.T, tpw = p.tpw;
+    const int nb = (int)gridDim.x, b = (int)blockIdx.x;
+    // dependents start launching only once every CTA of this grid has passed
+    // this point, i.e. once all of them are resident
+    pdl_launch_dependents();
+
+    const int wt = p.tstr >> 1;
+    const int hs = p.hs;  // workspace row length in words (multiple of 4, >= wt)
+    const int nch_max = (p.tpc + tpw - 1) / tpw;
+    const int nq = hs >> 2;
+    const int G = (int)blockDim.x / nq > 1 ? (int)blockDim.x / nq : 1;
+
+    uint32_t *tab = reinterpret_cast<uint32_t *>(smem);  // [chunks][wt]
+    Smem sm;
+    sm.M = nullptr;
+    sm.codes = nullptr;
+    sm.hit = nullptr;
+    sm.scan = reinterpret_cast<unsigned long long *>(smem + warp_table_words(nch_max, wt));
+    sm.tot = reinterpret_cast<int32_t *>(sm.scan + 34);
+    sm.base = sm.tot + E + R;
+    sm.low = sm.base + E + R;
+    sm.misc = sm.low + E + R;  // [0] bad flag, [1] real tokens, [2] barrier gave up
+    sm.all_tot = sm.misc + 3;  // [G][2][2 * hs] partial sums
+    int *s_fail = sm.misc + 2;
+
+    const int c0 = min(T, b * p.tpc);
+    const int nt = min(T, c0 + p.tpc) - c0;
+    const int nuse = (nt + tpw - 1) / tpw;
+
+    if (tid < 2) sm.misc[tid] = 0;
+    zero_words(tab, nuse * wt);
+    __syncthreads();
+    pdl_wait_previous();
+
+    WarpRoutes<PASSES> wr;
+    warp_count<IdxT, PASSES>(p, tab, sm, c0, nt, wr);
+
+    // ---- publish this CTA's totals, then the grid barrier
+    int32_t *hdr = p.work;
+    uint32_t *rows = reinterpret_cast<uint32_t *>(p.work + kGridHeader);
+    for (int w = tid; w < hs; w += blockDim.x) {
+        const uint32_t lo = 2 * w < E + R ? (uint32_t)sm.tot[2 * w] : 0u;
+        const uint32_t hi = 2 * w + 1 < E + R ? (uint32_t)sm.tot[2 * w + 1] : 0u;
+        rows[(size_t)b * hs + w] = lo | (hi << 16);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if (sm.misc[0]) atomicOr(&hdr[2], (int)EP_DEVERR_BAD_INDEX);
+        if (sm.misc[1]) atomicAdd(&hdr[3], sm.misc[1]);
+        __threadfence();
+        atomicAdd(&hdr[0], 1);
+        bool ok = false;
+        for (long long i = 0; i < kGridWaitLimit; ++i) {
+            if (ld_acquire_gpu(&hdr[0]) >= nb) {
+                ok = true;
+                break;
+            }
+            __nanosleep(32);
+        }
+        if (!ok) atomicOr(&hdr[2], (int)EP_DEVERR_TIMEOUT);
+        *s_fail = ok ? 0 : 1;
+        __threadfence();
+    }
+    __syncthreads();
+
+    // ---- column sums over all CTAs and over the CTAs below this one
+    for (int i = tid; i < nq * G; i += blockDim.x) {
+        const int q = i % nq, g = i / nq;
+        const int b0 = g * nb / G, b1 = (g + 1) * nb / G;
+        uint32_t tot[8], low[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) tot[u] = low[u] = 0u;
+        for (int bb = b0; bb < b1; bb += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (bb + u < b1)
+                    v[u] = __ldcg(reinterpret_cast<const uint4 *>(rows + (size_t)(bb + u) * hs) + q);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (bb + u < b1) {
+                    const uint32_t x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                    const bool below = bb + u < b;
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        tot[2 * h] += x4[h] & 0xffffu;
+                        tot[2 * h + 1] += x4[h] >> 16;
+                        if (below) {
+                            low[2 * h] += x4[h] & 0xffffu;
+                            low[2 * h + 1] += x4[h] >> 16;
+                        }
+                    }
+                }
+            }
+        }
+        uint32_t *pt = reinterpret_cast<uint32_t *>(sm.all_tot) + (size_t)g * 4 * hs;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            pt[8 * q + u] = tot[u];
+            pt[2 * hs + 8 * q + u] = low[u];
+        }
+    }
+    __syncthreads();
+    for (int c = tid; c < E + R; c += blockDim.x) {
+        uint32_t t = 0, l = 0;
+        for (int g = 0; g < G; ++g) {
+            const uint32_t *pt = reinterpret_cast<const uint32_t *>(sm.all_tot) + (size_t)g * 4 * hs;
+            t += pt[c];
+            l += pt[2 * hs + c];
+        }
+        sm.tot[c] = (int32_t)t;
+        sm.low[c] = (int32_t)l;
+    }
+    __syncthreads();
+    // this CTA no longer reads the workspace: leave (the last one out
+    // publishes the header's counts and zeroes it)
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&hdr[1], 1) == nb - 1) {
+            p.totals[2] = atomicExch(&hdr[3], 0);
+            p.totals[3] = atomicExch(&hdr[2], 0);
+            atomicExch(&hdr[0], 0);
+            atomicExch(&hdr[1], 0);
+        }
+    }
+
+    global_offsets<kModeGrid>(p, sm, b, nb);
+    __syncthreads();
+    if (*s_fail) {  // the sums are not trustworthy: no route gets a row
+        for (int i = tid; i < nt * p.k; i += blockDim.x) p.pos[(size_t)c0 * p.k + i] = -1;
+        return;
+    }
+    warp_place<PASSES>(p, tab, sm, c0, nt, wr);
 }
 
 // ------------------------------------------------------------------- host
@@ -701,6 +938,39 @@ bool plan_warp(int T, int k, int E, int R, int csize, WarpGeometry *g)
     }
 }
 
+// Grid-schedule geometry: CTAs of ~kGridRoutesPerCta routes (at most one
+// per SM), warps and passes as in the warp-chunk schedule; false when fewer
+// than two CTAs would be used or shared memory does not suffice.
+bool plan_grid(int T, int k, int E, int R, int nsm, WarpGeometry *g, int *hs)
+{
+    const long long routes = (long long)T * k;
+    int nb = grid_max_ctas(routes);
+    if (nb > nsm) nb = nsm;
+    if (nb < 2) return false;
+    g->tpw = 32 / k;
+    g->tstr = (E + R + 1) & ~1;
+    g->tpc = (T + nb - 1) / nb;
+    g->csize = (T + g->tpc - 1) / g->tpc;  // CTAs that hold tokens
+    if (g->csize < 2) return false;
+    const int nch = (g->tpc + g->tpw - 1) / g->tpw;
+    int min_threads = (E + 3) / 4 > R ? (E + 3) / 4 : R;
+    min_threads = ((min_threads + 31) / 32) * 32;
+    int warps = 8;
+    while (warps * 32 < kGridMaxThreads && nch > 4 * warps) warps *= 2;
+    if (warps * 32 < min_threads) warps = (min_threads + 31) / 32;
+    if (warps * 32 > kGridMaxThreads) return false;
+    const int passes = (nch + warps - 1) / warps;
+    if (passes > 4) return false;
+    g->passes = passes <= 1 ? 1 : passes <= 2 ? 2 : 4;
+    g->threads = warps * 32;
+    *hs = grid_row_words(E, R);
+    const int nq = *hs / 4;
+    const int G = g->threads / nq > 1 ? g->threads / nq : 1;
+    g->smem = warp_table_words(nch, g->tstr >> 1) * 4 + 34 * 8 +
+              sizeof(int32_t) * (3 * (size_t)(E + R) + 3) + sizeof(uint32_t) * (size_t)G * 4 * *hs;
+    return g->smem <= (size_t)kMaxDynSmem;
+}
+
 using LayoutKernel = void (*)(LayoutParams);
 
 template <typename IdxT, bool CLUSTER>
@@ -749,6 +1019,14 @@ int max_clusters(LayoutKernel fn, int csize, int threads, size_t smem, int dev)
 }
 
 template <typename IdxT>
+LayoutKernel grid_kernel(int passes)
+{
+    return passes == 1   ? layout_grid_kernel<IdxT, 1>
+           : passes == 2 ? layout_grid_kernel<IdxT, 2>
+                         : layout_grid_kernel<IdxT, 4>;
+}
+
+template <typename IdxT>
 cudaError_t set_attributes_once(int dev)
 {
     static std::atomic<unsigned> done{0};  // per device (up to 32)
@@ -758,6 +1036,11 @@ cudaError_t set_attributes_once(int dev)
     const LayoutKernel clustered[] = {layout_kernel<IdxT, true>, warp_kernel<IdxT, true>(1),
                                       warp_kernel<IdxT, true>(2), warp_kernel<IdxT, true>(4)};
     cudaError_t err = cudaSuccess;
+    const LayoutKernel grid[] = {grid_kernel<IdxT>(1), grid_kernel<IdxT>(2), grid_kernel<IdxT>(4)};
+    for (LayoutKernel fn : grid)
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxDynSmem);
     for (LayoutKernel fn : single)
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -773,9 +1056,10 @@ cudaError_t set_attributes_once(int dev)
     return err;
 }
 
-// variant: 0 = warp chunks where they fit, else the count matrix;
-// 1 = warp chunks (cudaErrorNotSupported where they do not fit);
-// 2 = count matrix
+// variant: 0 = the grid schedule for large batches, else warp chunks where
+// they fit, else the count matrix; 1 = warp chunks (cudaErrorNotSupported
+// where they do not fit); 2 = count matrix; 3 = grid schedule
+// (cudaErrorNotSupported without a workspace or where it does not fit)
 template <typename IdxT>
 cudaError_t launch_layout_t(const LayoutParams &p0, int variant, cudaStream_t s)
 {
@@ -787,6 +1071,22 @@ cudaError_t launch_layout_t(const LayoutParams &p0, int variant, cudaStream_t s)
 
     LayoutParams p = p0;
     const long long routes = (long long)p.T * p.k;
+    if (variant == 3 || (variant == 0 && routes > kGridAutoRoutes && p.work)) {
+        WarpGeometry g;
+        int hs = 0;
+        if (p.work && plan_grid(p.T, p.k, p.E, p.R, sm_count(dev), &g, &hs)) {
+            p.tpc = g.tpc;
+            p.tpw = g.tpw;
+            p.tstr = g.tstr;
+            p.hs = hs;
+            p.inv_k = 1.0f / (float)p.k;
+            p.bits_e = bits_for(p.E);
+            p.bits_r = bits_for(p.R);
+            return launch_pdl(grid_kernel<IdxT>(g.passes), dim3(g.csize), dim3(g.threads),
+                              g.smem, s, p);
+        }
+        if (variant == 3) return cudaErrorNotSupported;
+    }
     // one CTA up to ~2K routes, then a cluster of up to 16 CTAs
     int csize = (int)((routes + 2047) / 2048);
     csize = csize < 1 ? 1 : (csize > 16 ? 16 : csize);

@@ -54,7 +54,8 @@ ep_status_t scratch_address(void **out)
 extern "C" ep_status_t ep_roundtrip_host_noalloc(const void *x_host, const void *topk_idx_host,
                                                  const float *topk_weights_host, int32_t T,
                                                  int32_t H, int32_t k, int32_t E, int32_t R,
-                                                 int32_t idx_bits, void *out_host, void *stream)
+                                                 int32_t idx_bits, void *out_host,
+                                                 int32_t *dev_err_host, void *stream)
 {
     const size_t need = ep_roundtrip_device_bytes(T, H, k, E, R, idx_bits);
     if (need == 0) return EP_ERR_INVALID_ARG;
@@ -63,5 +64,6 @@ extern "C" ep_status_t ep_roundtrip_host_noalloc(const void *x_host, const void 
     const ep_status_t st = scratch_address(&base);
     if (st != EP_OK) return st;
     return ep_roundtrip_host(x_host, topk_idx_host, topk_weights_host, T, H, k, E, R, idx_bits,
-                             base, (size_t)EPX_NOALLOC_SCRATCH_BYTES, out_host, stream);
+                             base, (size_t)EPX_NOALLOC_SCRATCH_BYTES, out_host, dev_err_host,
+                             stream);
 }

@@ -22,15 +22,18 @@ import torch
 __all__ = [
     "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
     "combine_reduce", "combine_local_reduce", "combine_epilogue", "read_totals",
-    "dispatch", "expand_index", "standin_expert_gather",
+    "dispatch", "expand_index", "standin_expert_gather", "layout_dispatch_expand",
+    "latency_floor", "route_meta",
     "roundtrip_host", "roundtrip_device_bytes",
-    "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES", "debug_dispatch_first_wait_limit",
     "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libepx.so")
 MAX_TOPK, MAX_RANKS, MAX_EXPERTS = 32, 64, 4096
 NOALLOC_SCRATCH_BYTES = 64 << 20  # EPX_NOALLOC_SCRATCH_BYTES
+FUSED_MAX_ROUTES = 8192           # EPX_FUSED_MAX_ROUTES
+FUSED_AUTO_ROUTES = 2048          # EPX_FUSED_AUTO_ROUTES
 
 EP_OK = 0
 _STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_MISALIGNED", 3: "EP_ERR_CAPACITY",
@@ -50,7 +53,7 @@ class _LayoutC(ctypes.Structure):
                 ("cnt_e", ctypes.c_void_p), ("off_e", ctypes.c_void_p),
                 ("cnt_r", ctypes.c_void_p), ("off_r", ctypes.c_void_p),
                 ("pos", ctypes.c_void_p), ("recv_pos", ctypes.c_void_p),
-                ("totals", ctypes.c_void_p)]
+                ("totals", ctypes.c_void_p), ("work", ctypes.c_void_p)]
 
 
 _lib = None
@@ -87,8 +90,15 @@ def lib():
         "ep_layout_read_totals": ([LP, ctypes.POINTER(I64), ctypes.POINTER(I64),
                                    ctypes.POINTER(I64), ctypes.POINTER(I32), P], I32),
         "ep_roundtrip_device_bytes": ([I32, I32, I32, I32, I32, I32], SZ),
-        "ep_roundtrip_host": ([P, P, P, I32, I32, I32, I32, I32, I32, P, SZ, P, P], I32),
-        "ep_roundtrip_host_noalloc": ([P, P, P, I32, I32, I32, I32, I32, I32, P, P], I32),
+        "ep_roundtrip_host": ([P, P, P, I32, I32, I32, I32, I32, I32, P, SZ, P,
+                               ctypes.POINTER(I32), P], I32),
+        "ep_roundtrip_host_noalloc": ([P, P, P, I32, I32, I32, I32, I32, I32, P,
+                                       ctypes.POINTER(I32), P], I32),
+        "ep_debug_dispatch_first_wait_limit": ([I64], None),
+        "ep_layout_dispatch_expand": ([P, LP, P, I32, P, I64, P, I64, P], I32),
+        "ep_layout_dispatch_expand_variant": ([P, LP, P, I32, P, I64, P, I64, I32, P], I32),
+        "ep_latency_floor": ([P, I64, I32, P], I32),
+        "ep_route_meta": ([P, P, LP, P, P, I64, P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -127,7 +137,8 @@ class Layout:
         if nbytes == 0:
             raise EpxError(6 if (k > MAX_TOPK or R > MAX_RANKS or E > MAX_EXPERTS) else 1,
                            f"ep_layout_bytes(T={T}, k={k}, E={E}, R={R})")
-        self.mem = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        # zeroed: the grid layout schedule's barrier words start at zero
+        self.mem = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.c = _LayoutC()
         _check(lib().ep_layout_init(ctypes.byref(self.c), T, k, E, R, idx_bits,
                                     self.mem.data_ptr(), nbytes), "ep_layout_init")
@@ -162,7 +173,8 @@ class Layout:
 def layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, out: Layout = None,
            variant: int = 0, stream=None) -> Layout:
     """ep_layout: routing layout of topk_idx (int32 or int64 [T, k], -1 = none).
-    variant: 0 automatic, 1 warp chunks, 2 count matrix (same results)."""
+    variant: 0 automatic, 1 warp chunks, 2 count matrix, 3 grid of up to one
+    CTA per SM (same results)."""
     if topk_idx.dim() != 2:
         raise ValueError("topk_idx must be [T, k]")
     T, k = topk_idx.shape
@@ -179,13 +191,50 @@ def layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, out: Layout
 
 
 def dispatch_expand(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None,
-                    expanded: torch.Tensor = None, variant: int = 0, stream=None):
+                    expanded: torch.Tensor = None, variant: int = 0, stream=None,
+                    expand_only: bool = False):
     """ep_dispatch_expand: returns (recv [T*min(k,R), H], expanded [T*k, H]) bf16;
-    rows past N_recv / N_route are left as allocated."""
+    rows past N_recv / N_route are left as allocated.  expand_only: no recv
+    copy (recv is None in the result)."""
     if x.dim() != 2 or x.shape[0] != lay.T:
         raise ValueError("x must be [T, H]")
     H = x.shape[1]
     xp = _dev(x, "x", torch.bfloat16)
+    if recv is None and not expand_only:
+        recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=x.device)
+    if expanded is None:
+        expanded = torch.empty((lay.exp_cap, H), dtype=torch.bfloat16, device=x.device)
+    for name, t in (("recv", recv), ("expanded", expanded)):
+        if t is not None and (t.dim() != 2 or t.shape[1] != H):
+            raise ValueError(f"{name} must be [rows, {H}]")
+    _check(lib().ep_dispatch_expand_variant(
+        xp, H, lay.ref, None if recv is None else _dev(recv, "recv", torch.bfloat16),
+        0 if recv is None else recv.shape[0],
+        _dev(expanded, "expanded", torch.bfloat16), expanded.shape[0], variant,
+        _stream(stream)), "ep_dispatch_expand")
+    return recv, expanded
+
+
+def layout_dispatch_expand(topk_idx: torch.Tensor, x: torch.Tensor, num_experts: int,
+                           num_ranks: int, out: Layout = None, recv: torch.Tensor = None,
+                           expanded: torch.Tensor = None, variant: int = 0, stream=None):
+    """ep_layout_dispatch_expand: layout + dispatch/expand in one call (one
+    launch for small batches).  Returns (layout, recv, expanded); the same
+    results as layout() followed by dispatch_expand().
+    variant: 0 automatic, 1 one launch, 2 two launches."""
+    if topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be [T, k]")
+    T, k = topk_idx.shape
+    bits = {torch.int64: 64, torch.int32: 32}.get(topk_idx.dtype)
+    if bits is None:
+        raise TypeError("topk_idx must be int32 or int64")
+    if x.dim() != 2 or x.shape[0] != T:
+        raise ValueError("x must be [T, H]")
+    H = x.shape[1]
+    lay = out if out is not None else Layout(T, k, num_experts, num_ranks, bits,
+                                             device=topk_idx.device)
+    if (lay.T, lay.k, lay.E, lay.R, lay.idx_bits) != (T, k, num_experts, num_ranks, bits):
+        raise ValueError("layout buffer does not match the sizes")
     if recv is None:
         recv = torch.empty((lay.recv_cap, H), dtype=torch.bfloat16, device=x.device)
     if expanded is None:
@@ -193,11 +242,40 @@ def dispatch_expand(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None,
     for name, t in (("recv", recv), ("expanded", expanded)):
         if t.dim() != 2 or t.shape[1] != H:
             raise ValueError(f"{name} must be [rows, {H}]")
-    _check(lib().ep_dispatch_expand_variant(
-        xp, H, lay.ref, _dev(recv, "recv", torch.bfloat16), recv.shape[0],
+    _check(lib().ep_layout_dispatch_expand_variant(
+        _dev(topk_idx, "topk_idx"), lay.ref, _dev(x, "x", torch.bfloat16), H,
+        _dev(recv, "recv", torch.bfloat16), recv.shape[0],
         _dev(expanded, "expanded", torch.bfloat16), expanded.shape[0], variant,
-        _stream(stream)), "ep_dispatch_expand")
-    return recv, expanded
+        _stream(stream)), "ep_layout_dispatch_expand")
+    return lay, recv, expanded
+
+
+def route_meta(topk_idx: torch.Tensor, topk_weights: torch.Tensor, lay: Layout,
+               meta_idx: torch.Tensor = None, meta_w: torch.Tensor = None, stream=None):
+    """ep_route_meta: per sent row (recv_pos order), the token's routes kept on
+    the destination rank (int32 expert ids, -1 elsewhere) and their weights
+    (0 elsewhere).  Returns (meta_idx [rows, k] int32, meta_w [rows, k] fp32)."""
+    if topk_idx.shape != (lay.T, lay.k) or topk_weights.shape != (lay.T, lay.k):
+        raise ValueError("topk_idx and topk_weights must be [T, k]")
+    dev = topk_idx.device
+    if meta_idx is None:
+        meta_idx = torch.empty((lay.recv_cap, lay.k), dtype=torch.int32, device=dev)
+    if meta_w is None:
+        meta_w = torch.empty((lay.recv_cap, lay.k), dtype=torch.float32, device=dev)
+    if meta_idx.shape[1:] != (lay.k,) or meta_w.shape != meta_idx.shape:
+        raise ValueError("meta buffers must be [rows, k]")
+    _check(lib().ep_route_meta(_dev(topk_idx, "topk_idx", (torch.int32, torch.int64)),
+                               _dev(topk_weights, "topk_weights", torch.float32), lay.ref,
+                               _dev(meta_idx, "meta_idx", torch.int32),
+                               _dev(meta_w, "meta_w", torch.float32), meta_idx.shape[0],
+                               _stream(stream)), "ep_route_meta")
+    return meta_idx, meta_w
+
+
+def latency_floor(buf: torch.Tensor, n_kernels: int = 3, stream=None) -> None:
+    """ep_latency_floor: n chained one-warp kernels, one dependent load each."""
+    _check(lib().ep_latency_floor(_dev(buf, "buf", torch.int32), buf.numel(), n_kernels,
+                                  _stream(stream)), "ep_latency_floor")
 
 
 def dispatch(x: torch.Tensor, lay: Layout, recv: torch.Tensor = None, stream=None):
@@ -312,35 +390,63 @@ def roundtrip_device_bytes(T, H, k, E, R, idx_bits=64) -> int:
     return int(lib().ep_roundtrip_device_bytes(T, H, k, E, R, idx_bits))
 
 
-def roundtrip_host(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.Tensor,
-                   E: int, R: int, dev_mem: torch.Tensor, out_host: torch.Tensor, stream=None):
-    """ep_roundtrip_host: host buffers in, host buffer out (asynchronous)."""
-    T, H = x_host.shape
-    k = idx_host.shape[1]
-    bits = {torch.int64: 64, torch.int32: 32}[idx_host.dtype]
-    for t in (x_host, idx_host, w_host, out_host):
+def _host_roundtrip_args(x_host, idx_host, w_host, out_host):
+    """Shapes and dtypes of the host buffers of a round trip (the C call
+    trusts them: out_host receives T*H bf16 values)."""
+    for name, t in (("x_host", x_host), ("idx_host", idx_host), ("w_host", w_host),
+                    ("out_host", out_host)):
         if t.is_cuda or not t.is_contiguous():
-            raise ValueError("host buffers must be contiguous CPU tensors")
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if x_host.dim() != 2 or x_host.dtype != torch.bfloat16:
+        raise TypeError("x_host must be bf16 [T, H]")
+    T, H = x_host.shape
+    if idx_host.dim() != 2 or idx_host.shape[0] != T:
+        raise ValueError("idx_host must be [T, k]")
+    bits = {torch.int64: 64, torch.int32: 32}.get(idx_host.dtype)
+    if bits is None:
+        raise TypeError("idx_host must be int32 or int64")
+    k = idx_host.shape[1]
+    if w_host.dtype != torch.float32 or tuple(w_host.shape) != (T, k):
+        raise TypeError("w_host must be float32 [T, k]")
+    if out_host.dtype != torch.bfloat16 or tuple(out_host.shape) != (T, H):
+        raise TypeError("out_host must be bf16 [T, H]")
+    return T, H, k, bits
+
+
+def roundtrip_host(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.Tensor,
+                   E: int, R: int, dev_mem: torch.Tensor, out_host: torch.Tensor, stream=None,
+                   dev_err=None):
+    """ep_roundtrip_host: host buffers in, host buffer out (asynchronous).
+    dev_err: optional ctypes.c_int32 that receives the layout's device error
+    word once the stream has synchronised."""
+    T, H, k, bits = _host_roundtrip_args(x_host, idx_host, w_host, out_host)
+    if not dev_mem.is_cuda:
+        raise ValueError("dev_mem must be a CUDA tensor")
     _check(lib().ep_roundtrip_host(x_host.data_ptr(), idx_host.data_ptr(), w_host.data_ptr(),
-                                   T, H, k, E, R, bits, dev_mem.data_ptr(), dev_mem.numel(),
-                                   out_host.data_ptr(), _stream(stream)), "ep_roundtrip_host")
+                                   T, H, k, E, R, bits, dev_mem.data_ptr(),
+                                   dev_mem.numel() * dev_mem.element_size(),
+                                   out_host.data_ptr(),
+                                   None if dev_err is None else ctypes.byref(dev_err),
+                                   _stream(stream)), "ep_roundtrip_host")
     return out_host
 
 
 def roundtrip_host_noalloc(x_host: torch.Tensor, idx_host: torch.Tensor, w_host: torch.Tensor,
-                           E: int, R: int, out_host: torch.Tensor, stream=None):
+                           E: int, R: int, out_host: torch.Tensor, stream=None, dev_err=None):
     """ep_roundtrip_host_noalloc: like roundtrip_host, for callers that cannot
     allocate device memory -- the device scratch is the library's fixed
     NOALLOC_SCRATCH_BYTES array (asynchronous; calls that overlap on the GPU
     race on that array)."""
-    T, H = x_host.shape
-    k = idx_host.shape[1]
-    bits = {torch.int64: 64, torch.int32: 32}[idx_host.dtype]
-    for t in (x_host, idx_host, w_host, out_host):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError("host buffers must be contiguous CPU tensors")
+    T, H, k, bits = _host_roundtrip_args(x_host, idx_host, w_host, out_host)
     _check(lib().ep_roundtrip_host_noalloc(x_host.data_ptr(), idx_host.data_ptr(),
                                            w_host.data_ptr(), T, H, k, E, R, bits,
-                                           out_host.data_ptr(), _stream(stream)),
+                                           out_host.data_ptr(),
+                                           None if dev_err is None else ctypes.byref(dev_err),
+                                           _stream(stream)),
            "ep_roundtrip_host_noalloc")
     return out_host
+
+
+def debug_dispatch_first_wait_limit(limit: int) -> None:
+    """ep_debug_dispatch_first_wait_limit (test setting; negative = normal)."""
+    lib().ep_debug_dispatch_first_wait_limit(int(limit))

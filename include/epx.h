@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define EPX_ABI_VERSION 1
+#define EPX_ABI_VERSION 2
 
 #define EPX_MAX_TOPK 32      /* k <= 32: one warp holds a token's routes      */
 #define EPX_MAX_RANKS 64     /* R <= 64: a token's rank set fits in 64 bits   */
@@ -83,6 +83,11 @@ typedef enum ep_status {
  *   recv_pos[T*R] row of token t in `recv` for rank r, -1 if not sent
  *   totals[4]     N_route = off_e[E], N_recv = off_r[R],
  *                 T_real = rows with >= 1 valid route, device error word
+ *   work          workspace of the grid layout schedule: a header of
+ *                 barrier words, then one row of counts per CTA.  The
+ *                 header must be zero before the first ep_layout call on
+ *                 the block (allocate it zeroed, or cudaMemset the block
+ *                 once); every call leaves it zero again.
  */
 typedef struct ep_layout {
     int32_t T, k, E, R;
@@ -95,6 +100,7 @@ typedef struct ep_layout {
     int32_t *pos;
     int32_t *recv_pos;
     int32_t *totals;
+    int32_t *work;
 } ep_layout_t;
 
 /* ABI version of the loaded library (EPX_ABI_VERSION at build time). */
@@ -121,19 +127,52 @@ ep_status_t ep_layout_init(ep_layout_t *L, int32_t T, int32_t k, int32_t E,
  * Routing layout from topk_idx (device, [T, k] row-major, int32 or int64 as
  * L->idx_bits says; -1 = no route).  Overwrites every array of *L, including
  * totals[3] (the error word is reset here).  Indices < -1 or >= E are
- * dropped and flagged EP_DEVERR_BAD_INDEX.  One launch (a thread-block
- * cluster whose CTAs share histograms through distributed shared memory).
+ * dropped and flagged EP_DEVERR_BAD_INDEX.  One launch: for up to a few
+ * thousand routes one thread-block cluster whose CTAs share their counts
+ * through distributed shared memory; for large batches a grid of up to one
+ * CTA per SM whose CTAs share their counts through L->work behind one grid
+ * barrier (a bounded wait: if it gives up, EP_DEVERR_TIMEOUT is set and
+ * every pos of the CTA is -1).  Two calls on one layout block must not
+ * overlap on the GPU.
  */
 ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream);
 
 /* Same, choosing the schedule: 0 = automatic, 1 = warp chunks (each warp
- * takes whole tokens, one lane per route, and ranks routes with warp match
- * instructions; EP_ERR_UNSUPPORTED when its per-warp count table does not
+ * takes whole tokens, one lane per route, and finds the lanes that share an
+ * expert or a rank with one warp ballot per bit of the key;
+ * EP_ERR_UNSUPPORTED when its per-warp count table does not
  * fit in shared memory or the CTA's tokens need more than four passes of
- * its warps), 2 = count matrix (one thread per token; any valid size).
- * Results are identical. */
+ * its warps), 2 = count matrix (one thread per token; any valid size),
+ * 3 = grid of up to one CTA per SM (EP_ERR_UNSUPPORTED below two CTAs or
+ * where its tables do not fit in shared memory).  Results are identical. */
 ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
                               int32_t variant, void *stream);
+
+/*
+ * Layout and dispatch + expand in one call: the same results as ep_layout
+ * followed by ep_dispatch_expand with the same arguments (every array of *L,
+ * recv, expanded and the error word).  For small batches (T*k up to
+ * EPX_FUSED_MAX_ROUTES) it can run as ONE launch: every CTA derives its own
+ * token's rows by counting over all routes while its chunk of x is in flight,
+ * so nothing waits for a separate layout kernel -- the fixed cost that
+ * dominates the low-batch regime of DeepEP issue #760's report.
+ * variant: 0 = automatic (one launch for small batches, else two), 1 = one
+ * launch (EP_ERR_UNSUPPORTED beyond EPX_FUSED_MAX_ROUTES), 2 = ep_layout then
+ * ep_dispatch_expand.  Rows beyond a capacity are skipped and flagged
+ * (EP_DEVERR_RECV_CAP / EP_DEVERR_EXP_CAP) as in ep_dispatch_expand.
+ */
+#define EPX_FUSED_MAX_ROUTES 8192
+#define EPX_FUSED_AUTO_ROUTES 2048 /* variant 0 takes one launch up to here */
+ep_status_t ep_layout_dispatch_expand(const void *topk_idx, const ep_layout_t *L,
+                                      const void *x, int32_t H, void *recv,
+                                      int64_t recv_cap, void *expanded,
+                                      int64_t exp_cap, void *stream);
+ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx,
+                                              const ep_layout_t *L, const void *x,
+                                              int32_t H, void *recv,
+                                              int64_t recv_cap, void *expanded,
+                                              int64_t exp_cap, int32_t variant,
+                                              void *stream);
 
 /*
  * Dispatch + expand.  x: device bf16 [T, H] row-major (16-byte aligned,
@@ -143,7 +182,9 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
  * recv: device bf16 [recv_cap, H]; expanded: device bf16 [exp_cap, H].
  * Worst-case capacities T*min(k, R) and T*k never overflow; a smaller
  * capacity is allowed, and rows beyond it are skipped and flagged.
- * Rows past N_recv / N_route are left untouched.
+ * Rows past N_recv / N_route are left untouched.  recv may be NULL with
+ * recv_cap 0: only the expanded rows are written (the receiving side of a
+ * multi-GPU dispatch, whose rows arrived already).
  */
 ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L,
                                void *recv, int64_t recv_cap, void *expanded,
@@ -167,6 +208,27 @@ ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H,
  */
 ep_status_t ep_dispatch(const void *x, int32_t H, const ep_layout_t *L, void *recv,
                         int64_t recv_cap, void *stream);
+
+/*
+ * Routing that travels with each sent row of a multi-GPU dispatch (one rank
+ * per GPU, rank r owning experts [r*E/R, (r+1)*E/R)): a token goes once to
+ * every rank that owns one of its experts together with its top-k routing
+ * (DeepEP issue #48, question), and that rank expands it per local expert
+ * and reduces the outputs before the combine travels back (issue #48,
+ * answer on the reduction before the combine all2all).  For every
+ * (token t, rank r) pair of the layout, row q = recv_pos[t, r] gets
+ *   meta_idx[q, j] = topk_idx[t, j] if expert topk_idx[t, j] is on rank r,
+ *                    else -1,
+ *   meta_w[q, j]   = topk_weights[t, j] if so, else 0,
+ * so the rows sent to rank r, with these as their routing, form a batch
+ * whose routes all stay on rank r.  topk_idx: device [T, k] (L->idx_bits
+ * wide); topk_weights: device fp32 [T, k]; meta_idx: device int32
+ * [rows, k]; meta_w: device fp32 [rows, k]; rows >= N_recv (worst case
+ * T*min(k, R)); a row >= rows is skipped and flagged EP_DEVERR_RECV_CAP.
+ */
+ep_status_t ep_route_meta(const void *topk_idx, const float *topk_weights,
+                          const ep_layout_t *L, int32_t *meta_idx, float *meta_w,
+                          int64_t rows, void *stream);
 
 /*
  * Gather index for a consumer that reads the received rows directly:
@@ -270,8 +332,12 @@ ep_status_t ep_layout_read_totals(const ep_layout_t *L, int64_t *n_route,
  * (pinned for asynchronous copies), runs layout, dispatch/expand, the
  * stand-in expert and combine on the device, and copies out (bf16 [T, H])
  * back to host memory.  dev_mem: caller-owned device scratch of at least
- * ep_roundtrip_device_bytes(...) bytes, 256-byte aligned.  Asynchronous:
- * the caller synchronises `stream` before reading out_host.
+ * ep_roundtrip_device_bytes(...) bytes, 256-byte aligned.  dev_err_host
+ * (host, may be NULL) receives the layout's device error word (EP_DEVERR_*
+ * bits; nonzero when a route or a row was dropped, e.g. an index >= E) --
+ * the status returned here only covers what the host can check before the
+ * work runs.  Asynchronous: the caller synchronises `stream` before reading
+ * out_host or *dev_err_host.
  */
 size_t ep_roundtrip_device_bytes(int32_t T, int32_t H, int32_t k, int32_t E,
                                  int32_t R, int32_t idx_bits);
@@ -279,7 +345,8 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
                               const float *topk_weights_host, int32_t T,
                               int32_t H, int32_t k, int32_t E, int32_t R,
                               int32_t idx_bits, void *dev_mem, size_t bytes,
-                              void *out_host, void *stream);
+                              void *out_host, int32_t *dev_err_host,
+                              void *stream);
 
 /*
  * Host round trip that allocates nothing.  The pages have no counterpart:
@@ -289,7 +356,8 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
  * loaded into a host that forbids allocation after initialisation, latency
  * paths that cannot afford an allocation's implicit synchronisation.
  *
- * Same arguments and result as ep_roundtrip_host, minus dev_mem/bytes: the
+ * Same arguments and result as ep_roundtrip_host (including the optional
+ * dev_err_host error word), minus dev_mem/bytes: the
  * device scratch is a fixed array of EPX_NOALLOC_SCRATCH_BYTES inside this
  * library, which every GPU that loads the library holds until the process
  * exits.  Sizes whose ep_roundtrip_device_bytes(...) exceeds it return
@@ -298,8 +366,10 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
  * top-16).  No cudaMalloc, cudaFree or other allocating call is made.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the array and it keeps the
+ * (cudaGetSymbolAddress) with that device current and keeps it for the
+ * life of the process; make that first call before any stream capture.
+ * cudaDeviceReset destroys the context that address belongs to, so this
+ * entry point must not be used in a process after a device reset.  All calls share the array and it keeps the
  * last call's contents (nothing in it needs to start at zero); calls whose
  * device work overlaps -- on different streams or from different host
  * threads -- race on it, so order them on one stream or synchronise.
@@ -308,7 +378,33 @@ ep_status_t ep_roundtrip_host(const void *x_host, const void *topk_idx_host,
 ep_status_t ep_roundtrip_host_noalloc(const void *x_host, const void *topk_idx_host,
                                       const float *topk_weights_host, int32_t T,
                                       int32_t H, int32_t k, int32_t E, int32_t R,
-                                      int32_t idx_bits, void *out_host, void *stream);
+                                      int32_t idx_bits, void *out_host,
+                                      int32_t *dev_err_host, void *stream);
+
+/*
+ * Measurement helper: the latency floor of a step of this path.  Launches
+ * n_kernels (1..64) one-warp kernels on `stream`, chained like the path's
+ * kernels (programmatic dependent launch), each loading one word of `buf`
+ * after its predecessor has finished and storing one word -- the skeleton
+ * of the low-batch step (launches, hand-offs, one DRAM round trip per
+ * kernel) with no work in it.  buf: device int32, at least
+ * 64 * (2 * n_kernels + 2) words, 16-byte aligned; its contents are
+ * irrelevant and get overwritten.
+ */
+ep_status_t ep_latency_floor(int32_t *buf, int64_t buf_words, int32_t n_kernels,
+                             void *stream);
+
+/*
+ * Test setting (not needed by any caller of the path): the number of polls
+ * the first bounded wait of every CTA of the bulk copy engine
+ * (ep_dispatch_expand_variant(..., 2, ...)) may take before it gives up,
+ * for later launches from this process; negative restores the normal limit.
+ * With 0 every CTA gives up at once: it flags EP_DEVERR_TIMEOUT, waits
+ * (bounded) for its copy in flight, and leaves its rows unwritten, so
+ * ep_layout_read_totals returns EP_ERR_CUDA -- the path that a copy which
+ * never completes would take, exercised without a stuck copy.
+ */
+void ep_debug_dispatch_first_wait_limit(int64_t limit);
 
 #ifdef __cplusplus
 }

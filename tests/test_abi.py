@@ -38,7 +38,7 @@ def test_header_declares_the_path():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.ep_abi_version() == 1
+    assert lib.ep_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -96,7 +96,7 @@ def test_calls_reject_bad_arguments_before_launching(lib):
     # misaligned 64-bit indices
     assert lib.ep_layout(fake + 4, ctypes.byref(c), None) == 2
     # unknown layout schedule or combine schedule
-    assert lib.ep_layout_variant(fake, ctypes.byref(c), 3, None) == 1
+    assert lib.ep_layout_variant(fake, ctypes.byref(c), 4, None) == 1
     assert lib.ep_layout_variant(fake, ctypes.byref(c), -1, None) == 1
     assert lib.ep_layout_variant(fake + 4, ctypes.byref(c), 1, None) == 2
     assert lib.ep_combine_reduce_variant(fake, fake, 16, ctypes.byref(c), fake, 8, 3, None) == 1
@@ -108,4 +108,56 @@ def test_roundtrip_sizes(lib):
     assert n >= 128 * row * (1 + 8 + 8 + 1) + 128 * 8 * row
     assert lib.ep_roundtrip_device_bytes(128, 7167, 8, 256, 16, 64) == 0
     assert lib.ep_roundtrip_host(None, None, None, 128, 7168, 8, 256, 16, 64, None, 0, None,
-                                 None) == 1
+                                 None, None) == 1
+
+
+def test_host_roundtrip_binding_checks_buffers():
+    """The binding rejects host buffers of the wrong dtype or shape before
+    calling the library (which trusts them: it copies T*H values back)."""
+    import torch
+    T, H, k = 4, 16, 2
+    x = torch.zeros((T, H), dtype=torch.bfloat16)
+    i = torch.zeros((T, k), dtype=torch.int64)
+    w = torch.zeros((T, k), dtype=torch.float32)
+    out = torch.zeros((T, H), dtype=torch.bfloat16)
+    bad = [
+        (x.float(), i, w, out),                      # x not bf16
+        (x, i.float(), w, out),                      # indices not integer
+        (x, i, w.double(), out),                     # weights not fp32
+        (x, i, w[:, :1].contiguous(), out),          # weights not [T, k]
+        (x, i, w, out[:2].contiguous()),             # out too small
+        (x, i, w, out.float()),                      # out not bf16
+        (x, i[:3].contiguous(), w, out),             # indices not [T, k]
+    ]
+    for args in bad:
+        with pytest.raises((TypeError, ValueError)):
+            epx._host_roundtrip_args(*args)
+    assert epx._host_roundtrip_args(x, i, w, out) == (T, H, k, 64)
+
+
+def test_binding_constants_mirror_the_header():
+    src = open(HEADER).read()
+    val = lambda name: int(re.search(r"#define %s \(?(\d+)" % name, src).group(1))  # noqa: E731
+    assert epx.MAX_TOPK == val("EPX_MAX_TOPK")
+    assert epx.MAX_RANKS == val("EPX_MAX_RANKS")
+    assert epx.MAX_EXPERTS == val("EPX_MAX_EXPERTS")
+    assert epx.FUSED_MAX_ROUTES == val("EPX_FUSED_MAX_ROUTES")
+    assert epx.FUSED_AUTO_ROUTES == val("EPX_FUSED_AUTO_ROUTES")
+    assert epx.NOALLOC_SCRATCH_BYTES == val("EPX_NOALLOC_SCRATCH_BYTES") << 20
+
+
+def test_one_launch_call_validates_on_host(lib):
+    c = epx._LayoutC()
+    fake = 0x10000
+    n = lib.ep_layout_bytes(4, 2, 4, 2)
+    assert lib.ep_layout_init(ctypes.byref(c), 4, 2, 4, 2, 64, fake, n) == 0
+    f = lib.ep_layout_dispatch_expand_variant
+    assert f(fake, ctypes.byref(c), fake, 16, fake, 8, fake, 8, 3, None) == 1    # variant
+    assert f(fake, ctypes.byref(c), fake, 12, fake, 8, fake, 8, 0, None) == 1    # H % 8
+    assert f(fake, ctypes.byref(c), fake + 2, 16, fake, 8, fake, 8, 0, None) == 2
+    assert f(fake + 4, ctypes.byref(c), fake, 16, fake, 8, fake, 8, 0, None) == 2
+    assert f(None, ctypes.byref(c), fake, 16, fake, 8, fake, 8, 0, None) == 1
+    assert f(fake, None, fake, 16, fake, 8, fake, 8, 0, None) == 1
+    assert lib.ep_latency_floor(None, 0, 3, None) == 1
+    assert lib.ep_latency_floor(fake, 64, 3, None) == 1                            # too small
+    assert lib.ep_latency_floor(fake + 4, 64 * 8, 3, None) == 2

@@ -29,6 +29,29 @@ def test_alg_bytes_variants():
     assert "expand_index" in ne and ne["dispatch"] == 128 * 14336 + 833 * 14336 + 128 * 16 * 4
 
 
+def test_alg_bytes_one_launch_step():
+    """Layout and dispatch/expand as one kernel: the layout's bytes plus the
+    copies, without the dispatch's re-read of pos / recv_pos."""
+    sep = bench.alg_bytes(128, 128, 833, 1024, 7168, 8, 16, 8)
+    one = bench.alg_bytes(128, 128, 833, 1024, 7168, 8, 16, 8, fused=True)
+    assert set(one) == {"layout_dispatch_expand", "combine_reduce", "total"}
+    assert one["layout_dispatch_expand"] == (sep["layout"] + sep["dispatch_expand"]
+                                             - 128 * 8 * 4 - 128 * 16 * 4)
+    assert one["combine_reduce"] == sep["combine_reduce"]
+
+
+def test_step_call_choice_follows_the_library_threshold():
+    from combine_ep_layout_07_b200 import epx
+    a = bench.parse_args([])
+    assert bench.fused_step(a, 128, 8) and bench.fused_step(a, 1, 16)
+    assert not bench.fused_step(a, 4096, 8)
+    assert bench.fused_step(a, epx.FUSED_AUTO_ROUTES // 8, 8)
+    assert not bench.fused_step(a, epx.FUSED_AUTO_ROUTES // 8 + 1, 8)
+    assert not bench.fused_step(bench.parse_args(["--step-calls", "separate"]), 128, 8)
+    assert bench.fused_step(bench.parse_args(["--step-calls", "fused"]), 960, 8)
+    assert not bench.fused_step(bench.parse_args(["--no-expand"]), 128, 8)
+
+
 def test_traffic_lookup_follows_source_and_engine(tmp_path, monkeypatch):
     h = bench.sources_hash("dispatch_expand")
     f = tmp_path / "traffic.txt"
@@ -76,3 +99,10 @@ def test_host_cpu_reports_model_and_cores():
     h = bench.host_cpu()
     assert isinstance(h["model"], str)
     assert h["nproc"] == os.cpu_count()
+
+
+def test_pinned_to_one_core_restores_affinity():
+    before = os.sched_getaffinity(0)
+    with bench.PinnedToOneCore() as pin:
+        assert os.sched_getaffinity(0) == {pin.core}
+    assert os.sched_getaffinity(0) == before

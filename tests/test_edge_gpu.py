@@ -86,6 +86,56 @@ def test_layout_schedules_shapes(case, lv):
     assert_layout_equal(lay, lay_o)
 
 
+GRID_CASES = [c for c in LAYOUT_CASES if c["T"] * c["k"] > 256] + [
+    dict(T=4096, H=8, E=256, R=16, k=8),       # the prefill shape: 128 CTAs
+    dict(T=16384, H=8, E=256, R=16, k=8),      # one CTA per SM, several passes
+    dict(T=2000, H=8, E=1024, R=64, k=5),      # wide tables, k not dividing 32
+]
+
+
+@pytest.mark.parametrize("case", GRID_CASES, ids=lambda c: "T{T}k{k}E{E}R{R}".format(**c))
+def test_layout_grid_schedule_shapes(case):
+    """The grid schedule (variant 3): bit-exact, twice in a row on the same
+    block (its barrier words are left zero by every call)."""
+    wl = _random_wl(seed=case["T"] * 5 + case["k"], p_pad=0.2, distinct=False, **case)
+    idx = wl["topk_idx"]
+    idx[2, 0] = case["E"] + 5
+    idx[3, :] = -1
+    idx[1, 1] = idx[1, 0]
+    lay_o = oracle.layout(idx, case["E"], case["R"])
+    it = torch.from_numpy(idx).cuda()
+    lay = epx.Layout(case["T"], case["k"], case["E"], case["R"], 64)
+    for _ in range(2):
+        epx.layout(it, case["E"], case["R"], out=lay, variant=3)
+        torch.cuda.synchronize()
+        assert_layout_equal(lay, lay_o)
+        off = lay.c.work - lay.mem.data_ptr()
+        assert torch.count_nonzero(lay.mem[off:off + 64]) == 0   # header back to zero
+
+
+def test_layout_grid_schedule_refuses_single_cta():
+    idx = torch.zeros((16, 8), dtype=torch.int64, device="cuda")
+    with pytest.raises(epx.EpxError) as ei:
+        epx.layout(idx, 16, 4, variant=3)
+    assert ei.value.status == 6
+
+
+def test_layout_grid_schedule_deterministic_and_interleaved():
+    wl = _random_wl(T=4096, H=8, E=256, R=16, k=8, seed=21)
+    it = torch.from_numpy(wl["topk_idx"]).cuda()
+    lay_o = oracle.layout(wl["topk_idx"], 256, 16)
+    lay = epx.Layout(4096, 8, 256, 16, 64)
+    ref = None
+    for i in range(20):
+        epx.layout(it, 256, 16, out=lay, variant=(3, 1, 2, 0)[i % 4])
+        snap = [a.clone() for a in (lay.cnt_e, lay.off_e, lay.cnt_r, lay.off_r, lay.pos,
+                                    lay.recv_pos, lay.totals)]
+        if ref is None:
+            ref = snap
+        assert all(torch.equal(a, b) for a, b in zip(snap, ref))
+    assert_layout_equal(lay, lay_o)
+
+
 def test_layout_warp_schedule_unsupported_shape():
     # the per-warp count table of E = 4096, R = 64 for 129 tokens of top-5
     # does not fit in shared memory: variant 1 refuses, auto and 2 agree

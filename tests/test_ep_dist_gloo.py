@@ -1,0 +1,172 @@
+"""Host logic of the multi-GPU expert-parallel path (ep_dist), on CPU with
+world-size-2 gloo groups.  The kernels' part of each step is played by the
+CPU oracle; what is under test is the plan and the exchanges: the counts
+all-gather, the all-to-all send plan, the order of received rows and the
+return trip of the partials.
+
+The check is the one the pages' setting fixes: with the ranks' batches
+concatenated in rank order, rank r must receive exactly the rows a single
+GPU puts in rank r's block of `recv` (DeepEP issue #48: a token goes once to
+every rank that owns one of its experts), with routing restricted to rank
+r's experts, and the combine that comes back must equal the single-GPU
+two-stage combine of the same tokens."""
+import os
+import socket
+import sys
+import traceback
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+E, K, H = 16, 4, 64
+T_OF = [37, 50]          # ranks hold different batch sizes
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _batch(g):
+    """Rank g's tokens (the same on every process): x bf16 bits, idx, w."""
+    from combine_ep_layout_07_b200 import workloads as wlmod
+    rng = np.random.default_rng(100 + g)
+    T = T_OF[g]
+    x = wlmod.to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    idx = np.argsort(rng.random((T, E)), axis=1)[:, :K].astype(np.int64)
+    idx[rng.random((T, K)) < 0.15] = -1
+    if T > 3:
+        idx[3, :] = -1          # a token that goes nowhere
+    w = rng.random((T, K), dtype=np.float32)
+    return x, idx, w
+
+
+def _meta(idx, w, lay, R):
+    """Expected routing of every sent row (recv_pos order): the token's
+    routes on the destination rank, -1 / 0 elsewhere."""
+    epr = E // R
+    n = lay["N_recv"]
+    mi = np.full((n, K), -1, np.int32)
+    mw = np.zeros((n, K), np.float32)
+    for t in range(lay["T"]):
+        for r in range(R):
+            row = lay["recv_pos"][t, r]
+            if row < 0:
+                continue
+            for j in range(K):
+                e = idx[t, j]
+                if e >= 0 and e // epr == r:
+                    mi[row, j] = e
+                    mw[row, j] = w[t, j]
+    return mi, mw
+
+
+def _worker(rank, world, port, out_q):
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        sys.path.insert(0, ROOT)
+        import oracle
+        from combine_ep_layout_07_b200 import ep_dist
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        pg = dist.group.WORLD
+        R = world
+        x, idx, w = _batch(rank)
+        # ---- source side (oracle standing in for the kernels)
+        lay = oracle.layout(idx, E, R)
+        send, _ = oracle.dispatch_expand(x, lay)
+        mi, mw = _meta(idx, w, lay, R)
+        counts = ep_dist.exchange_counts(torch.from_numpy(lay["cnt_r"]), pg)
+        plan = ep_dist.send_plan(counts, rank)
+        assert plan["n_send"] == lay["N_recv"]
+        recv_x = ep_dist.exchange_rows(torch.from_numpy(send.view(np.int16)), plan, pg)
+        recv_i = ep_dist.exchange_rows(torch.from_numpy(mi), plan, pg)
+        recv_w = ep_dist.exchange_rows(torch.from_numpy(mw), plan, pg)
+
+        # ---- the single-GPU view of all ranks' tokens
+        parts = [_batch(g) for g in range(world)]
+        gx = np.concatenate([p[0] for p in parts])
+        gidx = np.concatenate([p[1] for p in parts])
+        gw = np.concatenate([p[2] for p in parts])
+        glay = oracle.layout(gidx, E, R)
+        grecv, _ = oracle.dispatch_expand(gx, glay)
+        gmi, gmw = _meta(gidx, gw, glay, R)
+        lo, hi = glay["off_r"][rank], glay["off_r"][rank + 1]
+        assert list(counts[:, rank]) == [int(v) for v in plan["recv_splits"]]
+        assert plan["n_recv"] == hi - lo
+        np.testing.assert_array_equal(recv_x.numpy().view(np.uint16), grecv[lo:hi])
+        np.testing.assert_array_equal(recv_i.numpy(), gmi[lo:hi])
+        np.testing.assert_array_equal(recv_w.numpy(), gmw[lo:hi])
+
+        # ---- receiving side: every received route is on this rank
+        lay_in = oracle.layout(recv_i.numpy(), E, R)
+        assert lay_in["cnt_r"][rank] == plan["n_recv"] and lay_in["N_recv"] == plan["n_recv"]
+        np.testing.assert_array_equal(lay_in["recv_pos"][:, rank], np.arange(plan["n_recv"]))
+        _, ex_in = oracle.dispatch_expand(recv_x.numpy().view(np.uint16), lay_in)
+        y_in = oracle.standin(ex_in, lay_in)
+        part = oracle.combine_local(y_in, recv_w.numpy(), lay_in, 32)
+        back = ep_dist.exchange_rows(torch.from_numpy(np.ascontiguousarray(part)), plan, pg,
+                                     reverse=True).numpy()
+        out = oracle.combine_epilogue(back, lay)
+
+        # ---- against the single-GPU two-stage combine of all tokens
+        _, gex = oracle.dispatch_expand(gx, glay)
+        gy = oracle.standin(gex, glay)
+        gpart = oracle.combine_local(gy, gw, glay, 32)
+        gout = oracle.combine_epilogue(gpart, glay)
+        t0 = sum(T_OF[:rank])
+        for t in range(lay["T"]):
+            for r in range(R):
+                row = lay["recv_pos"][t, r]
+                if row >= 0:
+                    np.testing.assert_array_equal(back[row],
+                                                  gpart[glay["recv_pos"][t0 + t, r]])
+        np.testing.assert_array_equal(out, gout[t0:t0 + lay["T"]])
+        out_q.put((rank, "ok"))
+    except Exception:
+        out_q.put((rank, traceback.format_exc()))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def test_send_plan_is_the_counts_matrix():
+    from combine_ep_layout_07_b200 import ep_dist
+    c = torch.tensor([[3, 0, 2], [1, 4, 0], [0, 5, 6]])
+    p = ep_dist.send_plan(c, 1)
+    assert p["send_splits"] == [1, 4, 0] and p["recv_splits"] == [0, 4, 5]
+    assert p["recv_offsets"] == [0, 0, 4] and p["n_send"] == 5 and p["n_recv"] == 9
+    with pytest.raises(ValueError):
+        ep_dist.send_plan(torch.tensor([[1, -1], [0, 0]]), 0)
+    with pytest.raises(ValueError):
+        ep_dist.send_plan(c, 3)
+
+
+def test_exchange_on_one_rank_is_the_identity():
+    from combine_ep_layout_07_b200 import ep_dist
+    plan = ep_dist.send_plan(torch.tensor([[5]]), 0)
+    rows = torch.arange(20, dtype=torch.int32).view(5, 4)
+    assert torch.equal(ep_dist.exchange_rows(rows, plan), rows)
+    assert torch.equal(ep_dist.exchange_rows(rows, plan, reverse=True), rows)
+    assert ep_dist.exchange_counts(torch.tensor([5])).tolist() == [[5]]
+
+
+def test_two_ranks_match_the_single_gpu_layout_split_by_rank():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+    for r in range(world):
+        assert res[r] == "ok", res[r]

@@ -59,6 +59,13 @@ def test_layout_schedules_int32(name, variant):
     assert_all_equal(run_gpu(wl, idx_dtype=torch.int32, layout_variant=variant), o)
 
 
+@pytest.mark.parametrize("idx_dtype", [torch.int64, torch.int32], ids=["i64", "i32"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "dp_compact", "dp_padded"])
+def test_layout_grid_schedule(name, idx_dtype):
+    wl, o = oracle_run(name, 0)
+    assert_all_equal(run_gpu(wl, idx_dtype=idx_dtype, layout_variant=3), o)
+
+
 @pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "lowbatch1", "dp_padded"])
 def test_dispatch_engines(name, variant):
