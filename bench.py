@@ -105,8 +105,9 @@ def parse_args(argv=None):
                          "against the one reading the expanded copy")
     ap.add_argument("--step-calls", choices=["auto", "separate", "fused"], default="auto",
                     help="layout and dispatch/expand as one call (one launch, small batches), "
-                         "as two calls, or automatic (one launch up to "
-                         "EPX_FUSED_AUTO_ROUTES routes, as the library's automatic choice)")
+                         "as two calls, or automatic (one launch for EPX_FUSED_AUTO_MIN_ROUTES "
+                         "to EPX_FUSED_AUTO_MAX_ROUTES routes, as the library's automatic "
+                         "choice)")
     ap.add_argument("--small-steps", type=int, default=1500,
                     help="steps of each small-batch workload measured beside the headline "
                          "(0 skips them)")
@@ -420,7 +421,7 @@ def fused_step(args, T, k):
     if args.step_calls == "fused":
         return True
     from combine_ep_layout_07_b200 import epx
-    return T * k <= epx.FUSED_AUTO_ROUTES
+    return epx.FUSED_AUTO_MIN_ROUTES <= T * k <= epx.FUSED_AUTO_MAX_ROUTES
 
 
 def workload_config(wl, args, lay_totals, flush_desc=None, fused=False):
@@ -611,12 +612,61 @@ def time_step(torch, launch, n_calls, stream, dev, steps, warmup, flush=None, ea
     return step_ms, (rec_k if (split or eager) else None), (t_lo, t_hi)
 
 
+def time_amortized(torch, launch, stream, dev, flush, reps=50, rounds=40, warmup=2):
+    """Per-step time of `launch` with L2 flushed by a read before every step,
+    amortised over `reps` steps between two events: one CUDA graph of reps x
+    [flush, step] against one of reps x [flush], replayed alternately;
+    per round, step = (A - B) / reps.  The events' timestamp granularity
+    (a few µs after a long kernel such as the flush) divides by reps, and
+    each step is charged the write-back of the lines it left dirty (which
+    the next flush has to write back).  Returns step_stats of the rounds,
+    plus their mean."""
+    with torch.cuda.stream(stream):
+        launch(stream)          # launchers set their function attributes here
+        flush()
+    torch.cuda.synchronize(dev)
+    graphs, evs = [], []
+    for with_step in (True, False):
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            cs = torch.cuda.current_stream()
+            ev[0].record(cs)
+            for _ in range(reps):
+                flush()
+                if with_step:
+                    launch(cs)
+            ev[1].record(cs)
+        graphs.append(g)
+        evs.append(ev)
+    torch.cuda.synchronize(dev)
+    per = []
+    with torch.cuda.stream(stream):
+        for r in range(warmup + rounds):
+            t = []
+            for g, ev in zip(graphs, evs):
+                g.replay()
+                torch.cuda.current_stream().synchronize()
+                t.append(ev[0].elapsed_time(ev[1]))
+            if r >= warmup:
+                per.append((t[0] - t[1]) / reps)
+    del graphs
+    st = step_stats(per)
+    st["mean"] = statistics.fmean(per) * 1e3
+    st["method"] = (f"graph of {reps} x [L2 read-flush, step] minus graph of {reps} x "
+                    f"[L2 read-flush], {rounds} rounds")
+    return st
+
+
 def time_floor(torch, epx, stream, dev, n_kernels, steps, warmup, flush):
-    """ep_latency_floor chain of n_kernels, timed exactly like a step."""
+    """ep_latency_floor chain of n_kernels, timed exactly like a step (per
+    step, and amortised)."""
     buf = torch.zeros(64 * (2 * n_kernels + 2), dtype=torch.int32, device=dev)
-    ms, _, _ = time_step(torch, lambda st, ev=None: epx.latency_floor(buf, n_kernels, stream=st),
-                         1, stream, dev, steps, warmup, flush=flush, split=False)
-    return step_stats(ms)
+    fn = lambda st, ev=None: epx.latency_floor(buf, n_kernels, stream=st)  # noqa: E731
+    ms, _, _ = time_step(torch, fn, 1, stream, dev, steps, warmup, flush=flush, split=False)
+    out = step_stats(ms)
+    out["amortized"] = time_amortized(torch, fn, stream, dev, flush)
+    return out
 
 
 SMALL_WORKLOADS = ("decode", "dp_compact", "dp_padded", "lowbatch1")
@@ -636,6 +686,7 @@ def measure_small(torch, epx, wlmod, args, dev, stream, peak, flush, floors):
         ms, rec_k, _ = time_step(torch, st.launch, len(st.calls), stream, dev, args.small_steps,
                                  max(3, args.warmup), flush=flush)
         stats = step_stats(ms)
+        am = time_amortized(torch, st.launch, stream, dev, flush)
         b = alg_bytes(wl["T"], tot["T_real"], tot["N_recv"], tot["N_route"], wl["H"], wl["k"],
                       wl["R"], args.idx_bits // 8, fused=fused)
         kern = {n: statistics.median([r[i] - (r[i - 1] if i else 0.0) for r in rec_k]) * 1e3
@@ -643,12 +694,13 @@ def measure_small(torch, epx, wlmod, args, dev, stream, peak, flush, floors):
         floor = floors.get(len(st.calls))
         res[name] = {
             "workload": DESCRIBE[name], "T_real": int(tot["T_real"]),
-            "step_us": stats, "tokens_per_s": tot["T_real"] / (stats["median"] / 1e6),
+            "step_us_amortized": am, "step_us": stats,
+            "tokens_per_s": tot["T_real"] / (am["median"] / 1e6),
             "alg_bytes": b["total"],
-            "hbm_frac": b["total"] / (stats["median"] / 1e6) / 1e9 / peak,
+            "hbm_frac": b["total"] / (am["median"] / 1e6) / 1e9 / peak,
             "launches": len(st.calls), "calls": st.names,
             "kernel_us_median_split": kern,
-            "x_floor": (stats["median"] / floor["median"]) if floor else None,
+            "x_floor": (am["median"] / floor["amortized"]["median"]) if floor else None,
         }
     return res
 
@@ -709,6 +761,9 @@ def run_epx(args):
         flush=l2flush if do_flush else None, eager=args.eager, split=True, pg=pg)
     if sampler:
         sampler.stop()
+    amortized = None
+    if do_flush and not args.eager:
+        amortized = time_amortized(torch, step.launch, stream, dev, l2flush)
     names = step.names
     k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)
@@ -764,6 +819,7 @@ def run_epx(args):
         "roofline": roofline,
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
         "step_us": step_stats(step_ms),
+        **({"step_us_amortized": amortized} if amortized else {}),
         "kernels": kernels,
         "gpu_launches": len(step.calls) * args.steps,
         **({"consumer": consumer} if consumer else {}),

@@ -183,15 +183,22 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     if (L->T > 0 && (!aligned(x, 16) || !aligned(recv, 16) || !aligned(expanded, 16)))
         return EP_ERR_MISALIGNED;
     const long long routes = (long long)L->T * L->k;
-    // automatic: one launch while each CTA's count over all routes stays
-    // cheap (measured on B200), else the layout and dispatch kernels
-    if (variant == 0) variant = routes <= kFusedAutoRoutes ? 1 : 2;
+    // automatic: one launch where it was measured faster on B200 (each CTA's
+    // count over all routes stays cheap, and there are tokens enough for the
+    // count to spread over the CTA's warps), else the layout and dispatch
+    // kernels
+    const bool automatic = variant == 0;
+    if (automatic)
+        variant = routes >= kFusedAutoMinRoutes && routes <= kFusedAutoMaxRoutes ? 1 : 2;
+    if (variant == 1 && routes > kFusedMaxRoutes) {
+        if (!automatic) return EP_ERR_UNSUPPORTED;
+        variant = 2;
+    }
     if (variant == 2) {
         ep_status_t st = ep_layout(topk_idx, L, stream);
         if (st != EP_OK || L->T == 0) return st;
         return ep_dispatch_expand(x, H, L, recv, recv_cap, expanded, exp_cap, stream);
     }
-    if (routes > kFusedMaxRoutes) return EP_ERR_UNSUPPORTED;
     FusedParams p;
     memset(&p, 0, sizeof p);
     p.idx = topk_idx;
@@ -214,7 +221,13 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     p.recv_pos = L->recv_pos;
     p.totals = L->totals;
     const cudaError_t e = launch_layout_dispatch(p, L->idx_bits, as_stream(stream));
-    return e == cudaErrorNotSupported ? EP_ERR_UNSUPPORTED : from_cuda(e);
+    if (e == cudaErrorNotSupported) {  // checked before launching anything
+        if (!automatic) return EP_ERR_UNSUPPORTED;
+        const ep_status_t st = ep_layout(topk_idx, L, stream);
+        if (st != EP_OK) return st;
+        return ep_dispatch_expand(x, H, L, recv, recv_cap, expanded, exp_cap, stream);
+    }
+    return from_cuda(e);
 }
 
 ep_status_t ep_layout_dispatch_expand(const void *topk_idx, const ep_layout_t *L, const void *x,

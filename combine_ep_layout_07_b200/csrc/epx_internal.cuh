@@ -34,15 +34,15 @@ struct LayoutParams {
 };
 
 // Grid schedule of the layout: one CTA per this many routes, at most
-// kGridMaxCtas CTAs (and never more than the SMs); its workspace holds a
-// header and one row of packed 16-bit (expert | rank) counts per CTA.
+// kGridMaxCtas CTAs (and never more than the SMs).  Its workspace holds a
+// header of barrier words, one row of packed 16-bit (expert | rank) counts
+// per CTA, one row of 32-bit exclusive prefixes per CTA, and the totals.
 constexpr int kGridRoutesPerCta = 256;
 constexpr int kGridMaxCtas = 256;
 constexpr int kGridHeaderWords = 16;
-// the automatic layout choice takes the grid schedule above this many routes
-constexpr int kGridAutoRoutes = 8192;
 
 inline int grid_row_words(int E, int R) { return (((E + R + 1) / 2) + 3) & ~3; }
+inline int grid_prefix_words(int E, int R) { return (E + R + 3) & ~3; }
 
 inline int grid_max_ctas(long long routes)
 {
@@ -52,9 +52,11 @@ inline int grid_max_ctas(long long routes)
 
 inline size_t grid_work_bytes(int T, int k, int E, int R)
 {
-    return sizeof(int32_t) *
-           ((size_t)kGridHeaderWords + (size_t)grid_max_ctas((long long)T * k) * grid_row_words(E, R));
+    const size_t nb = (size_t)grid_max_ctas((long long)T * k);
+    return sizeof(int32_t) * ((size_t)kGridHeaderWords + nb * grid_row_words(E, R) +
+                              (nb + 1) * grid_prefix_words(E, R));
 }
+
 
 struct DispatchParams {
     const uint4 *x;
@@ -91,8 +93,9 @@ struct FusedParams {
 
 // the one-launch layout + dispatch handles at most this many routes (T*k)
 constexpr int kFusedMaxRoutes = EPX_FUSED_MAX_ROUTES;
-// ... and is the automatic choice up to this many
-constexpr int kFusedAutoRoutes = EPX_FUSED_AUTO_ROUTES;
+// ... and is the automatic choice in this range of routes
+constexpr int kFusedAutoMinRoutes = EPX_FUSED_AUTO_MIN_ROUTES;
+constexpr int kFusedAutoMaxRoutes = EPX_FUSED_AUTO_MAX_ROUTES;
 
 // routing that travels with each row of a multi-GPU dispatch
 struct MetaParams {

@@ -27,9 +27,12 @@
 //  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
 //    counts and exclusive scans, the totals and the error word.
 //
-// No CTA waits for another, so there is no grid-wide barrier.  The work per
-// CTA grows with T*k, so the launcher takes this kernel only for small
-// batches (routes per CTA bounded) and otherwise runs the two kernels.
+// No CTA waits for another, so there is no grid-wide barrier.  The count
+// costs every CTA work in proportion to T*k, and at one or a few tokens the
+// single warp that holds them walks its queries alone; measured on B200 the
+// one launch is faster than the layout and dispatch kernels for batches of
+// a few hundred to about two thousand routes (EPX_FUSED_AUTO_MIN_ROUTES to
+// EPX_FUSED_AUTO_MAX_ROUTES), which is where the automatic choice takes it.
 // Rows beyond a caller's capacity are skipped; the summary CTA flags them
 // (a row beyond the capacity exists exactly when the total exceeds it).
 #include "epx_internal.cuh"
@@ -61,10 +64,25 @@ __device__ __forceinline__ int load_expert(const IdxT *idx, size_t i, int E, boo
 }
 
 // ----------------------------------------------------------- summary CTA
-// cnt_e / off_e / cnt_r / off_r / totals for the whole batch.  Expert counts
+// cnt_e / off_e / cnt_r / off_r / totals for the whole batch.  A warp takes
+// floor(32 / k) whole tokens per step, one lane per route (one coalesced
+// load per lane, the steps independent of each other); the first route of
+// every (token, rank) pair -- no lower lane of its token has its rank, found
+// with one ballot per bit of the rank -- counts for the rank.  Expert counts
 // are 16-bit halves of 32-bit shared words (a count is at most T*k, which the
 // launcher keeps below 2^16).
-template <typename IdxT, int KM>
+__device__ __forceinline__ unsigned same_key_lanes(unsigned key, int bits, unsigned active)
+{
+    unsigned m = active;
+    for (int b = 0; b < bits; ++b) {
+        const bool set = (key >> b) & 1u;
+        const unsigned bb = __ballot_sync(kFull, set);
+        m &= set ? bb : ~bb;
+    }
+    return m;
+}
+
+template <typename IdxT>
 __device__ void summary_cta(const FusedParams &p, uint32_t *smem)
 {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -81,24 +99,37 @@ __device__ void summary_cta(const FusedParams &p, uint32_t *smem)
     __syncthreads();
 
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
+    const int tpw = 32 / k;
+    const int tl = lane / k, jl = lane - tl * k;
+    const unsigned kmask = k == 32 ? kFull : ((1u << k) - 1u);
+    const unsigned tokmask = tl < tpw ? kmask << (tl * k) : 0u;
+    const unsigned lt = lanemask_lt();
+    int bits_r = 1;
+    while ((1 << bits_r) < R) ++bits_r;
     bool bad = false;
     int nreal = 0;
-    for (int u = tid; u < p.T; u += kFusedThreads) {
-        unsigned long long m = 0ull;
-        int ev[KM];
+    const int nsteps = (p.T + tpw - 1) / tpw;
+    // four steps per iteration: their loads are issued together
+    for (int s0 = wid * 4; s0 < nsteps; s0 += kFusedWarps * 4) {
+        int ev[4];
 #pragma unroll
-        for (int j = 0; j < KM; ++j) ev[j] = j < k ? load_expert(idx, (size_t)u * k + j, E, &bad) : -1;
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-            const int e = ev[j];
-            if (e < 0) continue;
-            atomicAdd(&he[e >> 1], 1u << ((e & 1) * 16));
-            m |= 1ull << rank_of_e(e, p.inv_epr);
+        for (int a = 0; a < 4; ++a) {
+            const int u = (s0 + a) * tpw + tl;
+            ev[a] = (tl < tpw && u < p.T) ? load_expert(idx, (size_t)u * k + jl, E, &bad) : -1;
         }
-        nreal += m != 0ull;
-        while (m) {
-            atomicAdd(&hr[__ffsll((long long)m) - 1], 1);
-            m &= m - 1ull;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int e = ev[a];
+            const bool valid = e >= 0;
+            const int r = valid ? rank_of_e(e, p.inv_epr) : 0;
+            const unsigned vb = __ballot_sync(kFull, valid);
+            const unsigned same_r = same_key_lanes((unsigned)r, bits_r, vb) & tokmask;
+            if (valid) {
+                atomicAdd(&he[e >> 1], 1u << ((e & 1) * 16));
+                if (!(same_r & lt)) atomicAdd(&hr[r], 1);
+            }
+            // the token's first valid route counts it as real
+            nreal += valid && !(vb & tokmask & lt);
         }
     }
     if (__any_sync(kFull, bad) && lane == 0) atomicOr(&misc[0], 1);
@@ -168,20 +199,29 @@ __device__ void summary_cta(const FusedParams &p, uint32_t *smem)
 }
 
 // ------------------------------------------------------------ token CTAs
+//
+// Counting: one thread per token of the batch, its k route keys in
+// registers; the own token's slots and ranks are the queries, visited by a
+// plain loop (the same query in every lane at a time): each thread counts
+// its routes against the query, a warp reduction sums the warp's tokens, and
+// the lane that owns the query keeps the running sum.  Only the loop over a
+// token's own k routes is unrolled, so the kernel's code stays small -- after
+// an L2 flush the instructions come from DRAM again, and a large unrolled
+// body stalls on instruction fetch.
 
 template <typename IdxT, int KM, int VPT>
 __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedParams p)
 {
     extern __shared__ __align__(16) uint32_t fsmem[];
-    __shared__ int s_part[kFusedWarps][2 * KM];
-    __shared__ int s_rrow[KM];
-    __shared__ uint4 *s_dst[2 * KM];
+    __shared__ int s_part[kFusedWarps][64];  // per warp: [0, 32) slot counts, [32, 64) rank counts
+    __shared__ int s_rrow[32];
+    __shared__ uint4 *s_dst[64];
     __shared__ int s_n;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     if (blockIdx.x == 0) {
-        summary_cta<IdxT, KM>(p, fsmem);
+        summary_cta<IdxT>(p, fsmem);
         return;
     }
     const int b = (int)blockIdx.x - 1;
@@ -190,21 +230,16 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     const int k = p.k, E = p.E, R = p.R;
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
 
-    // this token's routes (the same k values in every thread)
-    bool bad = false;
-    int q_own[KM];
-    unsigned long long m_own = 0ull;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        q_own[j] = -1;
-        if (j < k) {
-            const int e = load_expert(idx, (size_t)t * k + j, E, &bad);
-            if (e >= 0) {
-                q_own[j] = 2 * e;
-                m_own |= 1ull << rank_of_e(e, p.inv_epr);
-            }
-        }
+    // this token's routes, one per lane (every warp reads them: no barrier)
+    int e_mine = -1;
+    if (lane < k) {
+        const long long ev = (long long)idx[(size_t)t * k + lane];
+        if (ev >= 0 && ev < E) e_mine = (int)ev;
     }
+    const int r_mine = e_mine >= 0 ? rank_of_e(e_mine, p.inv_epr) : -1;
+    const unsigned m_lo = __reduce_or_sync(kFull, r_mine >= 0 && r_mine < 32 ? 1u << r_mine : 0u);
+    const unsigned m_hi = __reduce_or_sync(kFull, r_mine >= 32 ? 1u << (r_mine - 32) : 0u);
+    const unsigned long long m_own = ((unsigned long long)m_hi << 32) | m_lo;
     if (m_own == 0ull) {  // no valid route: nothing to copy, rows of -1
         if (c == 0) {
             for (int j = tid; j < k; j += kFusedThreads) p.pos[(size_t)t * k + j] = -1;
@@ -224,87 +259,90 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         if (v < v1) val[u] = ld_nc_v4(src + v);
     }
 
-    // the token's ranks in increasing order
+    // queries: slot j's key 2 e_j (lane j); the q-th rank of the token in
+    // increasing order (lane q)
     const int nr = __popcll((long long)m_own);
-    int r_own[KM];
-    {
+    const int q_slot = e_mine >= 0 ? 2 * e_mine : -1;
+    int q_rank = 0;
+    if (lane < nr) {
         unsigned long long m = m_own;
+        for (int i = 0; i < lane; ++i) m &= m - 1ull;
+        q_rank = __ffsll((long long)m) - 1;
+    }
+
+    int acc_slot = 0, acc_rank = 0;
+    for (int u0 = wid * 32; u0 < p.T; u0 += kFusedThreads) {
+        const int u = u0 + lane;
+        const int after = u >= t;
+        // this thread's token: k route keys 2 e + [u >= t] (INT_MAX for no
+        // route) and its set of ranks
+        int key[KM];
+        unsigned long long m = 0ull;
 #pragma unroll
-        for (int q = 0; q < KM; ++q) {
-            r_own[q] = 64;
-            if (m) {
-                r_own[q] = __ffsll((long long)m) - 1;
-                m &= m - 1ull;
+        for (int j = 0; j < KM; ++j) {
+            key[j] = 0x7fffffff;
+            if (j < k && u < p.T) {
+                const long long ev = (long long)idx[(size_t)u * k + j];
+                if (ev >= 0 && ev < E) {
+                    key[j] = 2 * (int)ev + after;
+                    m |= 1ull << rank_of_e((int)ev, p.inv_epr);
+                }
+            }
+        }
+        // four queries at a time: their shuffles, compares and warp
+        // reductions are independent, so their latencies overlap
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            int n[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                // lanes >= k hold -1, which no key is below
+                const int qj = __shfl_sync(kFull, q_slot, (j0 + a) & 31);
+                n[a] = 0;
+#pragma unroll
+                for (int i = 0; i < KM; ++i) n[a] += key[i] <= qj;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int sum = __reduce_add_sync(kFull, n[a]);
+                if (lane == j0 + a) acc_slot += sum;
+            }
+        }
+        const int before = 1 - after;
+        for (int q0 = 0; q0 < nr; q0 += 4) {
+            int n[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int rq = __shfl_sync(kFull, q_rank, (q0 + a) & 31);
+                n[a] = q0 + a < nr ? __popcll((long long)(m & lowmask64(rq + before))) : 0;
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const int sum = __reduce_add_sync(kFull, n[a]);
+                if (lane == q0 + a) acc_rank += sum;
             }
         }
     }
-
-    // count routes (t', j') with 2 e' + [t' >= t] <= 2 e_j, and pairs
-    // (t', r') with r' < r_q + [t' < t]
-    int cnt[KM], cpr[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) cnt[j] = cpr[j] = 0;
-    for (int u = tid; u < p.T; u += kFusedThreads) {
-        const int after = u >= t;
-        // all k loads of the token first, so they are in flight together
-        long long ev[KM];
-#pragma unroll
-        for (int j2 = 0; j2 < KM; ++j2) ev[j2] = j2 < k ? (long long)idx[(size_t)u * k + j2] : -1;
-        unsigned long long m = 0ull;
-#pragma unroll
-        for (int j2 = 0; j2 < KM; ++j2) {
-            if (ev[j2] < 0 || ev[j2] >= E) continue;
-            const int e = (int)ev[j2];
-            const int key = 2 * e + after;
-#pragma unroll
-            for (int j = 0; j < KM; ++j) cnt[j] += key <= q_own[j];
-            m |= 1ull << rank_of_e(e, p.inv_epr);
-        }
-        if (m) {
-            const int before = 1 - after;
-#pragma unroll
-            for (int q = 0; q < KM; ++q)
-                if (q < nr) cpr[q] += __popcll((long long)(m & lowmask64(r_own[q] + before)));
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        if (j < k) {
-            const int s = __reduce_add_sync(kFull, cnt[j]);
-            if (lane == 0) s_part[wid][j] = s;
-        }
-        if (j < nr) {
-            const int s = __reduce_add_sync(kFull, cpr[j]);
-            if (lane == 0) s_part[wid][KM + j] = s;
-        }
-    }
+    s_part[wid][lane] = acc_slot;
+    s_part[wid][32 + lane] = acc_rank;
     __syncthreads();
 
     // warp 0: rows of the token's routes and pairs, destination list
     if (wid == 0) {
         const unsigned lt = lanemask_lt();
-        int e_mine = -1;
-        if (lane < k) {
-            bool b2 = false;
-            e_mine = load_expert(idx, (size_t)t * k + lane, E, &b2);
-        }
-        int dup = 0;
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
+        int dup = 0;  // earlier slots of this token with the same expert
+        for (int j = 0; j < k; ++j) {
             const int ej = __shfl_sync(kFull, e_mine, j);
             dup += (j < lane && ej == e_mine) ? 1 : 0;
         }
         int row = -1;
         if (lane < k && e_mine >= 0) {
             row = dup;
-#pragma unroll
             for (int w = 0; w < kFusedWarps; ++w) row += s_part[w][lane];
         }
         int rrow = -1;
         if (lane < nr) {
             rrow = 0;
-#pragma unroll
-            for (int w = 0; w < kFusedWarps; ++w) rrow += s_part[w][KM + lane];
+            for (int w = 0; w < kFusedWarps; ++w) rrow += s_part[w][32 + lane];
             s_rrow[lane] = rrow;
         }
         const bool ok_e = row >= 0 && (int64_t)row < p.exp_cap;
@@ -337,6 +375,10 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         }
     }
 }
+
+}  // namespace
+
+namespace {
 
 template <typename IdxT, int KM>
 cudaError_t launch_km(const FusedParams &p, int vpt, dim3 grid, size_t smem, cudaStream_t s)

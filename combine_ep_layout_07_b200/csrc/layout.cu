@@ -682,22 +682,26 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
 // ordinary grid -- up to one per SM, each with a few hundred routes -- in
 // place of one cluster of at most 16.  CTA totals cannot go through
 // distributed shared memory across a grid, so they go through a workspace
-// in global memory:
-//  * count phase as above, then the CTA's (expert | rank) totals are stored
-//    as one row of packed 16-bit counts;
-//  * one grid barrier: every CTA adds one to an arrival counter and waits
-//    (bounded: after kGridWaitLimit polls it flags EP_DEVERR_TIMEOUT and goes
-//    on) until all have arrived.  The grid never has more CTAs than SMs, and
-//    programmatic launch lets dependent grids start only once every CTA of
-//    this one has started, so all CTAs are resident together;
-//  * every CTA sums the rows -- over all CTAs (the totals) and over the CTAs
-//    below it (its bases) -- with many 16-byte loads in flight per thread,
-//    then runs the packed block scan and places its routes;
-//  * bad-index and real-token counts go into two more header words, and the
-//    last CTA to leave writes them to totals[2..3] and zeroes the header, so
-//    the workspace is clean after every call (it must be zero before the
-//    first one).
-constexpr int kGridHeader = kGridHeaderWords;  // workspace header words (first four used)
+// in global memory, with two grid barriers:
+//  * count phase as above; the CTA's (expert | rank) totals are stored as
+//    one row of packed 16-bit counts; barrier 1;
+//  * column scan: CTA b owns the count words b, b + nb, ...; for each, one
+//    thread per CTA row loads that row's word, a block scan turns the
+//    column into exclusive prefixes over the CTAs, stored in every CTA's
+//    prefix row, and the column totals; barrier 2;
+//  * every CTA reads its own prefix row and the totals (a few KB), runs the
+//    packed global scan and places its routes.
+// Each barrier is an arrival counter every CTA adds one to and then waits
+// on (bounded: after kGridWaitLimit polls it flags EP_DEVERR_TIMEOUT and goes
+// on).  The grid never has more CTAs than SMs, and programmatic launch lets
+// dependent grids start only once every CTA of this one has started, so all
+// CTAs are resident together.  Bad-index and real-token counts go into two
+// more header words; the last CTA to leave writes them to totals[2..3] and
+// zeroes the header, so the workspace is clean after every call (its header
+// must be zero before the first one).
+constexpr int kGridHeader = kGridHeaderWords;  // [0] arrivals 1, [1] departures,
+                                               // [2] error bits, [3] real tokens,
+                                               // [4] arrivals 2
 constexpr long long kGridWaitLimit = 1ll << 21;
 
 __device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
@@ -705,6 +709,23 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t *p)
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+// One thread: arrive at the counter and wait (bounded) for all nb CTAs;
+// false if the wait gave up (flagged in the header).
+__device__ __forceinline__ bool grid_arrive_wait(int32_t *counter, int32_t *flags, int nb)
+{
+    __threadfence();
+    atomicAdd(counter, 1);
+    for (long long i = 0; i < kGridWaitLimit; ++i) {
+        if (ld_acquire_gpu(counter) >= nb) {
+            __threadfence();
+            return true;
+        }
+        __nanosleep(32);
+    }
+    atomicOr(flags, (int)EP_DEVERR_TIMEOUT);
+    return false;
 }
 
 constexpr int kGridMaxThreads = 512;
@@ -722,29 +743,28 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
     pdl_launch_dependents();
 
     const int wt = p.tstr >> 1;
-    const int hs = p.hs;  // workspace row length in words (multiple of 4, >= wt)
+    const int hs = p.hs;                   // count row length in words (multiple of 4)
+    const int ps = (E + R + 3) & ~3;       // prefix row length in words
     const int nch_max = (p.tpc + tpw - 1) / tpw;
-    const int nq = hs >> 2;
-    const int G = (int)blockDim.x / nq > 1 ? (int)blockDim.x / nq : 1;
 
     uint32_t *tab = reinterpret_cast<uint32_t *>(smem);  // [chunks][wt]
     Smem sm;
     sm.M = nullptr;
     sm.codes = nullptr;
     sm.hit = nullptr;
+    sm.all_tot = nullptr;
     sm.scan = reinterpret_cast<unsigned long long *>(smem + warp_table_words(nch_max, wt));
     sm.tot = reinterpret_cast<int32_t *>(sm.scan + 34);
     sm.base = sm.tot + E + R;
     sm.low = sm.base + E + R;
-    sm.misc = sm.low + E + R;  // [0] bad flag, [1] real tokens, [2] barrier gave up
-    sm.all_tot = sm.misc + 3;  // [G][2][2 * hs] partial sums
+    sm.misc = sm.low + E + R;  // [0] bad flag, [1] real tokens, [2] a barrier gave up
     int *s_fail = sm.misc + 2;
 
     const int c0 = min(T, b * p.tpc);
     const int nt = min(T, c0 + p.tpc) - c0;
     const int nuse = (nt + tpw - 1) / tpw;
 
-    if (tid < 2) sm.misc[tid] = 0;
+    if (tid < 3) sm.misc[tid] = 0;
     zero_words(tab, nuse * wt);
     __syncthreads();
     pdl_wait_previous();
@@ -752,9 +772,12 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
     WarpRoutes<PASSES> wr;
     warp_count<IdxT, PASSES>(p, tab, sm, c0, nt, wr);
 
-    // ---- publish this CTA's totals, then the grid barrier
     int32_t *hdr = p.work;
-    uint32_t *rows = reinterpret_cast<uint32_t *>(p.work + kGridHeader);
+    uint32_t *rows = reinterpret_cast<uint32_t *>(p.work + kGridHeader);  // [nb][hs]
+    uint32_t *pref = rows + (size_t)nb * hs;                               // [nb][ps]
+    uint32_t *gtot = pref + (size_t)nb * ps;                               // [ps]
+
+    // ---- this CTA's totals as one row of packed 16-bit counts; barrier 1
     for (int w = tid; w < hs; w += blockDim.x) {
         const uint32_t lo = 2 * w < E + R ? (uint32_t)sm.tot[2 * w] : 0u;
         const uint32_t hi = 2 * w + 1 < E + R ? (uint32_t)sm.tot[2 * w + 1] : 0u;
@@ -764,69 +787,34 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
     if (tid == 0) {
         if (sm.misc[0]) atomicOr(&hdr[2], (int)EP_DEVERR_BAD_INDEX);
         if (sm.misc[1]) atomicAdd(&hdr[3], sm.misc[1]);
-        __threadfence();
-        atomicAdd(&hdr[0], 1);
-        bool ok = false;
-        for (long long i = 0; i < kGridWaitLimit; ++i) {
-            if (ld_acquire_gpu(&hdr[0]) >= nb) {
-                ok = true;
-                break;
-            }
-            __nanosleep(32);
-        }
-        if (!ok) atomicOr(&hdr[2], (int)EP_DEVERR_TIMEOUT);
-        *s_fail = ok ? 0 : 1;
-        __threadfence();
+        if (!grid_arrive_wait(&hdr[0], &hdr[2], nb)) *s_fail = 1;
     }
     __syncthreads();
 
-    // ---- column sums over all CTAs and over the CTAs below this one
-    for (int i = tid; i < nq * G; i += blockDim.x) {
-        const int q = i % nq, g = i / nq;
-        const int b0 = g * nb / G, b1 = (g + 1) * nb / G;
-        uint32_t tot[8], low[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) tot[u] = low[u] = 0u;
-        for (int bb = b0; bb < b1; bb += 8) {
-            uint4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (bb + u < b1)
-                    v[u] = __ldcg(reinterpret_cast<const uint4 *>(rows + (size_t)(bb + u) * hs) + q);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (bb + u < b1) {
-                    const uint32_t x4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                    const bool below = bb + u < b;
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        tot[2 * h] += x4[h] & 0xffffu;
-                        tot[2 * h + 1] += x4[h] >> 16;
-                        if (below) {
-                            low[2 * h] += x4[h] & 0xffffu;
-                            low[2 * h + 1] += x4[h] >> 16;
-                        }
-                    }
-                }
-            }
+    // ---- column scan of the words this CTA owns, over the CTAs; barrier 2
+    for (int w = b; 2 * w < E + R; w += nb) {
+        const uint32_t v = tid < nb ? __ldcg(rows + (size_t)tid * hs + w) : 0u;
+        unsigned long long total;
+        const unsigned long long ex = block_exclusive_scan64(
+            ((unsigned long long)(v >> 16) << 32) | (v & 0xffffu), sm.scan, &total);
+        if (tid < nb) {
+            pref[(size_t)tid * ps + 2 * w] = (uint32_t)(ex & 0xffffffffull);
+            if (2 * w + 1 < E + R) pref[(size_t)tid * ps + 2 * w + 1] = (uint32_t)(ex >> 32);
         }
-        uint32_t *pt = reinterpret_cast<uint32_t *>(sm.all_tot) + (size_t)g * 4 * hs;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            pt[8 * q + u] = tot[u];
-            pt[2 * hs + 8 * q + u] = low[u];
+        if (tid == 0) {
+            gtot[2 * w] = (uint32_t)(total & 0xffffffffull);
+            if (2 * w + 1 < E + R) gtot[2 * w + 1] = (uint32_t)(total >> 32);
         }
+        __syncthreads();  // sm.scan is reused by the next word
     }
     __syncthreads();
+    if (tid == 0 && !grid_arrive_wait(&hdr[4], &hdr[2], nb)) *s_fail = 1;
+    __syncthreads();
+
+    // ---- this CTA's bases: its prefix row and the totals
     for (int c = tid; c < E + R; c += blockDim.x) {
-        uint32_t t = 0, l = 0;
-        for (int g = 0; g < G; ++g) {
-            const uint32_t *pt = reinterpret_cast<const uint32_t *>(sm.all_tot) + (size_t)g * 4 * hs;
-            t += pt[c];
-            l += pt[2 * hs + c];
-        }
-        sm.tot[c] = (int32_t)t;
-        sm.low[c] = (int32_t)l;
+        sm.tot[c] = (int32_t)__ldcg(gtot + c);
+        sm.low[c] = (int32_t)__ldcg(pref + (size_t)b * ps + c);
     }
     __syncthreads();
     // this CTA no longer reads the workspace: leave (the last one out
@@ -837,6 +825,7 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
             p.totals[2] = atomicExch(&hdr[3], 0);
             p.totals[3] = atomicExch(&hdr[2], 0);
             atomicExch(&hdr[0], 0);
+            atomicExch(&hdr[4], 0);
             atomicExch(&hdr[1], 0);
         }
     }
@@ -963,11 +952,10 @@ bool plan_grid(int T, int k, int E, int R, int nsm, WarpGeometry *g, int *hs)
     if (passes > 4) return false;
     g->passes = passes <= 1 ? 1 : passes <= 2 ? 2 : 4;
     g->threads = warps * 32;
+    if (g->threads < g->csize) return false;  // the column scan takes one thread per CTA
     *hs = grid_row_words(E, R);
-    const int nq = *hs / 4;
-    const int G = g->threads / nq > 1 ? g->threads / nq : 1;
     g->smem = warp_table_words(nch, g->tstr >> 1) * 4 + 34 * 8 +
-              sizeof(int32_t) * (3 * (size_t)(E + R) + 3) + sizeof(uint32_t) * (size_t)G * 4 * *hs;
+              sizeof(int32_t) * (3 * (size_t)(E + R) + 3);
     return g->smem <= (size_t)kMaxDynSmem;
 }
 
@@ -1056,8 +1044,8 @@ cudaError_t set_attributes_once(int dev)
     return err;
 }
 
-// variant: 0 = the grid schedule for large batches, else warp chunks where
-// they fit, else the count matrix; 1 = warp chunks (cudaErrorNotSupported
+// variant: 0 = warp chunks where they fit, else the grid schedule where it
+// fits, else the count matrix; 1 = warp chunks (cudaErrorNotSupported
 // where they do not fit); 2 = count matrix; 3 = grid schedule
 // (cudaErrorNotSupported without a workspace or where it does not fit)
 template <typename IdxT>
@@ -1071,7 +1059,19 @@ cudaError_t launch_layout_t(const LayoutParams &p0, int variant, cudaStream_t s)
 
     LayoutParams p = p0;
     const long long routes = (long long)p.T * p.k;
-    if (variant == 3 || (variant == 0 && routes > kGridAutoRoutes && p.work)) {
+    // one CTA up to ~2K routes, then a cluster of up to 16 CTAs
+    int csize = (int)((routes + 2047) / 2048);
+    csize = csize < 1 ? 1 : (csize > 16 ? 16 : csize);
+    // automatic: the warp-chunk cluster where it fits (measured faster than
+    // the grid schedule at 4096 x top-8: its two grid barriers cost more
+    // than the cluster's exchange saves), then the grid schedule, then the
+    // count matrix
+    bool grid = variant == 3;
+    if (variant == 0 && p.work) {
+        WarpGeometry gw;
+        grid = !plan_warp(p.T, p.k, p.E, p.R, csize, &gw);
+    }
+    if (grid) {
         WarpGeometry g;
         int hs = 0;
         if (p.work && plan_grid(p.T, p.k, p.E, p.R, sm_count(dev), &g, &hs)) {
@@ -1087,9 +1087,6 @@ cudaError_t launch_layout_t(const LayoutParams &p0, int variant, cudaStream_t s)
         }
         if (variant == 3) return cudaErrorNotSupported;
     }
-    // one CTA up to ~2K routes, then a cluster of up to 16 CTAs
-    int csize = (int)((routes + 2047) / 2048);
-    csize = csize < 1 ? 1 : (csize > 16 ? 16 : csize);
 
     if (variant != 2) {
         WarpGeometry g;

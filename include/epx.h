@@ -153,16 +153,20 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
  * followed by ep_dispatch_expand with the same arguments (every array of *L,
  * recv, expanded and the error word).  For small batches (T*k up to
  * EPX_FUSED_MAX_ROUTES) it can run as ONE launch: every CTA derives its own
- * token's rows by counting over all routes while its chunk of x is in flight,
- * so nothing waits for a separate layout kernel -- the fixed cost that
- * dominates the low-batch regime of DeepEP issue #760's report.
- * variant: 0 = automatic (one launch for small batches, else two), 1 = one
- * launch (EP_ERR_UNSUPPORTED beyond EPX_FUSED_MAX_ROUTES), 2 = ep_layout then
+ * token's rows by counting over all routes (one thread per token, the
+ * token's slots and ranks as queries) while its chunk of x is in flight, so
+ * nothing waits for a separate layout kernel.  variant: 0 = automatic (one launch where it was
+ * measured faster, see EPX_FUSED_AUTO_MIN_ROUTES; else two), 1 = one launch
+ * (EP_ERR_UNSUPPORTED beyond EPX_FUSED_MAX_ROUTES), 2 = ep_layout then
  * ep_dispatch_expand.  Rows beyond a capacity are skipped and flagged
  * (EP_DEVERR_RECV_CAP / EP_DEVERR_EXP_CAP) as in ep_dispatch_expand.
  */
-#define EPX_FUSED_MAX_ROUTES 8192
-#define EPX_FUSED_AUTO_ROUTES 2048 /* variant 0 takes one launch up to here */
+#define EPX_FUSED_MAX_ROUTES 4096
+/* variant 0 takes one launch for T*k in [MIN, MAX]: measured on B200, below
+ * it the one warp that holds a handful of tokens walks the queries alone,
+ * above it every CTA's count over all routes outweighs the launch saved */
+#define EPX_FUSED_AUTO_MIN_ROUTES 512
+#define EPX_FUSED_AUTO_MAX_ROUTES 2048
 ep_status_t ep_layout_dispatch_expand(const void *topk_idx, const ep_layout_t *L,
                                       const void *x, int32_t H, void *recv,
                                       int64_t recv_cap, void *expanded,

@@ -142,7 +142,8 @@ def test_binding_constants_mirror_the_header():
     assert epx.MAX_RANKS == val("EPX_MAX_RANKS")
     assert epx.MAX_EXPERTS == val("EPX_MAX_EXPERTS")
     assert epx.FUSED_MAX_ROUTES == val("EPX_FUSED_MAX_ROUTES")
-    assert epx.FUSED_AUTO_ROUTES == val("EPX_FUSED_AUTO_ROUTES")
+    assert epx.FUSED_AUTO_MIN_ROUTES == val("EPX_FUSED_AUTO_MIN_ROUTES")
+    assert epx.FUSED_AUTO_MAX_ROUTES == val("EPX_FUSED_AUTO_MAX_ROUTES")
     assert epx.NOALLOC_SCRATCH_BYTES == val("EPX_NOALLOC_SCRATCH_BYTES") << 20
 
 

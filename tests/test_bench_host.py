@@ -43,10 +43,12 @@ def test_alg_bytes_one_launch_step():
 def test_step_call_choice_follows_the_library_threshold():
     from combine_ep_layout_07_b200 import epx
     a = bench.parse_args([])
-    assert bench.fused_step(a, 128, 8) and bench.fused_step(a, 1, 16)
-    assert not bench.fused_step(a, 4096, 8)
-    assert bench.fused_step(a, epx.FUSED_AUTO_ROUTES // 8, 8)
-    assert not bench.fused_step(a, epx.FUSED_AUTO_ROUTES // 8 + 1, 8)
+    assert bench.fused_step(a, 128, 8) and bench.fused_step(a, 128, 4)
+    assert not bench.fused_step(a, 4096, 8) and not bench.fused_step(a, 1, 16)
+    assert bench.fused_step(a, epx.FUSED_AUTO_MAX_ROUTES // 8, 8)
+    assert not bench.fused_step(a, epx.FUSED_AUTO_MAX_ROUTES // 8 + 1, 8)
+    assert bench.fused_step(a, epx.FUSED_AUTO_MIN_ROUTES // 8, 8)
+    assert not bench.fused_step(a, epx.FUSED_AUTO_MIN_ROUTES // 8 - 1, 8)
     assert not bench.fused_step(bench.parse_args(["--step-calls", "separate"]), 128, 8)
     assert bench.fused_step(bench.parse_args(["--step-calls", "fused"]), 960, 8)
     assert not bench.fused_step(bench.parse_args(["--no-expand"]), 128, 8)

@@ -40,6 +40,12 @@ def run_fused(wl, variant=0, idx_dtype=torch.int64, caps=None):
 @pytest.mark.parametrize("idx_dtype", [torch.int64, torch.int32], ids=["i64", "i32"])
 def test_fused_matches_oracle(name, seed, variant, idx_dtype):
     wl, o = oracle_run(name, seed)
+    if variant == 1 and wl["T"] * wl["k"] > epx.FUSED_MAX_ROUTES:
+        x, idx, _ = gpu_inputs(wl, idx_dtype)
+        with pytest.raises(epx.EpxError) as ei:   # beyond the one-launch limit
+            epx.layout_dispatch_expand(idx, x, wl["E"], wl["R"], variant=1)
+        assert ei.value.status == 6
+        return
     g = run_fused(wl, variant, idx_dtype)
     assert_all_equal(g, o)
 
@@ -65,8 +71,9 @@ FUSED_CASES = [
     dict(T=77, H=64, E=64, R=4, k=32),          # k = 32
     dict(T=5, H=8, E=8, R=8, k=1),
     dict(T=3, H=14336, E=16, R=4, k=4),         # wide rows: four vectors per thread
-    dict(T=1024, H=64, E=256, R=16, k=8),       # at the one-launch limit
-    dict(T=256, H=136, E=4096, R=64, k=32),     # every size limit at its maximum
+    dict(T=512, H=64, E=256, R=16, k=8),        # at the one-launch limit (4096 routes)
+    dict(T=128, H=136, E=4096, R=64, k=32),     # E, R and k at their maxima
+    dict(T=4096, H=8, E=8, R=2, k=1),           # one route per token, many tokens
     dict(T=200, H=128, E=96, R=48, k=12),       # R > 32: 64-bit rank sets
 ]
 
@@ -145,7 +152,7 @@ def test_fused_guard_bands_untouched():
 
 
 def test_fused_deterministic_across_runs():
-    wl, _ = oracle_run("dp_padded", 0)
+    wl, _ = oracle_run("dp_compact", 0)
     x, idx, _ = gpu_inputs(wl)
     ref = None
     for _ in range(10):
