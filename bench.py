@@ -519,17 +519,20 @@ class L2Flush:
     """Evicts L2 between steps by READING a buffer of twice its size (outside
     the timed events): lines the previous step left dirty are written back
     during the flush, and the step starts with its inputs in DRAM and no
-    dirty lines of anyone else's to write back."""
+    dirty lines of anyone else's to write back.  The buffer is float32 and
+    is summed in float32 into a preallocated scalar: no conversion copy (an
+    integer buffer summed into int64 is first converted, i.e. written, by
+    torch), one reduction kernel that only reads."""
 
     def __init__(self, torch, dev):
-        self.buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
-        self.sink = torch.empty((), dtype=torch.int64, device=dev)
+        self.buf = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
         self.torch = torch
 
     def __call__(self):
-        self.torch.sum(self.buf, dim=0, dtype=self.torch.int64, out=self.sink)
+        self.torch.sum(self.buf, dim=0, out=self.sink)
 
-    DESC = "L2 flushed between steps (256 MiB read, outside the timed events)"
+    DESC = "L2 flushed between steps (256 MiB float32 read, outside the timed events)"
 
 
 def time_step(torch, launch, n_calls, stream, dev, steps, warmup, flush=None, eager=False,

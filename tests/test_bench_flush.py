@@ -13,9 +13,25 @@ import bench  # noqa: E402
 def test_flush_reads_and_leaves_buffer_untouched():
     f = bench.L2Flush.__new__(bench.L2Flush)
     f.torch = torch
-    f.buf = torch.arange(1000, dtype=torch.int32)
-    f.sink = torch.empty((), dtype=torch.int64)
+    f.buf = torch.arange(1000, dtype=torch.float32)
+    f.sink = torch.empty((), dtype=torch.float32)
     before = f.buf.clone()
     f()
-    assert int(f.sink) == sum(range(1000))
+    assert float(f.sink) == float(sum(range(1000)))
     assert torch.equal(f.buf, before)
+
+
+def test_flush_reduction_needs_no_conversion_copy():
+    """The flush must only read: a float32 sum into a float32 scalar runs one
+    reduction (an int32 buffer summed with dtype=int64 would be converted --
+    written -- first).  On CPU, check that no temporary as large as the
+    buffer is created by watching the profiler's allocations."""
+    from torch.profiler import ProfilerActivity, profile
+    f = bench.L2Flush.__new__(bench.L2Flush)
+    f.torch = torch
+    f.buf = torch.zeros(1 << 22, dtype=torch.float32)
+    f.sink = torch.empty((), dtype=torch.float32)
+    with profile(activities=[ProfilerActivity.CPU], profile_memory=True) as prof:
+        f()
+    big = [e for e in prof.events() if e.cpu_memory_usage >= f.buf.numel() * 4]
+    assert not big
