@@ -230,12 +230,19 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     const int k = p.k, E = p.E, R = p.R;
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
 
-    // this token's routes, one per lane (every warp reads them: no barrier)
-    int e_mine = -1;
-    if (lane < k) {
-        const long long ev = (long long)idx[(size_t)t * k + lane];
-        if (ev >= 0 && ev < E) e_mine = (int)ev;
+    // the loads the count needs are issued before anything waits on one:
+    // this token's routes (one per lane; every warp reads them, so no
+    // barrier) and the first batch of route indices (one token per thread)
+    long long own = -1;
+    if (lane < k) own = (long long)idx[(size_t)t * k + lane];
+    long long kv[KM];
+    {
+        const int u = wid * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            kv[j] = (j < k && u < p.T) ? (long long)idx[(size_t)u * k + j] : -1;
     }
+    const int e_mine = (own >= 0 && own < E) ? (int)own : -1;
     const int r_mine = e_mine >= 0 ? rank_of_e(e_mine, p.inv_epr) : -1;
     const unsigned m_lo = __reduce_or_sync(kFull, r_mine >= 0 && r_mine < 32 ? 1u << r_mine : 0u);
     const unsigned m_hi = __reduce_or_sync(kFull, r_mine >= 32 ? 1u << (r_mine - 32) : 0u);
@@ -281,13 +288,17 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
             key[j] = 0x7fffffff;
-            if (j < k && u < p.T) {
-                const long long ev = (long long)idx[(size_t)u * k + j];
-                if (ev >= 0 && ev < E) {
-                    key[j] = 2 * (int)ev + after;
-                    m |= 1ull << rank_of_e((int)ev, p.inv_epr);
-                }
+            if (kv[j] >= 0 && kv[j] < E) {
+                key[j] = 2 * (int)kv[j] + after;
+                m |= 1ull << rank_of_e((int)kv[j], p.inv_epr);
             }
+        }
+        // the next batch's indices, in flight while this one is counted
+        {
+            const int un = u + kFusedThreads;
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                kv[j] = (j < k && un < p.T) ? (long long)idx[(size_t)un * k + j] : -1;
         }
         // four queries at a time: their shuffles, compares and warp
         // reductions are independent, so their latencies overlap
