@@ -8,11 +8,13 @@
 // layout launch is a chain of dependent steps (load, count, exchange, scan,
 // place) that the dispatch must wait for; here that chain is removed:
 //
-//  * CTA (token t, chunk c) loads its chunk of x[t] into registers first, so
-//    the DRAM latency of x overlaps everything below;
-//  * it then derives its own token's rows by counting over all T*k routes
-//    (topk_idx is a few KB and stays in L2 after the first CTA reads it).
-//    In (expert, token, slot) order the row of route (t, j) with expert e is
+//  * CTA (token t, chunk c) first issues every load it needs: its token's
+//    k routes, the route indices of its first batch of tokens (one token per
+//    thread; topk_idx is a few KB and stays in L2 after the first CTA reads
+//    it) and, once the token is known to have a route, its chunk of x[t], so
+//    the DRAM latency of x overlaps the count;
+//  * it derives its own token's rows by counting over all T*k routes.  In
+//    (expert, token, slot) order the row of route (t, j) with expert e is
 //    the number of valid routes before it:
 //        pos[t, j] = #{(t', j') : e' < e, or e' == e and t' < t}
 //                  + #{j' < j : e_{t, j'} == e}.
@@ -20,10 +22,11 @@
 //    routes with K' <= Q, one compare per (route, slot).  Likewise a
 //    (token, rank) pair's row is the number of pairs (t', r') with r' < r,
 //    or r' == r and t' < t: popcount(M' & lowmask(r + [t' < t])) summed over
-//    tokens t', M' being t''s set of ranks;
-//  * the per-thread counts are summed with warp reductions, and the CTA
-//    stores its chunk to every destination row;
-//  * chunk 0 of token t writes pos[t, :] and recv_pos[t, :];
+//    tokens t', M' being t''s set of ranks.  Each thread holds one token's
+//    keys and rank set; the token's slots and ranks are the queries, four at
+//    a time, each summed over the warp by a warp reduction;
+//  * warp 0 adds the warps' counts, and the CTA stores its chunk to every
+//    destination row; chunk 0 of token t writes pos[t, :] and recv_pos[t, :];
 //  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
 //    counts and exclusive scans, the totals and the error word.
 //
@@ -412,8 +415,12 @@ cudaError_t launch_t(const FusedParams &p, int vpt, dim3 grid, size_t smem, cuda
 
 }  // namespace
 
+// Target CTAs per SM.  Every CTA counts over all routes, so fewer, wider
+// chunks cost less count work in total; measured on B200 (amortised steps):
+// decode 20.3 us at 1 CTA per SM against 20.7 at 2 and 21.0 at 4, DP
+// compact 20.4 / 20.6 / 20.9 us, tiny unchanged.
 #ifndef EPX_FUSED_CTAS_PER_SM
-#define EPX_FUSED_CTAS_PER_SM 4
+#define EPX_FUSED_CTAS_PER_SM 1
 #endif
 
 cudaError_t launch_layout_dispatch(const FusedParams &p0, int idx_bits, cudaStream_t s)
