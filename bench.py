@@ -103,11 +103,11 @@ def parse_args(argv=None):
                     help="dispatch writes recv rows only plus a gather index (the expert "
                          "consumer reads recv through it); also times that consumer "
                          "against the one reading the expanded copy")
-    ap.add_argument("--step-calls", choices=["auto", "separate", "fused"], default="auto",
-                    help="layout and dispatch/expand as one call (one launch, small batches), "
-                         "as two calls, or automatic (one launch for EPX_FUSED_AUTO_MIN_ROUTES "
-                         "to EPX_FUSED_AUTO_MAX_ROUTES routes, as the library's automatic "
-                         "choice)")
+    ap.add_argument("--step-calls", choices=["auto", "separate", "fused", "paired"],
+                    default="auto",
+                    help="layout and dispatch/expand as one kernel (fused), as one call of two "
+                         "kernels whose dispatch reads x early (paired), as two calls "
+                         "(separate), or automatic (see step_mode)")
     ap.add_argument("--small-steps", type=int, default=1500,
                     help="steps of each small-batch workload measured beside the headline "
                          "(0 skips them)")
@@ -136,6 +136,8 @@ def load_peaks():
 
 def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None,
               no_expand=False, fused=False):
+    # fused: False / "separate" (layout and dispatch_expand apart), True /
+    # "one_launch" (one kernel), "paired" (one call of the two kernels)
     """Algorithmic HBM bytes per step of each kernel (each byte the definition
     must move once; no re-reads).  With part_bytes (4 or 2) the combine is the
     two-stage form: local reduce + epilogue through N_recv partial rows.  With
@@ -144,8 +146,11 @@ def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None,
     layout's own pos / recv_pos stores replace the dispatch's loads of them)."""
     row = H * 2
     layout = T * k * idx_bytes + T * k * 4 + T * R * 4
-    if fused:
+    if fused is True or fused == "one_launch":
         out = dict(layout_dispatch_expand=layout + T_real * row + (N_recv + N_route) * row)
+    elif fused == "paired":
+        out = dict(layout_dispatch_expand=layout + T_real * row + (N_recv + N_route) * row
+                   + T * k * 4 + T * R * 4)
     elif no_expand:
         out = dict(layout=layout,
                    dispatch=T_real * row + N_recv * row + T * R * 4,
@@ -414,22 +419,35 @@ def run_reference(args):
     return 0
 
 
-def fused_step(args, T, k):
-    """Whether the step runs layout + dispatch/expand as one launch."""
+def step_mode(args, T, k):
+    """How the step runs layout and dispatch/expand: "one_launch" (one kernel,
+    ep_layout_dispatch_expand variant 1), "paired" (ep_layout_dispatch_expand
+    variant 2: the layout and a dispatch that reads x before its wait, one
+    call), or "separate" (ep_layout, then ep_dispatch_expand).  Automatic: the
+    library's choice for small batches (one launch from
+    EPX_FUSED_AUTO_MIN_ROUTES to EPX_FUSED_AUTO_MAX_ROUTES routes, paired
+    below), separate calls above (so that the per-kernel split keeps the
+    layout and the dispatch apart)."""
     if getattr(args, "no_expand", False) or args.step_calls == "separate":
-        return False
+        return "separate"
     if args.step_calls == "fused":
-        return True
+        return "one_launch"
+    if args.step_calls == "paired":
+        return "paired"
     from combine_ep_layout_07_b200 import epx
-    return epx.FUSED_AUTO_MIN_ROUTES <= T * k <= epx.FUSED_AUTO_MAX_ROUTES
+    if epx.FUSED_AUTO_MIN_ROUTES <= T * k <= epx.FUSED_AUTO_MAX_ROUTES:
+        return "one_launch"
+    return "paired" if T * k < epx.FUSED_AUTO_MIN_ROUTES else "separate"
 
 
-def workload_config(wl, args, lay_totals, flush_desc=None, fused=False):
+def workload_config(wl, args, lay_totals, flush_desc=None, mode="separate"):
     cfg = {"workload": DESCRIBE[args.workload], "T": wl["T"], "H": wl["H"], "E": wl["E"],
            "R": wl["R"], "k": wl["k"], "seed": args.seed, "idx_bits": args.idx_bits,
            "T_real": int(lay_totals["T_real"]), "N_recv": int(lay_totals["N_recv"]),
            "N_route": int(lay_totals["N_route"]),
-           "timed": ("layout_dispatch_expand (one launch) + " if fused else "layout + " + (
+           "timed": ({"one_launch": "layout_dispatch_expand (one launch) + ",
+                      "paired": "layout_dispatch_expand (layout + dispatch_expand in one call) + "
+                      }.get(mode) or "layout + " + (
                "dispatch (recv only) + expand_index + " if getattr(args, "no_expand", False)
                else "dispatch_expand + ")) + (
                "combine_reduce" if not getattr(args, "two_stage", None) else
@@ -447,7 +465,7 @@ def workload_config(wl, args, lay_totals, flush_desc=None, fused=False):
 class Step:
     """Device buffers and the calls of one step of the path on one workload."""
 
-    def __init__(self, torch, epx, wl, args, dev, fused, two_stage=None, no_expand=False):
+    def __init__(self, torch, epx, wl, args, dev, mode, two_stage=None, no_expand=False):
         self.torch, self.epx, self.wl = torch, epx, wl
         T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
         itype = torch.int64 if args.idx_bits == 64 else torch.int32
@@ -467,11 +485,12 @@ class Step:
                 dtype=torch.float32 if two_stage == "fp32" else torch.bfloat16)
         self.src = src = (torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev)
                           if no_expand else None)
-        self.fused, self.no_expand = fused, no_expand
+        self.mode, self.no_expand = mode, no_expand
         calls = []
-        if fused:
+        if mode in ("one_launch", "paired"):
+            v = 1 if mode == "one_launch" else 2
             calls.append(("layout_dispatch_expand", lambda st: epx.layout_dispatch_expand(
-                idx, x, E, R, out=lay, recv=recv, expanded=expanded, variant=1, stream=st)))
+                idx, x, E, R, out=lay, recv=recv, expanded=expanded, variant=v, stream=st)))
         else:
             calls.append(("layout", lambda st: epx.layout(
                 idx, E, R, out=lay, variant=args.layout_variant, stream=st)))
@@ -683,15 +702,15 @@ def measure_small(torch, epx, wlmod, args, dev, stream, peak, flush, floors):
         if name == args.workload:
             continue
         wl = wlmod.make(name, seed=args.seed)
-        fused = fused_step(args, wl["T"], wl["k"])
-        st = Step(torch, epx, wl, args, dev, fused)
+        mode = step_mode(args, wl["T"], wl["k"])
+        st = Step(torch, epx, wl, args, dev, mode)
         tot = st.prepare(stream)
         ms, rec_k, _ = time_step(torch, st.launch, len(st.calls), stream, dev, args.small_steps,
                                  max(3, args.warmup), flush=flush)
         stats = step_stats(ms)
         am = time_amortized(torch, st.launch, stream, dev, flush)
         b = alg_bytes(wl["T"], tot["T_real"], tot["N_recv"], tot["N_route"], wl["H"], wl["k"],
-                      wl["R"], args.idx_bits // 8, fused=fused)
+                      wl["R"], args.idx_bits // 8, fused=mode)
         kern = {n: statistics.median([r[i] - (r[i - 1] if i else 0.0) for r in rec_k]) * 1e3
                 for i, n in enumerate(st.names)}
         floor = floors.get(len(st.calls))
@@ -731,8 +750,8 @@ def run_epx(args):
     wl = wlmod.make(args.workload, seed=args.seed + rank)
     T, H, E, R, k = wl["T"], wl["H"], wl["E"], wl["R"], wl["k"]
     stream = torch.cuda.Stream(device=dev)
-    fused = fused_step(args, T, k)
-    step = Step(torch, epx, wl, args, dev, fused, two_stage=args.two_stage,
+    mode = step_mode(args, T, k)
+    step = Step(torch, epx, wl, args, dev, mode, two_stage=args.two_stage,
                 no_expand=args.no_expand)
     tot = step.prepare(stream)
     lay, recv, expanded, y, out = step.lay, step.recv, step.expanded, step.y, step.out
@@ -744,7 +763,7 @@ def run_epx(args):
     bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
                        args.idx_bits // 8,
                        None if step.part is None else step.part.element_size(), args.no_expand,
-                       fused=fused)
+                       fused=mode)
     working = bytes_["total"]
     do_flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
     l2flush = L2Flush(torch, dev)
@@ -800,7 +819,7 @@ def run_epx(args):
     engine = {"dispatch": "recv_only", "expand_index": "gather_index",
               "combine_local": "two_stage_" + str(args.two_stage),
               "combine_epilogue": "two_stage_" + str(args.two_stage),
-              "layout_dispatch_expand": "one_launch",
+              "layout_dispatch_expand": mode,
               "dispatch_expand": "bulk" if args.dispatch_variant == 2 or
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
               "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split",
@@ -818,7 +837,7 @@ def run_epx(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(wl, args, tot, flush_desc, fused),
+        "config": workload_config(wl, args, tot, flush_desc, mode),
         "roofline": roofline,
         "step_hbm": {"alg_bytes": bytes_["total"], "gbs": step_gbs, "frac": step_gbs / peak},
         "step_us": step_stats(step_ms),

@@ -136,9 +136,16 @@ ep_status_t ep_layout(const void *topk_idx, const ep_layout_t *L, void *stream)
     return ep_layout_variant(topk_idx, L, 0, stream);
 }
 
-ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout_t *L,
-                                       void *recv, int64_t recv_cap, void *expanded,
-                                       int64_t exp_cap, int32_t variant, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Dispatch + expand; topk_idx non-null means the previous kernel on the
+// stream is this library's layout kernel for the same batch (see
+// DispatchParams::prefetch).
+ep_status_t dispatch_expand_impl(const void *x, int32_t H, const ep_layout_t *L, void *recv,
+                                 int64_t recv_cap, void *expanded, int64_t exp_cap,
+                                 int32_t variant, const void *topk_idx, void *stream)
 {
     if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
     if (H <= 0 || H % 8 != 0 || recv_cap < 0 || exp_cap < 0) return EP_ERR_INVALID_ARG;
@@ -161,7 +168,23 @@ ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout
     p.expanded = static_cast<uint4 *>(expanded);
     p.exp_cap = exp_cap;
     p.err = L->totals + 3;
+    p.prefetch = topk_idx != nullptr;
+    p.idx = topk_idx;
+    p.idx_bits = L->idx_bits;
+    p.E = L->E;
     return from_cuda(launch_dispatch(p, variant, as_stream(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+ep_status_t ep_dispatch_expand_variant(const void *x, int32_t H, const ep_layout_t *L,
+                                       void *recv, int64_t recv_cap, void *expanded,
+                                       int64_t exp_cap, int32_t variant, void *stream)
+{
+    return dispatch_expand_impl(x, H, L, recv, recv_cap, expanded, exp_cap, variant, nullptr,
+                                stream);
 }
 
 ep_status_t ep_dispatch_expand(const void *x, int32_t H, const ep_layout_t *L, void *recv,
@@ -197,7 +220,9 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     if (variant == 2) {
         ep_status_t st = ep_layout(topk_idx, L, stream);
         if (st != EP_OK || L->T == 0) return st;
-        return ep_dispatch_expand(x, H, L, recv, recv_cap, expanded, exp_cap, stream);
+        // the layout kernel just launched lets the dispatch read x early
+        return dispatch_expand_impl(x, H, L, recv, recv_cap, expanded, exp_cap, 0, topk_idx,
+                                    stream);
     }
     FusedParams p;
     memset(&p, 0, sizeof p);
@@ -224,8 +249,9 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     if (e == cudaErrorNotSupported) {  // checked before launching anything
         if (!automatic) return EP_ERR_UNSUPPORTED;
         const ep_status_t st = ep_layout(topk_idx, L, stream);
-        if (st != EP_OK) return st;
-        return ep_dispatch_expand(x, H, L, recv, recv_cap, expanded, exp_cap, stream);
+        if (st != EP_OK || L->T == 0) return st;
+        return dispatch_expand_impl(x, H, L, recv, recv_cap, expanded, exp_cap, 0, topk_idx,
+                                    stream);
     }
     return from_cuda(e);
 }

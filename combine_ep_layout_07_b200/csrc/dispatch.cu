@@ -61,12 +61,47 @@ __device__ __forceinline__ int build_dst_list(const DispatchParams &p, int t,
 
 // ---------------------------------------------------------------- vector
 
+// Whether token t has a valid route (warp-collective, from topk_idx).
+__device__ __forceinline__ bool token_has_route(const DispatchParams &p, int t)
+{
+    const int lane = threadIdx.x & 31;
+    long long e = -1;
+    if (lane < p.k)
+        e = p.idx_bits == 64 ? static_cast<const long long *>(p.idx)[(size_t)t * p.k + lane]
+                             : (long long)static_cast<const int *>(p.idx)[(size_t)t * p.k + lane];
+    return __any_sync(kFull, e >= 0 && e < p.E);
+}
+
 template <int VPT, bool STREAM>
 __global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
 {
     __shared__ uint4 *s_dst[kMaxDst];
     __shared__ int s_n;
+    __shared__ int s_pre;
     if (p.early_pdl) pdl_launch_dependents();
+    // with prefetch, the first token's chunk of x is loaded before the wait
+    // (only if the token has a route: rows without one are never read), so
+    // its DRAM latency overlaps the layout kernel
+    uint4 pre[VPT];
+    bool have_pre = false;
+    const int v0 = blockIdx.x * p.vpc;
+    const int v1 = min(p.V, v0 + p.vpc);
+    if (p.prefetch) {
+        if (threadIdx.x < 32) {
+            const bool ok = token_has_route(p, blockIdx.y);
+            if (threadIdx.x == 0) s_pre = ok;
+        }
+        __syncthreads();
+        if (s_pre) {
+            const uint4 *src = p.x + (size_t)blockIdx.y * p.V;
+#pragma unroll
+            for (int u = 0; u < VPT; ++u) {
+                const int vv = v0 + threadIdx.x + u * blockDim.x;
+                if (vv < v1) pre[u] = ld_nc_v4(src + vv);
+            }
+            have_pre = true;
+        }
+    }
     pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
@@ -76,15 +111,14 @@ __global__ void __launch_bounds__(128) dispatch_vec_kernel(DispatchParams p)
         __syncthreads();
         const int n = s_n;
         if (n > 0) {
-            const int v0 = blockIdx.x * p.vpc;
-            const int v1 = min(p.V, v0 + p.vpc);
             const uint4 *src = p.x + (size_t)t * p.V;
             for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x * VPT) {
                 uint4 val[VPT];
+                const bool use_pre = have_pre && t == (int)blockIdx.y && v == v0 + (int)threadIdx.x;
 #pragma unroll
                 for (int u = 0; u < VPT; ++u) {
                     const int vv = v + u * blockDim.x;
-                    if (vv < v1) val[u] = ld_nc_v4(src + vv);
+                    if (vv < v1) val[u] = use_pre ? pre[u] : ld_nc_v4(src + vv);
                 }
                 for (int i = 0; i < n; ++i) {
                     uint4 *d = s_dst[i];

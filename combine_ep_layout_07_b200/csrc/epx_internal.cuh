@@ -72,6 +72,13 @@ struct DispatchParams {
     int32_t *err;
     int early_pdl;  // trigger dependents at start (grid fits in one wave)
     long long first_wait_limit;  // bulk engine: polls allowed by a CTA's first bounded wait
+    // vector engine: the previous kernel is this library's layout kernel,
+    // launched for the same batch: it lets this grid start only once every
+    // kernel before it has completed, so x and topk_idx (which the layout
+    // does not write) may be read before this kernel's wait
+    int prefetch;
+    const void *idx;  // topk_idx [T, k], idx_bits wide (prefetch only)
+    int idx_bits, E;
 };
 
 // layout + dispatch/expand in one launch (small batches)

@@ -384,7 +384,6 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     extern __shared__ __align__(16) int32_t smem[];
     const int tid = threadIdx.x;
     const int E = p.E, R = p.R, T = p.T;
-    pdl_launch_dependents();
 
     int crank = 0, csize = 1;
     if (CLUSTER) {
@@ -423,6 +422,12 @@ __global__ void __launch_bounds__(1024, 1) layout_kernel(LayoutParams p)
     // peers write into this CTA's shared memory only once every CTA runs
     if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     pdl_wait_previous();
+    // the dependent grid (normally the dispatch) launches only now, when
+    // every kernel before this one has completed: it may then read the
+    // batch's inputs (x, topk_idx) before its own wait.  For the grid
+    // schedule this also means dependents start only once every CTA of this
+    // grid is resident.
+    pdl_launch_dependents();
 
     if (nchunks <= 1) {
         nreal = build_tokens(p, idx, c0, nt, sm, false, &bad);
@@ -634,7 +639,6 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
     extern __shared__ __align__(16) int32_t smem[];
     const int tid = threadIdx.x;
     const int E = p.E, R = p.R, T = p.T, tpw = p.tpw;
-    pdl_launch_dependents();
 
     int crank = 0, csize = 1;
     if (CLUSTER) {
@@ -668,6 +672,12 @@ __global__ void __launch_bounds__(1024, 1) layout_warp_kernel(LayoutParams p)
     __syncthreads();
     if (CLUSTER) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     pdl_wait_previous();
+    // the dependent grid (normally the dispatch) launches only now, when
+    // every kernel before this one has completed: it may then read the
+    // batch's inputs (x, topk_idx) before its own wait.  For the grid
+    // schedule this also means dependents start only once every CTA of this
+    // grid is resident.
+    pdl_launch_dependents();
 
     WarpRoutes<PASSES> wr;
     warp_count<IdxT, PASSES>(p, tab, sm, c0, nt, wr);
@@ -738,9 +748,6 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
     const int tid = threadIdx.x;
     const int E = p.E, R = p.R, T = p.T, tpw = p.tpw;
     const int nb = (int)gridDim.x, b = (int)blockIdx.x;
-    // dependents start launching only once every CTA of this grid has passed
-    // this point, i.e. once all of them are resident
-    pdl_launch_dependents();
 
     const int wt = p.tstr >> 1;
     const int hs = p.hs;                   // count row length in words (multiple of 4)
@@ -768,6 +775,12 @@ __global__ void __launch_bounds__(kGridMaxThreads, 1) layout_grid_kernel(LayoutP
     zero_words(tab, nuse * wt);
     __syncthreads();
     pdl_wait_previous();
+    // the dependent grid (normally the dispatch) launches only now, when
+    // every kernel before this one has completed: it may then read the
+    // batch's inputs (x, topk_idx) before its own wait.  For the grid
+    // schedule this also means dependents start only once every CTA of this
+    // grid is resident.
+    pdl_launch_dependents();
 
     WarpRoutes<PASSES> wr;
     warp_count<IdxT, PASSES>(p, tab, sm, c0, nt, wr);

@@ -155,10 +155,15 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
  * EPX_FUSED_MAX_ROUTES) it can run as ONE launch: every CTA derives its own
  * token's rows by counting over all routes (one thread per token, the
  * token's slots and ranks as queries) while its chunk of x is in flight, so
- * nothing waits for a separate layout kernel.  variant: 0 = automatic (one launch where it was
- * measured faster, see EPX_FUSED_AUTO_MIN_ROUTES; else two), 1 = one launch
- * (EP_ERR_UNSUPPORTED beyond EPX_FUSED_MAX_ROUTES), 2 = ep_layout then
- * ep_dispatch_expand.  Rows beyond a capacity are skipped and flagged
+ * nothing waits for a separate layout kernel.  Otherwise it runs the layout
+ * kernel and the dispatch kernel back to back; since the layout kernel lets
+ * its successor start only once every earlier kernel on the stream has
+ * completed, the dispatch launched here reads topk_idx and its first chunk
+ * of x (for a token with a route) before waiting for the layout, so the
+ * DRAM latency of x overlaps the layout.  variant: 0 = automatic (one
+ * launch where it was measured faster, see EPX_FUSED_AUTO_MIN_ROUTES; else
+ * two), 1 = one launch (EP_ERR_UNSUPPORTED beyond EPX_FUSED_MAX_ROUTES),
+ * 2 = the two kernels.  Rows beyond a capacity are skipped and flagged
  * (EP_DEVERR_RECV_CAP / EP_DEVERR_EXP_CAP) as in ep_dispatch_expand.
  */
 #define EPX_FUSED_MAX_ROUTES 4096

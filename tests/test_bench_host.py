@@ -43,15 +43,24 @@ def test_alg_bytes_one_launch_step():
 def test_step_call_choice_follows_the_library_threshold():
     from combine_ep_layout_07_b200 import epx
     a = bench.parse_args([])
-    assert bench.fused_step(a, 128, 8) and bench.fused_step(a, 128, 4)
-    assert not bench.fused_step(a, 4096, 8) and not bench.fused_step(a, 1, 16)
-    assert bench.fused_step(a, epx.FUSED_AUTO_MAX_ROUTES // 8, 8)
-    assert not bench.fused_step(a, epx.FUSED_AUTO_MAX_ROUTES // 8 + 1, 8)
-    assert bench.fused_step(a, epx.FUSED_AUTO_MIN_ROUTES // 8, 8)
-    assert not bench.fused_step(a, epx.FUSED_AUTO_MIN_ROUTES // 8 - 1, 8)
-    assert not bench.fused_step(bench.parse_args(["--step-calls", "separate"]), 128, 8)
-    assert bench.fused_step(bench.parse_args(["--step-calls", "fused"]), 960, 8)
-    assert not bench.fused_step(bench.parse_args(["--no-expand"]), 128, 8)
+    m = lambda T, k, argv=(): bench.step_mode(bench.parse_args(list(argv)), T, k)  # noqa: E731
+    assert m(128, 8) == "one_launch" and m(128, 4) == "one_launch"
+    assert m(4096, 8) == "separate" and m(1, 16) == "paired"
+    assert m(epx.FUSED_AUTO_MAX_ROUTES // 8, 8) == "one_launch"
+    assert m(epx.FUSED_AUTO_MAX_ROUTES // 8 + 1, 8) == "separate"
+    assert m(epx.FUSED_AUTO_MIN_ROUTES // 8, 8) == "one_launch"
+    assert m(epx.FUSED_AUTO_MIN_ROUTES // 8 - 1, 8) == "paired"
+    assert m(128, 8, ["--step-calls", "separate"]) == "separate"
+    assert m(960, 8, ["--step-calls", "fused"]) == "one_launch"
+    assert m(4096, 8, ["--step-calls", "paired"]) == "paired"
+    assert m(128, 8, ["--no-expand"]) == "separate"
+    assert a.step_calls == "auto"
+
+
+def test_alg_bytes_paired_step_keeps_the_position_reads():
+    one = bench.alg_bytes(8, 1, 16, 16, 3584, 16, 32, 8, fused="one_launch")
+    two = bench.alg_bytes(8, 1, 16, 16, 3584, 16, 32, 8, fused="paired")
+    assert two["layout_dispatch_expand"] - one["layout_dispatch_expand"] == 8 * 16 * 4 + 8 * 32 * 4
 
 
 def test_traffic_lookup_follows_source_and_engine(tmp_path, monkeypatch):

@@ -1,7 +1,9 @@
-"""GPU parity of the one-launch layout + dispatch/expand
-(ep_layout_dispatch_expand): every array of the layout, the received and the
-expanded rows bit-exact against the CPU oracle, the combine on top of it
-within tolerance, on the seeded workloads and on edge shapes."""
+"""GPU parity of ep_layout_dispatch_expand -- the one-launch kernel (variant
+1), the layout kernel followed by a dispatch that reads x before its wait
+(variant 2) and the automatic choice between them (0): every array of the
+layout, the received and the expanded rows bit-exact against the CPU oracle,
+the combine on top of it within tolerance, on the seeded workloads and on
+edge shapes (padding rows, bad indices, duplicates)."""
 import numpy as np
 import pytest
 import torch
@@ -36,7 +38,7 @@ def run_fused(wl, variant=0, idx_dtype=torch.int64, caps=None):
 
 @pytest.mark.parametrize("name", SMALL)
 @pytest.mark.parametrize("seed", [0, 1, 2])
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2])
 @pytest.mark.parametrize("idx_dtype", [torch.int64, torch.int32], ids=["i64", "i32"])
 def test_fused_matches_oracle(name, seed, variant, idx_dtype):
     wl, o = oracle_run(name, seed)
@@ -79,7 +81,7 @@ FUSED_CASES = [
 
 
 @pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "T{T}k{k}E{E}R{R}H{H}".format(**c))
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [0, 1, 2])
 def test_fused_edge_shapes(case, variant):
     wl = _random_wl(seed=case["T"] * 7 + case["k"], p_pad=0.2, distinct=False, **case)
     idx = wl["topk_idx"]
