@@ -162,3 +162,21 @@ def test_one_launch_call_validates_on_host(lib):
     assert lib.ep_latency_floor(None, 0, 3, None) == 1
     assert lib.ep_latency_floor(fake, 64, 3, None) == 1                            # too small
     assert lib.ep_latency_floor(fake + 4, 64 * 8, 3, None) == 2
+
+
+def test_layout_block_holds_the_grid_workspace(lib):
+    """ep_layout_bytes covers the grid schedule's workspace after the
+    totals: a 16-word header, one row of packed counts and one row of
+    32-bit prefixes per CTA (one CTA per 256 routes, at most 256 CTAs), and
+    the totals row."""
+    c = epx._LayoutC()
+    fake = 0x100000
+    for (T, k, E, R) in [(4096, 8, 256, 16), (1, 1, 1, 1), (128, 32, 4096, 64), (70000, 8, 256, 16)]:
+        n = lib.ep_layout_bytes(T, k, E, R)
+        assert lib.ep_layout_init(ctypes.byref(c), T, k, E, R, 64, fake, n) == 0
+        assert c.work > c.totals and c.work % 16 == 0
+        nb = min(-(-(T * k) // 256), 256)
+        rows = ((E + R + 1) // 2 + 3) // 4 * 4
+        pref = (E + R + 3) // 4 * 4
+        need = 4 * (16 + nb * rows + (nb + 1) * pref)
+        assert c.work + need <= fake + n
