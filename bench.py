@@ -175,6 +175,18 @@ def sources_hash(kernel):
     return h.hexdigest()[:16]
 
 
+def layout_auto_engine(T, k):
+    """The layout schedule the automatic choice takes for T tokens x top-k
+    (label for the traffic lookup only): the warp-chunk cluster while a
+    cluster of up to 16 CTAs covers the batch in at most four passes of 32
+    warps of floor(32/k)-token chunks, else the grid schedule.  The
+    shared-memory limit of the warp-chunk table is not mirrored here."""
+    csize = max(1, min(16, (T * k + 2047) // 2048))
+    tpc = -(-T // csize)
+    tpw = max(1, 32 // k)
+    return "warp_chunks" if -(-tpc // tpw) <= 4 * 32 else "grid"
+
+
 def committed_traffic(kernel, workload, engine=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel source (and copy engine); otherwise None."""
@@ -824,7 +836,7 @@ def run_epx(args):
               (args.dispatch_variant == 0 and T >= 1024) else "vec",
               "combine_reduce": "warp_per_token" if args.combine_variant == 1 else "split",
               "layout": {1: "warp_chunks", 2: "count_matrix", 3: "grid"}.get(
-                  args.layout_variant, "grid" if T * k > 8192 else "warp_chunks")}
+                  args.layout_variant, layout_auto_engine(T, k))}
     traffic = committed_traffic(dom, args.workload, engine.get(dom))
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
