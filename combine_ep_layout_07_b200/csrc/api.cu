@@ -234,6 +234,7 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     p.R = L->R;
     p.V = H / 8;
     p.inv_epr = 1.0f / (float)(L->E / L->R);
+    p.inv_k = 1.0f / (float)L->k;
     p.recv = static_cast<uint4 *>(recv);
     p.recv_cap = recv_cap;
     p.expanded = static_cast<uint4 *>(expanded);

@@ -216,6 +216,10 @@ std::atomic<long long> dispatch_first_wait_limit{-1};
 namespace {
 
 // One warp per CTA; the CTA handles chunk blockIdx.x (vpc vectors) of token t.
+// With prefetch, the bulk load of the first token's chunk of x is issued
+// before the wait (if the token has a route), so that the first wave of
+// CTAs reads its rows while the layout kernel runs; the CTA always waits for
+// that load before it leaves or reuses the buffer.
 __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
 {
     extern __shared__ __align__(128) uint4 sbuf[];
@@ -223,22 +227,31 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
     __shared__ __align__(8) uint64_t bar;
     const int lane = threadIdx.x;
     if (p.early_pdl) pdl_launch_dependents();
-    if (lane == 0) mbar_init(&bar, 1);
-    __syncwarp();
-    pdl_wait_previous();
-    unsigned phase = 0;
-    bool first = true;
     const int v0 = blockIdx.x * p.vpc;
     const int nv = min(p.V, v0 + p.vpc) - v0;
     if (nv <= 0) return;
     const unsigned bytes = (unsigned)nv * 16u;
+    if (lane == 0) mbar_init(&bar, 1);
+    __syncwarp();
+    bool in_flight = false;  // a load of token blockIdx.y issued before the wait
+    if (p.prefetch && token_has_route(p, blockIdx.y)) {
+        if (lane == 0) {
+            mbar_expect_tx(&bar, bytes);
+            bulk_g2s(sbuf, p.x + (size_t)blockIdx.y * p.V + v0, bytes, &bar);
+        }
+        in_flight = true;
+    }
+    pdl_wait_previous();
+    unsigned phase = 0;
+    bool first = true;
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         const int n = build_dst_list(p, t, s_dst);
-        if (n == 0) continue;
-        if (lane == 0) {
+        if (n == 0 && !in_flight) continue;
+        if (!in_flight && lane == 0) {
             mbar_expect_tx(&bar, bytes);
             bulk_g2s(sbuf, p.x + (size_t)t * p.V + v0, bytes, &bar);
         }
+        in_flight = false;
         // the first wait of the CTA may take a shorter limit (a test setting;
         // kWaitLimit unless changed)
         const long long limit = first ? p.first_wait_limit : kWaitLimit;
@@ -251,6 +264,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(DispatchParams p)
             return;
         }
         phase ^= 1u;
+        if (n == 0) continue;  // prefetched, but every route was dropped
         for (int i = lane; i < n; i += 32) bulk_s2g(s_dst[i] + v0, sbuf, bytes);
         bulk_commit_and_wait_read();  // sbuf and s_dst are reused next token
         __syncwarp();

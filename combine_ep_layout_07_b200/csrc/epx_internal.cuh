@@ -72,7 +72,7 @@ struct DispatchParams {
     int32_t *err;
     int early_pdl;  // trigger dependents at start (grid fits in one wave)
     long long first_wait_limit;  // bulk engine: polls allowed by a CTA's first bounded wait
-    // vector engine: the previous kernel is this library's layout kernel,
+    // both engines: the previous kernel is this library's layout kernel,
     // launched for the same batch: it lets this grid start only once every
     // kernel before it has completed, so x and topk_idx (which the layout
     // does not write) may be read before this kernel's wait
@@ -90,6 +90,7 @@ struct FusedParams {
     int vpc;     // vectors per CTA chunk
     int chunks;  // CTAs per token
     float inv_epr;
+    float inv_k;  // 1.0f / k: token of flat route i = floor((i + 0.5) * inv_k)
     uint4 *recv;
     int64_t recv_cap;
     uint4 *expanded;

@@ -9,30 +9,30 @@
 // place) that the dispatch must wait for; here that chain is removed:
 //
 //  * CTA (token t, chunk c) first issues every load it needs: its token's
-//    k routes, the route indices of its first batch of tokens (one token per
-//    thread; topk_idx is a few KB and stays in L2 after the first CTA reads
-//    it) and, once the token is known to have a route, its chunk of x[t], so
-//    the DRAM latency of x overlaps the count;
+//    k routes, its chunk of x[t] and the routes of the whole batch (read
+//    coalesced into a shared-memory table of experts, one row per token,
+//    then each token's set of ranks), so the DRAM latency of x overlaps the
+//    count;
 //  * it derives its own token's rows by counting over all T*k routes.  In
 //    (expert, token, slot) order the row of route (t, j) with expert e is
 //    the number of valid routes before it:
 //        pos[t, j] = #{(t', j') : e' < e, or e' == e and t' < t}
-//                  + #{j' < j : e_{t, j'} == e}.
-//    With key K' = 2 e' + [t' >= t] and query Q = 2 e, the first term counts
-//    routes with K' <= Q, one compare per (route, slot).  Likewise a
-//    (token, rank) pair's row is the number of pairs (t', r') with r' < r,
-//    or r' == r and t' < t: popcount(M' & lowmask(r + [t' < t])) summed over
-//    tokens t', M' being t''s set of ranks.  Each thread holds one token's
-//    keys and rank set; the token's slots and ranks are the queries, four at
-//    a time, each summed over the warp by a warp reduction;
+//                  + #{j' < j : e_{t, j'} == e},
+//    i.e. the routes of token t' with e' < e + [t' < t], plus the earlier
+//    slots of t with the same expert.  Likewise a (token, rank) pair's row
+//    is the number of pairs (t', r') with r' < r + [t' < t]:
+//    popcount(M' & lowmask(r + [t' < t])) summed over tokens t', M' being
+//    t''s set of ranks.  Each thread owns one query (a slot or a rank of
+//    token t) and a subset of the tokens, so the count has no cross-lane
+//    dependency until one shuffle sum at the end;
 //  * warp 0 adds the warps' counts, and the CTA stores its chunk to every
 //    destination row; chunk 0 of token t writes pos[t, :] and recv_pos[t, :];
 //  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
 //    counts and exclusive scans, the totals and the error word.
 //
 // No CTA waits for another, so there is no grid-wide barrier.  The count
-// costs every CTA work in proportion to T*k, and at one or a few tokens the
-// single warp that holds them walks its queries alone; measured on B200 the
+// costs every CTA work in proportion to T*k, and at one or a few tokens
+// most of the CTA's threads have no token to visit; measured on B200 the
 // one launch is faster than the layout and dispatch kernels for batches of
 // a few hundred to about two thousand routes (EPX_FUSED_AUTO_MIN_ROUTES to
 // EPX_FUSED_AUTO_MAX_ROUTES), which is where the automatic choice takes it.
@@ -43,7 +43,15 @@
 namespace epx {
 namespace {
 
-constexpr int kFusedThreads = 128;
+// Threads per CTA.  Measured on B200 (amortised steps, L2 flushed): 256
+// against 128 took decode from 20.3 to 20.2 us and DP compact from 20.4 to
+// 20.3 us (tiny 6.6 -> 6.7 us); 512 was no better than 128.  The kernel is
+// bound by instruction latency (about 11 cycles per issued instruction with
+// two warps per scheduler at 128 threads), not by its loads.
+#ifndef EPX_FUSED_THREADS
+#define EPX_FUSED_THREADS 256
+#endif
+constexpr int kFusedThreads = EPX_FUSED_THREADS;
 constexpr int kFusedWarps = kFusedThreads / 32;
 
 __device__ __forceinline__ int rank_of_e(int e, float inv_epr)
@@ -203,14 +211,15 @@ __device__ void summary_cta(const FusedParams &p, uint32_t *smem)
 
 // ------------------------------------------------------------ token CTAs
 //
-// Counting: one thread per token of the batch, its k route keys in
-// registers; the own token's slots and ranks are the queries, visited by a
-// plain loop (the same query in every lane at a time): each thread counts
-// its routes against the query, a warp reduction sums the warp's tokens, and
-// the lane that owns the query keeps the running sum.  Only the loop over a
-// token's own k routes is unrolled, so the kernel's code stays small -- after
-// an L2 flush the instructions come from DRAM again, and a large unrolled
-// body stalls on instruction fetch.
+// Counting: the batch's experts sit in a shared-memory table, one row of
+// KM entries per token (INT_MAX for no route), next to each token's set of
+// ranks.  Thread (query j, subset s) -- j = tid mod KM, s = tid div KM --
+// visits the tokens u = s, s + S, ... (S = threads / KM) and counts, for slot j of its
+// own token (expert e_j), the routes of u with expert below e_j + [u < t],
+// and for the j-th rank r_j of its own token whether u reaches a rank below
+// r_j + [u < t].  Lanes of a warp with the same j are summed by shuffles,
+// the warps by warp 0.  Rows are read by all KM threads of a subset at once
+// (a shared-memory broadcast); nothing in the count waits on another lane.
 
 template <typename IdxT, int KM, int VPT>
 __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedParams p)
@@ -230,20 +239,43 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     const int b = (int)blockIdx.x - 1;
     const int t = b / p.chunks;
     const int c = b - t * p.chunks;
-    const int k = p.k, E = p.E, R = p.R;
+    const int k = p.k, E = p.E, R = p.R, T = p.T;
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
+    int *s_e = reinterpret_cast<int *>(fsmem);                       // [T][KM]
+    unsigned long long *s_m = reinterpret_cast<unsigned long long *>(s_e + T * KM);  // [T]
 
-    // the loads the count needs are issued before anything waits on one:
-    // this token's routes (one per lane; every warp reads them, so no
-    // barrier) and the first batch of route indices (one token per thread)
+    // every load is issued before anything waits on one: this token's
+    // routes (one per lane; every warp reads them, so no barrier), its chunk
+    // of x[t] and the batch's routes (coalesced, eight per thread at a time)
     long long own = -1;
     if (lane < k) own = (long long)idx[(size_t)t * k + lane];
-    long long kv[KM];
-    {
-        const int u = wid * 32 + lane;
+    const int v0 = c * p.vpc;
+    const int v1 = min(p.V, v0 + p.vpc);
+    const uint4 *src = p.x + (size_t)t * p.V;
+    uint4 val[VPT];
 #pragma unroll
-        for (int j = 0; j < KM; ++j)
-            kv[j] = (j < k && u < p.T) ? (long long)idx[(size_t)u * k + j] : -1;
+    for (int u = 0; u < VPT; ++u) {
+        const int v = v0 + tid + u * kFusedThreads;
+        if (v < v1) val[u] = ld_nc_v4(src + v);
+    }
+    const int nk = T * k;
+    for (int i0 = 0; i0 < nk; i0 += 8 * kFusedThreads) {
+        long long ev[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const int i = i0 + a * kFusedThreads + tid;
+            ev[a] = i < nk ? (long long)idx[i] : -1;
+        }
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const int i = i0 + a * kFusedThreads + tid;
+            if (i < nk) {
+                // i = u k + j; (i + 1/2) / k is at least 1/(2k) from an
+                // integer, far more than the fp32 roundings move it
+                const int u = __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), p.inv_k));
+                s_e[u * KM + (i - u * k)] = (ev[a] >= 0 && ev[a] < E) ? (int)ev[a] : 0x7fffffff;
+            }
+        }
     }
     const int e_mine = (own >= 0 && own < E) ? (int)own : -1;
     const int r_mine = e_mine >= 0 ? rank_of_e(e_mine, p.inv_epr) : -1;
@@ -257,87 +289,60 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         }
         return;
     }
-
-    // this CTA's chunk of x[t], in flight while the rows are counted
-    const int v0 = c * p.vpc;
-    const int v1 = min(p.V, v0 + p.vpc);
-    const uint4 *src = p.x + (size_t)t * p.V;
-    uint4 val[VPT];
-#pragma unroll
-    for (int u = 0; u < VPT; ++u) {
-        const int v = v0 + tid + u * kFusedThreads;
-        if (v < v1) val[u] = ld_nc_v4(src + v);
-    }
-
-    // queries: slot j's key 2 e_j (lane j); the q-th rank of the token in
-    // increasing order (lane q)
-    const int nr = __popcll((long long)m_own);
-    const int q_slot = e_mine >= 0 ? 2 * e_mine : -1;
-    int q_rank = 0;
-    if (lane < nr) {
-        unsigned long long m = m_own;
-        for (int i = 0; i < lane; ++i) m &= m - 1ull;
-        q_rank = __ffsll((long long)m) - 1;
-    }
-
-    int acc_slot = 0, acc_rank = 0;
-    for (int u0 = wid * 32; u0 < p.T; u0 += kFusedThreads) {
-        const int u = u0 + lane;
-        const int after = u >= t;
-        // this thread's token: k route keys 2 e + [u >= t] (INT_MAX for no
-        // route) and its set of ranks
-        int key[KM];
+    __syncthreads();  // s_e complete
+    // every token's set of ranks
+    for (int u = tid; u < T; u += kFusedThreads) {
         unsigned long long m = 0ull;
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
-            key[j] = 0x7fffffff;
-            if (kv[j] >= 0 && kv[j] < E) {
-                key[j] = 2 * (int)kv[j] + after;
-                m |= 1ull << rank_of_e((int)kv[j], p.inv_epr);
-            }
+            const int e = s_e[u * KM + j];
+            if (j < k && e != 0x7fffffff) m |= 1ull << rank_of_e(e, p.inv_epr);
         }
-        // the next batch's indices, in flight while this one is counted
-        {
-            const int un = u + kFusedThreads;
-#pragma unroll
-            for (int j = 0; j < KM; ++j)
-                kv[j] = (j < k && un < p.T) ? (long long)idx[(size_t)un * k + j] : -1;
-        }
-        // four queries at a time: their shuffles, compares and warp
-        // reductions are independent, so their latencies overlap
-        for (int j0 = 0; j0 < k; j0 += 4) {
-            int n[4];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                // lanes >= k hold -1, which no key is below
-                const int qj = __shfl_sync(kFull, q_slot, (j0 + a) & 31);
-                n[a] = 0;
-#pragma unroll
-                for (int i = 0; i < KM; ++i) n[a] += key[i] <= qj;
-            }
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const int sum = __reduce_add_sync(kFull, n[a]);
-                if (lane == j0 + a) acc_slot += sum;
-            }
-        }
-        const int before = 1 - after;
-        for (int q0 = 0; q0 < nr; q0 += 4) {
-            int n[4];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const int rq = __shfl_sync(kFull, q_rank, (q0 + a) & 31);
-                n[a] = q0 + a < nr ? __popcll((long long)(m & lowmask64(rq + before))) : 0;
-            }
-#pragma unroll
-            for (int a = 0; a < 4; ++a) {
-                const int sum = __reduce_add_sync(kFull, n[a]);
-                if (lane == q0 + a) acc_rank += sum;
-            }
-        }
+        s_m[u] = m;
     }
-    s_part[wid][lane] = acc_slot;
-    s_part[wid][32 + lane] = acc_rank;
+    __syncthreads();  // s_m complete
+
+    // this thread's queries: slot j of token t (expert eq, -1 for none) and
+    // the j-th smallest rank of token t (rq, -1 for none)
+    const int j = tid & (KM - 1);
+    const int sub = tid / KM;
+    constexpr int kSubsets = kFusedThreads / KM;
+    int eq = -1;
+    if (j < k) {
+        const int e = s_e[t * KM + j];
+        eq = e == 0x7fffffff ? -1 : e;
+    }
+    const int nr = __popcll((long long)m_own);
+    int rq = -1;
+    if (j < nr) {
+        unsigned long long m = m_own;
+        for (int i = 0; i < j; ++i) m &= m - 1ull;
+        rq = __ffsll((long long)m) - 1;
+    }
+    int n_slot = 0, n_rank = 0;
+#pragma unroll 2
+    for (int u = sub; u < T; u += kSubsets) {
+        const int bt = u < t;
+        const int thr = eq + bt;  // eq = -1: no valid expert is below -1 + bt
+        const int4 *row = reinterpret_cast<const int4 *>(s_e + u * KM);
+#pragma unroll
+        for (int q = 0; q < KM / 4; ++q) {
+            const int4 w = row[q];
+            // entries beyond k are never written: mask them by index
+            n_slot += (4 * q + 0 < k && w.x < thr) + (4 * q + 1 < k && w.y < thr) +
+                      (4 * q + 2 < k && w.z < thr) + (4 * q + 3 < k && w.w < thr);
+        }
+        if (rq >= 0) n_rank += __popcll((long long)(s_m[u] & lowmask64(rq + bt)));
+    }
+#pragma unroll
+    for (int off = KM; off < 32; off <<= 1) {
+        n_slot += __shfl_xor_sync(kFull, n_slot, off);
+        n_rank += __shfl_xor_sync(kFull, n_rank, off);
+    }
+    if (lane < KM) {
+        s_part[wid][lane] = n_slot;
+        s_part[wid][32 + lane] = n_rank;
+    }
     __syncthreads();
 
     // warp 0: rows of the token's routes and pairs, destination list
@@ -394,13 +399,25 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
 
 namespace {
 
+template <typename K>
+cudaError_t launch_smem(K kernel, const FusedParams &p, dim3 grid, size_t smem, cudaStream_t s)
+{
+    // above the default 48 KB (one route per token at the largest batches)
+    if (smem > 48 * 1024) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(kernel, grid, dim3(kFusedThreads), smem, s, p);
+}
+
 template <typename IdxT, int KM>
 cudaError_t launch_km(const FusedParams &p, int vpt, dim3 grid, size_t smem, cudaStream_t s)
 {
     switch (vpt) {
-    case 1: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 1>, grid, dim3(kFusedThreads), smem, s, p);
-    case 2: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 2>, grid, dim3(kFusedThreads), smem, s, p);
-    default: return launch_pdl(layout_dispatch_kernel<IdxT, KM, 4>, grid, dim3(kFusedThreads), smem, s, p);
+    case 1: return launch_smem(layout_dispatch_kernel<IdxT, KM, 1>, p, grid, smem, s);
+    case 2: return launch_smem(layout_dispatch_kernel<IdxT, KM, 2>, p, grid, smem, s);
+    default: return launch_smem(layout_dispatch_kernel<IdxT, KM, 4>, p, grid, smem, s);
     }
 }
 
@@ -448,9 +465,13 @@ cudaError_t launch_layout_dispatch(const FusedParams &p0, int idx_bits, cudaStre
     p.chunks = chunks;
     const long long ctas = 1 + (long long)p.T * chunks;
     if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;
-    // summary CTA: packed expert counts, rank counts, flags, scan scratch
-    const size_t smem = (((size_t)(p.E + 1) / 2 + p.R + 2 + 1) & ~(size_t)1) * 4 +
-                        (kFusedWarps + 1) * 8;
+    // summary CTA: packed expert counts, rank counts, flags, scan scratch;
+    // token CTAs: the batch's experts (rows padded to KM entries) and rank sets
+    const size_t km = p.k <= 4 ? 4 : p.k <= 8 ? 8 : p.k <= 16 ? 16 : 32;
+    const size_t smem_sum = (((size_t)(p.E + 1) / 2 + p.R + 2 + 1) & ~(size_t)1) * 4 +
+                            (kFusedWarps + 1) * 8;
+    const size_t smem_tok = (size_t)p.T * km * 4 + (size_t)p.T * 8;
+    const size_t smem = smem_sum > smem_tok ? smem_sum : smem_tok;
     p.early_pdl = early_trigger(ctas);
     const dim3 grid((unsigned)ctas);
     return idx_bits == 64 ? launch_t<long long>(p, vpt, grid, smem, s)

@@ -114,24 +114,35 @@ def test_fused_empty_batch():
     assert lay.off_e.cpu().sum().item() == 0 and lay.cnt_r.cpu().sum().item() == 0
 
 
-def test_fused_capacity_overflow_flagged_not_written():
-    wl = _random_wl(T=64, H=64, E=16, R=4, k=4, seed=10)
+@pytest.mark.parametrize("T,variant", [(64, 1), (64, 2), (1536, 2)],
+                         ids=["one_launch", "paired_vec", "paired_bulk"])
+@pytest.mark.parametrize("which", ["recv", "expanded", "both"])
+def test_fused_capacity_overflow_flagged_not_written(T, variant, which):
+    # "both": tokens whose every row lies beyond the capacities have their
+    # chunk of x loaded before the dispatch's wait (paired path) and nothing
+    # to write
+    wl = _random_wl(T=T, H=64, E=16, R=4, k=4, seed=10)
     o = oracle.run_all(wl)
     x, idx, _ = gpu_inputs(wl)
-    for which in ("recv", "expanded"):
-        cap = 10
-        canary = torch.full((cap + 4, 64), 7, dtype=torch.int16, device="cuda")
-        small = canary[:cap].view(torch.bfloat16)
-        full_r = torch.empty((64 * 4, 64), dtype=torch.bfloat16, device="cuda")
-        full_e = torch.empty((64 * 4, 64), dtype=torch.bfloat16, device="cuda")
-        recv, ex = (small, full_e) if which == "recv" else (full_r, small)
-        lay, _, _ = epx.layout_dispatch_expand(idx, x, 16, 4, recv=recv, expanded=ex, variant=1)
-        t = epx.read_totals(lay, raise_on_error=False)
-        assert t["status"] == 3 and (t["dev_err"] & (2 if which == "recv" else 4))
-        want = o["recv"] if which == "recv" else o["expanded"]
-        np.testing.assert_array_equal(torch_to_bits(small), want[:cap])
-        assert torch.all(canary[cap:] == 7)
-        assert_layout_equal(lay, o["layout"])
+    cap = 10
+    canary = {n: torch.full((cap + 4, 64), 7, dtype=torch.int16, device="cuda")
+              for n in ("recv", "expanded")}
+    bufs = {n: (canary[n][:cap].view(torch.bfloat16) if which in (n, "both") else
+                torch.empty((T * 4, 64), dtype=torch.bfloat16, device="cuda"))
+            for n in ("recv", "expanded")}
+    lay, _, _ = epx.layout_dispatch_expand(idx, x, 16, 4, recv=bufs["recv"],
+                                           expanded=bufs["expanded"], variant=variant)
+    t = epx.read_totals(lay, raise_on_error=False)
+    want_err = {"recv": 2, "expanded": 4, "both": 6}[which]
+    assert t["status"] == 3 and (t["dev_err"] & want_err) == want_err
+    for n in ("recv", "expanded"):
+        if which in (n, "both"):
+            np.testing.assert_array_equal(torch_to_bits(bufs[n]), o[n][:cap])
+            assert torch.all(canary[n][cap:] == 7)
+        else:
+            rows = o["layout"]["N_recv" if n == "recv" else "N_route"]
+            np.testing.assert_array_equal(torch_to_bits(bufs[n][:rows]), o[n])
+    assert_layout_equal(lay, o["layout"])
 
 
 def test_fused_guard_bands_untouched():
