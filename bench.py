@@ -436,10 +436,9 @@ def step_mode(args, T, k):
     ep_layout_dispatch_expand variant 1), "paired" (ep_layout_dispatch_expand
     variant 2: the layout and a dispatch that reads x before its wait, one
     call), or "separate" (ep_layout, then ep_dispatch_expand).  Automatic: the
-    library's choice for small batches (one launch from
-    EPX_FUSED_AUTO_MIN_ROUTES to EPX_FUSED_AUTO_MAX_ROUTES routes, paired
-    below), separate calls above (so that the per-kernel split keeps the
-    layout and the dispatch apart)."""
+    library's choice, i.e. what ep_layout_dispatch_expand does with variant 0
+    (one launch from EPX_FUSED_AUTO_MIN_ROUTES to EPX_FUSED_AUTO_MAX_ROUTES
+    routes, paired elsewhere)."""
     if getattr(args, "no_expand", False) or args.step_calls == "separate":
         return "separate"
     if args.step_calls == "fused":
@@ -449,7 +448,7 @@ def step_mode(args, T, k):
     from combine_ep_layout_07_b200 import epx
     if epx.FUSED_AUTO_MIN_ROUTES <= T * k <= epx.FUSED_AUTO_MAX_ROUTES:
         return "one_launch"
-    return "paired" if T * k < epx.FUSED_AUTO_MIN_ROUTES else "separate"
+    return "paired"
 
 
 def workload_config(wl, args, lay_totals, flush_desc=None, mode="separate"):
@@ -498,6 +497,19 @@ class Step:
         self.src = src = (torch.empty((lay.exp_cap,), dtype=torch.int32, device=dev)
                           if no_expand else None)
         self.mode, self.no_expand = mode, no_expand
+        self.args = args
+        self.calls = self.calls_for(mode)
+        self.names = [n for n, _ in self.calls]
+        # kernels per step: the paired call launches the layout and the dispatch
+        self.n_kernels = len(self.calls) + (1 if mode == "paired" else 0)
+
+    def calls_for(self, mode):
+        """The step's calls in `mode` on this step's buffers."""
+        epx, args, wl = self.epx, self.args, self.wl
+        E, R = wl["E"], wl["R"]
+        idx, x, w, lay = self.idx, self.x, self.w, self.lay
+        recv, expanded, y, out, part, src = (self.recv, self.expanded, self.y, self.out,
+                                             self.part, self.src)
         calls = []
         if mode in ("one_launch", "paired"):
             v = 1 if mode == "one_launch" else 2
@@ -506,7 +518,7 @@ class Step:
         else:
             calls.append(("layout", lambda st: epx.layout(
                 idx, E, R, out=lay, variant=args.layout_variant, stream=st)))
-            if no_expand:
+            if self.no_expand:
                 calls.append(("dispatch", lambda st: epx.dispatch(x, lay, recv=recv, stream=st)))
                 calls.append(("expand_index", lambda st: epx.expand_index(lay, src=src,
                                                                           stream=st)))
@@ -522,8 +534,7 @@ class Step:
                 y, w, lay, partial=part, stream=st)))
             calls.append(("combine_epilogue", lambda st: epx.combine_epilogue(
                 part, lay, out=out, stream=st)))
-        self.calls = calls
-        self.names = [n for n, _ in calls]
+        return calls
 
     def prepare(self, stream):
         """The stand-in expert's output that combine reads (made once,
@@ -537,13 +548,14 @@ class Step:
         self.tot = epx.read_totals(self.lay, stream=stream)
         return self.tot
 
-    def launch(self, st, events=None):
-        for i, (_, fn) in enumerate(self.calls):
+    def launch(self, st, events=None, calls=None):
+        calls = self.calls if calls is None else calls
+        for i, (_, fn) in enumerate(calls):
             if events is not None:
                 events[i].record(st)
             fn(st)
         if events is not None:
-            events[len(self.calls)].record(st)
+            events[len(calls)].record(st)
 
 
 class L2Flush:
@@ -725,14 +737,14 @@ def measure_small(torch, epx, wlmod, args, dev, stream, peak, flush, floors):
                       wl["R"], args.idx_bits // 8, fused=mode)
         kern = {n: statistics.median([r[i] - (r[i - 1] if i else 0.0) for r in rec_k]) * 1e3
                 for i, n in enumerate(st.names)}
-        floor = floors.get(len(st.calls))
+        floor = floors.get(st.n_kernels)
         res[name] = {
             "workload": DESCRIBE[name], "T_real": int(tot["T_real"]),
             "step_us_amortized": am, "step_us": stats,
             "tokens_per_s": tot["T_real"] / (am["median"] / 1e6),
             "alg_bytes": b["total"],
             "hbm_frac": b["total"] / (am["median"] / 1e6) / 1e9 / peak,
-            "launches": len(st.calls), "calls": st.names,
+            "launches": st.n_kernels, "calls": st.names,
             "kernel_us_median_split": kern,
             "x_floor": (am["median"] / floor["amortized"]["median"]) if floor else None,
         }
@@ -798,6 +810,20 @@ def run_epx(args):
     amortized = None
     if do_flush and not args.eager:
         amortized = time_amortized(torch, step.launch, stream, dev, l2flush)
+    # the paired call's two kernels cannot be split by events without
+    # undoing their overlap: the per-kernel times of the roofline come from a
+    # split pass of the same step as separate calls (layout, dispatch_expand)
+    sep_ms = sep_bytes = None
+    if mode == "paired" and not args.eager:
+        sep_calls = step.calls_for("separate")
+        _, rec_sep, _ = time_step(
+            torch, lambda st, ev=None: step.launch(st, ev, sep_calls), len(sep_calls), stream,
+            dev, args.steps, args.warmup, flush=l2flush if do_flush else None, split=True,
+            pg=pg)
+        sep_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_sep]
+                  for i, (n, _) in enumerate(sep_calls)}
+        sep_bytes = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
+                              args.idx_bits // 8, fused="separate")
     names = step.names
     k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)
@@ -809,25 +835,39 @@ def run_epx(args):
 
     peak, peak_kind = load_peaks()
     # ---- latency floor and the small-batch workloads, same run, same protocol
-    floors, small = {}, None
+    floors, small, small_clocks = {}, None, None
     if args.small_steps > 0 and rank == 0:
+        # clocks sampled over this phase too: a latency-bound step follows the
+        # SM clock, which may differ from the headline's timed region
+        sampler2 = ClockSampler(gpu_uuid(torch, local))
+        sampler2.start()
+        s_lo = time.time()
         n_floor = max(3, min(args.small_steps, 1000))
         for n in (2, 3):
             floors[n] = time_floor(torch, epx, stream, dev, n, n_floor, max(3, args.warmup),
                                    l2flush)
         small = measure_small(torch, epx, wlmod, args, dev, stream, peak, l2flush, floors)
+        s_hi = time.time()
+        sampler2.stop()
+        small_clocks = sampler2.summary(s_lo, s_hi)
 
     if rank != 0:
         finish(pg)
         return 0
 
-    kernels = {}
-    for name, ms in k_ms.items():
-        avg_s = statistics.fmean(ms) / 1e3
-        gbs = bytes_[name] / avg_s / 1e9
-        kernels[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
-                         "alg_bytes": bytes_[name], "gbs": gbs, "frac": gbs / peak}
-    dom = max(kernels, key=lambda n: kernels[n]["us"])
+    def kernel_stats(ms_by_name, nbytes):
+        out = {}
+        for name, ms in ms_by_name.items():
+            avg_s = statistics.fmean(ms) / 1e3
+            gbs = nbytes[name] / avg_s / 1e9
+            out[name] = {"us": avg_s * 1e6, "us_median": statistics.median(ms) * 1e3,
+                         "alg_bytes": nbytes[name], "gbs": gbs, "frac": gbs / peak}
+        return out
+
+    kernels = kernel_stats(k_ms, bytes_)
+    kernels_sep = kernel_stats(sep_ms, sep_bytes) if sep_ms else None
+    roof_k = kernels_sep or kernels
+    dom = max(roof_k, key=lambda n: roof_k[n]["us"])
     engine = {"dispatch": "recv_only", "expand_index": "gather_index",
               "combine_local": "two_stage_" + str(args.two_stage),
               "combine_epilogue": "two_stage_" + str(args.two_stage),
@@ -838,8 +878,11 @@ def run_epx(args):
               "layout": {1: "warp_chunks", 2: "count_matrix", 3: "grid"}.get(
                   args.layout_variant, layout_auto_engine(T, k))}
     traffic = committed_traffic(dom, args.workload, engine.get(dom))
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
-                "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak,
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": roof_k[dom]["gbs"], "peak": peak,
+                "unit": "GB/s", "frac": roof_k[dom]["gbs"] / peak,
+                "timed_in": ("split pass of the step as separate calls (the paired call's "
+                             "kernels are not split by events)") if kernels_sep else
+                "split pass of the step's calls",
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind ==
                 "measured" else "fallback 6.65 TB/s",
                 "traffic": traffic}
@@ -855,7 +898,8 @@ def run_epx(args):
         "step_us": step_stats(step_ms),
         **({"step_us_amortized": amortized} if amortized else {}),
         "kernels": kernels,
-        "gpu_launches": len(step.calls) * args.steps,
+        **({"kernels_separate_calls": kernels_sep} if kernels_sep else {}),
+        "gpu_launches": step.n_kernels * args.steps,
         **({"consumer": consumer} if consumer else {}),
         "e2e": e2e,
     }
@@ -867,6 +911,7 @@ def run_epx(args):
             for n, v in floors.items()}
     if small:
         line["small_batch"] = small
+        line["small_batch_clocks"] = small_clocks
     if sampler:
         line["clocks"] = sampler.summary(t_lo, t_hi)
     if world == 1 and not args.no_cpu_baseline:

@@ -206,9 +206,8 @@ ep_status_t ep_layout_dispatch_expand_variant(const void *topk_idx, const ep_lay
     if (L->T > 0 && (!aligned(x, 16) || !aligned(recv, 16) || !aligned(expanded, 16)))
         return EP_ERR_MISALIGNED;
     const long long routes = (long long)L->T * L->k;
-    // automatic: one launch where it was measured faster on B200 (each CTA's
-    // count over all routes stays cheap, and there are tokens enough for the
-    // count to spread over the CTA's warps), else the layout and dispatch
+    // automatic: one launch where it was measured faster on B200 (while each
+    // CTA's count over all routes stays cheap), else the layout and dispatch
     // kernels
     const bool automatic = variant == 0;
     if (automatic)

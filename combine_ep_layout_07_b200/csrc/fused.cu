@@ -31,10 +31,9 @@
 //    counts and exclusive scans, the totals and the error word.
 //
 // No CTA waits for another, so there is no grid-wide barrier.  The count
-// costs every CTA work in proportion to T*k, and at one or a few tokens
-// most of the CTA's threads have no token to visit; measured on B200 the
-// one launch is faster than the layout and dispatch kernels for batches of
-// a few hundred to about two thousand routes (EPX_FUSED_AUTO_MIN_ROUTES to
+// costs every CTA work in proportion to T*k; measured on B200 the one
+// launch is faster than the layout and dispatch kernels from one token up
+// to about two thousand routes (EPX_FUSED_AUTO_MIN_ROUTES to
 // EPX_FUSED_AUTO_MAX_ROUTES), which is where the automatic choice takes it.
 // Rows beyond a caller's capacity are skipped; the summary CTA flags them
 // (a row beyond the capacity exists exactly when the total exceeds it).

@@ -33,7 +33,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libepx.so")
 MAX_TOPK, MAX_RANKS, MAX_EXPERTS = 32, 64, 4096
 NOALLOC_SCRATCH_BYTES = 64 << 20  # EPX_NOALLOC_SCRATCH_BYTES
 FUSED_MAX_ROUTES = 4096           # EPX_FUSED_MAX_ROUTES
-FUSED_AUTO_MIN_ROUTES = 512       # EPX_FUSED_AUTO_MIN_ROUTES
+FUSED_AUTO_MIN_ROUTES = 1         # EPX_FUSED_AUTO_MIN_ROUTES
 FUSED_AUTO_MAX_ROUTES = 2048      # EPX_FUSED_AUTO_MAX_ROUTES
 
 EP_OK = 0

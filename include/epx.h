@@ -153,9 +153,10 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
  * followed by ep_dispatch_expand with the same arguments (every array of *L,
  * recv, expanded and the error word).  For small batches (T*k up to
  * EPX_FUSED_MAX_ROUTES) it can run as ONE launch: every CTA derives its own
- * token's rows by counting over all routes (one thread per token, the
- * token's slots and ranks as queries) while its chunk of x is in flight, so
- * nothing waits for a separate layout kernel.  Otherwise it runs the layout
+ * token's rows by counting over all routes (the batch's experts in a
+ * shared-memory table, one thread per query of the token: a slot or a rank)
+ * while its chunk of x is in flight, so nothing waits for a separate layout
+ * kernel.  Otherwise it runs the layout
  * kernel and the dispatch kernel back to back; since the layout kernel lets
  * its successor start only once every earlier kernel on the stream has
  * completed, the dispatch launched here reads topk_idx and its first chunk
@@ -167,10 +168,11 @@ ep_status_t ep_layout_variant(const void *topk_idx, const ep_layout_t *L,
  * (EP_DEVERR_RECV_CAP / EP_DEVERR_EXP_CAP) as in ep_dispatch_expand.
  */
 #define EPX_FUSED_MAX_ROUTES 4096
-/* variant 0 takes one launch for T*k in [MIN, MAX]: measured on B200, below
- * it the one warp that holds a handful of tokens walks the queries alone,
- * above it every CTA's count over all routes outweighs the launch saved */
-#define EPX_FUSED_AUTO_MIN_ROUTES 512
+/* variant 0 takes one launch for T*k in [MIN, MAX]: measured on B200 it is
+ * faster from one token (16 routes: 7.7 against 8.6 us per step) to 2048
+ * routes; above that every CTA's count over all routes outweighs the launch
+ * saved (2560 routes: 42.8 against 42.0 us) */
+#define EPX_FUSED_AUTO_MIN_ROUTES 1
 #define EPX_FUSED_AUTO_MAX_ROUTES 2048
 ep_status_t ep_layout_dispatch_expand(const void *topk_idx, const ep_layout_t *L,
                                       const void *x, int32_t H, void *recv,

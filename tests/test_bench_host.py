@@ -45,14 +45,14 @@ def test_step_call_choice_follows_the_library_threshold():
     a = bench.parse_args([])
     m = lambda T, k, argv=(): bench.step_mode(bench.parse_args(list(argv)), T, k)  # noqa: E731
     assert m(128, 8) == "one_launch" and m(128, 4) == "one_launch"
-    assert m(4096, 8) == "separate" and m(1, 16) == "paired"
+    assert m(4096, 8) == "paired"
     assert m(epx.FUSED_AUTO_MAX_ROUTES // 8, 8) == "one_launch"
-    assert m(epx.FUSED_AUTO_MAX_ROUTES // 8 + 1, 8) == "separate"
-    assert m(epx.FUSED_AUTO_MIN_ROUTES // 8, 8) == "one_launch"
-    assert m(epx.FUSED_AUTO_MIN_ROUTES // 8 - 1, 8) == "paired"
+    assert m(epx.FUSED_AUTO_MAX_ROUTES // 8 + 1, 8) == "paired"
+    assert m(1, 16) == "one_launch" and m(1, 1) == "one_launch"
+    assert m(0, 8) == "paired"          # empty batch: below the one-launch range
     assert m(128, 8, ["--step-calls", "separate"]) == "separate"
     assert m(960, 8, ["--step-calls", "fused"]) == "one_launch"
-    assert m(4096, 8, ["--step-calls", "paired"]) == "paired"
+    assert m(4096, 8, ["--step-calls", "separate"]) == "separate"
     assert m(128, 8, ["--no-expand"]) == "separate"
     assert a.step_calls == "auto"
 
