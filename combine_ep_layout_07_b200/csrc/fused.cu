@@ -11,8 +11,8 @@
 //  * CTA (token t, chunk c) first issues every load it needs: its token's
 //    k routes, its chunk of x[t] and the routes of the whole batch (read
 //    coalesced into a shared-memory table of experts, one row per token,
-//    then each token's set of ranks), so the DRAM latency of x overlaps the
-//    count;
+//    with each token's set of ranks OR-ed together on the way), so the DRAM
+//    latency of x overlaps the count;
 //  * it derives its own token's rows by counting over all T*k routes.  In
 //    (expert, token, slot) order the row of route (t, j) with expert e is
 //    the number of valid routes before it:
@@ -25,8 +25,11 @@
 //    t''s set of ranks.  Each thread owns one query (a slot or a rank of
 //    token t) and a subset of the tokens, so the count has no cross-lane
 //    dependency until one shuffle sum at the end;
-//  * warp 0 adds the warps' counts, and the CTA stores its chunk to every
-//    destination row; chunk 0 of token t writes pos[t, :] and recv_pos[t, :];
+//  * warp 0 adds the warps' counts and lists the destination rows; the CTA
+//    stores its chunk (staged in shared memory) to every destination row,
+//    the (row, vector) pairs spread over all threads so that a chunk of a
+//    few vectors still uses the whole CTA; chunk 0 of token t writes
+//    pos[t, :] and recv_pos[t, :];
 //  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
 //    counts and exclusive scans, the totals and the error word.
 //
@@ -226,6 +229,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     extern __shared__ __align__(16) uint32_t fsmem[];
     __shared__ int s_part[kFusedWarps][64];  // per warp: [0, 32) slot counts, [32, 64) rank counts
     __shared__ int s_rrow[32];
+    __shared__ int s_rq[64];                 // the token's ranks in increasing order
     __shared__ uint4 *s_dst[64];
     __shared__ int s_n;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -240,8 +244,10 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     const int c = b - t * p.chunks;
     const int k = p.k, E = p.E, R = p.R, T = p.T;
     const IdxT *idx = static_cast<const IdxT *>(p.idx);
-    int *s_e = reinterpret_cast<int *>(fsmem);                       // [T][KM]
-    unsigned long long *s_m = reinterpret_cast<unsigned long long *>(s_e + T * KM);  // [T]
+    // shared memory: the chunk of x[t] [vpc], the experts [T][KM], the rank sets [T]
+    uint4 *s_x = reinterpret_cast<uint4 *>(fsmem);
+    int *s_e = reinterpret_cast<int *>(s_x + p.vpc);
+    unsigned long long *s_m = reinterpret_cast<unsigned long long *>(s_e + T * KM);
 
     // every load is issued before anything waits on one: this token's
     // routes (one per lane; every warp reads them, so no barrier), its chunk
@@ -249,14 +255,22 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     long long own = -1;
     if (lane < k) own = (long long)idx[(size_t)t * k + lane];
     const int v0 = c * p.vpc;
-    const int v1 = min(p.V, v0 + p.vpc);
-    const uint4 *src = p.x + (size_t)t * p.V;
+    const int nv = min(p.V, v0 + p.vpc) - v0;
+    const uint4 *src = p.x + (size_t)t * p.V + v0;
     uint4 val[VPT];
 #pragma unroll
     for (int u = 0; u < VPT; ++u) {
-        const int v = v0 + tid + u * kFusedThreads;
-        if (v < v1) val[u] = ld_nc_v4(src + v);
+        const int v = tid + u * kFusedThreads;
+        if (v < nv) val[u] = ld_nc_v4(src + v);
     }
+    // the table: expert of route i = u k + j at s_e[u KM + j] (INT_MAX for
+    // no route), and token u's set of ranks.  When k divides 32 a token's
+    // routes sit in k aligned lanes of one warp load, and an OR over those
+    // lanes (shuffles) gives the set; otherwise each route ORs its rank bit
+    // in with a 32-bit shared atomic (64-bit ones were measured slow)
+    const bool seg = (32 % k) == 0;
+    if (!seg)
+        for (int u = tid; u < T; u += kFusedThreads) s_m[u] = 0ull;
     const int nk = T * k;
     for (int i0 = 0; i0 < nk; i0 += 8 * kFusedThreads) {
         long long ev[8];
@@ -265,14 +279,24 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
             const int i = i0 + a * kFusedThreads + tid;
             ev[a] = i < nk ? (long long)idx[i] : -1;
         }
+        if (!seg && i0 == 0) __syncthreads();  // s_m zeroed (the loads are in flight)
 #pragma unroll
         for (int a = 0; a < 8; ++a) {
+            if (i0 + a * kFusedThreads >= nk) break;  // the same for every thread
             const int i = i0 + a * kFusedThreads + tid;
-            if (i < nk) {
-                // i = u k + j; (i + 1/2) / k is at least 1/(2k) from an
-                // integer, far more than the fp32 roundings move it
-                const int u = __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), p.inv_k));
-                s_e[u * KM + (i - u * k)] = (ev[a] >= 0 && ev[a] < E) ? (int)ev[a] : 0x7fffffff;
+            const bool ok = i < nk && ev[a] >= 0 && ev[a] < E;
+            const int r = ok ? rank_of_e((int)ev[a], p.inv_epr) : 0;
+            // i = u k + j; (i + 1/2) / k is at least 1/(2k) from an integer,
+            // far more than the fp32 roundings move it
+            const int u = __float2int_rd(__fmul_rn(__fadd_rn((float)i, 0.5f), p.inv_k));
+            const int jj = i - u * k;
+            if (i < nk) s_e[u * KM + jj] = ok ? (int)ev[a] : 0x7fffffff;
+            if (seg) {
+                unsigned long long m = ok ? 1ull << r : 0ull;
+                for (int off = 1; off < k; off <<= 1) m |= __shfl_xor_sync(kFull, m, off);
+                if (i < nk && jj == 0) s_m[u] = m;
+            } else if (ok) {
+                atomicOr(reinterpret_cast<unsigned int *>(&s_m[u]) + (r >> 5), 1u << (r & 31));
             }
         }
     }
@@ -288,18 +312,9 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         }
         return;
     }
-    __syncthreads();  // s_e complete
-    // every token's set of ranks
-    for (int u = tid; u < T; u += kFusedThreads) {
-        unsigned long long m = 0ull;
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-            const int e = s_e[u * KM + j];
-            if (j < k && e != 0x7fffffff) m |= 1ull << rank_of_e(e, p.inv_epr);
-        }
-        s_m[u] = m;
-    }
-    __syncthreads();  // s_m complete
+    for (int r = tid; r < R; r += kFusedThreads)
+        if ((m_own >> r) & 1ull) s_rq[__popcll((long long)(m_own & lowmask64(r)))] = r;
+    __syncthreads();  // s_e, s_m, s_rq complete
 
     // this thread's queries: slot j of token t (expert eq, -1 for none) and
     // the j-th smallest rank of token t (rq, -1 for none)
@@ -312,12 +327,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         eq = e == 0x7fffffff ? -1 : e;
     }
     const int nr = __popcll((long long)m_own);
-    int rq = -1;
-    if (j < nr) {
-        unsigned long long m = m_own;
-        for (int i = 0; i < j; ++i) m &= m - 1ull;
-        rq = __ffsll((long long)m) - 1;
-    }
+    const int rq = j < nr ? s_rq[j] : -1;
     int n_slot = 0, n_rank = 0;
 #pragma unroll 2
     for (int u = sub; u < T; u += kSubsets) {
@@ -342,15 +352,26 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         s_part[wid][lane] = n_slot;
         s_part[wid][32 + lane] = n_rank;
     }
+    // the chunk of x into shared memory, for the stores below
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        const int v = tid + u * kFusedThreads;
+        if (v < nv) s_x[v] = val[u];
+    }
     __syncthreads();
 
     // warp 0: rows of the token's routes and pairs, destination list
     if (wid == 0) {
         const unsigned lt = lanemask_lt();
         int dup = 0;  // earlier slots of this token with the same expert
-        for (int j = 0; j < k; ++j) {
-            const int ej = __shfl_sync(kFull, e_mine, j);
-            dup += (j < lane && ej == e_mine) ? 1 : 0;
+        {
+            const int4 *row = reinterpret_cast<const int4 *>(s_e + t * KM);
+#pragma unroll
+            for (int q = 0; q < KM / 4; ++q) {
+                const int4 w = row[q];
+                dup += (4 * q + 0 < lane && w.x == e_mine) + (4 * q + 1 < lane && w.y == e_mine) +
+                       (4 * q + 2 < lane && w.z == e_mine) + (4 * q + 3 < lane && w.w == e_mine);
+            }
         }
         int row = -1;
         if (lane < k && e_mine >= 0) {
@@ -365,11 +386,11 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
         }
         const bool ok_e = row >= 0 && (int64_t)row < p.exp_cap;
         const unsigned me = __ballot_sync(kFull, ok_e);
-        if (ok_e) s_dst[__popc(me & lt)] = p.expanded + (size_t)row * p.V;
+        if (ok_e) s_dst[__popc(me & lt)] = p.expanded + (size_t)row * p.V + v0;
         const int ne = __popc(me);
         const bool ok_r = rrow >= 0 && (int64_t)rrow < p.recv_cap;
         const unsigned mr = __ballot_sync(kFull, ok_r);
-        if (ok_r) s_dst[ne + __popc(mr & lt)] = p.recv + (size_t)rrow * p.V;
+        if (ok_r) s_dst[ne + __popc(mr & lt)] = p.recv + (size_t)rrow * p.V + v0;
         if (lane == 0) s_n = ne + __popc(mr);
         if (c == 0 && lane < k) p.pos[(size_t)t * k + lane] = row;
         __syncwarp();
@@ -383,13 +404,20 @@ __global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(FusedPar
     }
     __syncthreads();
 
-    const int n = s_n;
-    for (int i = 0; i < n; ++i) {
-        uint4 *d = s_dst[i];
-#pragma unroll
-        for (int u = 0; u < VPT; ++u) {
-            const int v = v0 + tid + u * kFusedThreads;
-            if (v < v1) st_v4(d + v, val[u]);
+    // the stores: item q = (destination i, vector v), q = i nv + v, spread
+    // over all threads (a few tokens' rows still use the whole CTA)
+    const int items = s_n * nv;
+    if (items > 0) {
+        int i = tid / nv, v = tid - (tid / nv) * nv;
+        const int si = kFusedThreads / nv, sv = kFusedThreads - si * nv;
+        for (int q = tid; q < items; q += kFusedThreads) {
+            st_v4(s_dst[i] + v, s_x[v]);
+            v += sv;
+            i += si;
+            if (v >= nv) {
+                v -= nv;
+                ++i;
+            }
         }
     }
 }
@@ -465,11 +493,12 @@ cudaError_t launch_layout_dispatch(const FusedParams &p0, int idx_bits, cudaStre
     const long long ctas = 1 + (long long)p.T * chunks;
     if (ctas > 0x7fffffffLL) return cudaErrorNotSupported;
     // summary CTA: packed expert counts, rank counts, flags, scan scratch;
-    // token CTAs: the batch's experts (rows padded to KM entries) and rank sets
+    // token CTAs: the chunk of x, the batch's experts (rows padded to KM
+    // entries) and rank sets
     const size_t km = p.k <= 4 ? 4 : p.k <= 8 ? 8 : p.k <= 16 ? 16 : 32;
     const size_t smem_sum = (((size_t)(p.E + 1) / 2 + p.R + 2 + 1) & ~(size_t)1) * 4 +
                             (kFusedWarps + 1) * 8;
-    const size_t smem_tok = (size_t)p.T * km * 4 + (size_t)p.T * 8;
+    const size_t smem_tok = (size_t)p.vpc * 16 + (size_t)p.T * km * 4 + (size_t)p.T * 8;
     const size_t smem = smem_sum > smem_tok ? smem_sum : smem_tok;
     p.early_pdl = early_trigger(ctas);
     const dim3 grid((unsigned)ctas);
