@@ -45,18 +45,17 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8])
     return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-// Warp-collective: compact token t's valid routes (k order) into
-// s_pos/s_w; returns the count on every lane.
+// Warp-collective: compact token t's valid routes (k order) into s_pos /
+// s_slot (the route's slot j); returns the count on every lane.  The
+// weights are not loaded here: the y loads that follow need only the
+// positions, so each thread reads its weights after issuing them, and the
+// weights' DRAM latency overlaps theirs.
 __device__ __forceinline__ int build_routes(const CombineParams &p, int t, int *s_pos,
-                                            float *s_w)
+                                            int *s_slot)
 {
     const int lane = threadIdx.x & 31;
     int q = -1;
-    float w = 0.f;
-    if (lane < p.k) {
-        q = p.pos[(size_t)t * p.k + lane];
-        w = p.w[(size_t)t * p.k + lane];
-    }
+    if (lane < p.k) q = p.pos[(size_t)t * p.k + lane];
     const bool over = q >= 0 && (int64_t)q >= p.y_rows;
     const bool ok = q >= 0 && !over;
     if (over) atomicOr(p.err, (int)EP_DEVERR_Y_ROWS);
@@ -64,28 +63,34 @@ __device__ __forceinline__ int build_routes(const CombineParams &p, int t, int *
     if (ok) {
         const int slot = __popc(m & lanemask_lt());
         s_pos[slot] = q;
-        s_w[slot] = w;
+        s_slot[slot] = lane;
     }
     __syncwarp();
     return __popc(m);
 }
 
-// Accumulate vector v of the n routes; G loads are kept in flight at once.
+// Accumulate vector v of token t's n routes; G loads are kept in flight at
+// once, the routes' weights read after them.
 template <int G>
 __device__ __forceinline__ uint4 reduce_vector(const CombineParams &p, const int *s_pos,
-                                               const float *s_w, int n, int v)
+                                               const int *s_slot, int t, int n, int v)
 {
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    const float *wt = p.w + (size_t)t * p.k;
     for (int i0 = 0; i0 < n; i0 += G) {
         uint4 q[G];
+        float w[G];
 #pragma unroll
         for (int u = 0; u < G; ++u)
             if (i0 + u < n) q[u] = ld_v4(p.y + (size_t)s_pos[i0 + u] * p.V + v);
 #pragma unroll
         for (int u = 0; u < G; ++u)
-            if (i0 + u < n) fma8(acc, q[u], s_w[i0 + u]);
+            if (i0 + u < n) w[u] = __ldg(wt + s_slot[i0 + u]);
+#pragma unroll
+        for (int u = 0; u < G; ++u)
+            if (i0 + u < n) fma8(acc, q[u], w[u]);
     }
     return pack8(acc);
 }
@@ -94,13 +99,13 @@ template <int G>
 __global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
 {
     __shared__ int s_pos[EPX_MAX_TOPK];
-    __shared__ float s_w[EPX_MAX_TOPK];
+    __shared__ int s_slot[EPX_MAX_TOPK];
     __shared__ int s_n;
     if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
-            int n = build_routes(p, t, s_pos, s_w);
+            int n = build_routes(p, t, s_pos, s_slot);
             if (threadIdx.x == 0) s_n = n;
         }
         __syncthreads();
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(128) combine_split_kernel(CombineParams p)
         const int v0 = blockIdx.x * p.vpc;
         const int v1 = min(p.V, v0 + p.vpc);
         for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x)
-            st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos, s_w, n, v));
+            st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos, s_slot, t, n, v));
         __syncthreads();
     }
     pdl_launch_dependents();
@@ -118,14 +123,15 @@ template <int G>
 __global__ void __launch_bounds__(128) combine_warp_per_token_kernel(CombineParams p)
 {
     __shared__ int s_pos[4][EPX_MAX_TOPK];
-    __shared__ float s_w[4][EPX_MAX_TOPK];
+    __shared__ int s_slot[4][EPX_MAX_TOPK];
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
     for (int t = blockIdx.x * 4 + wid; t < p.T; t += gridDim.x * 4) {
-        const int n = build_routes(p, t, s_pos[wid], s_w[wid]);
+        const int n = build_routes(p, t, s_pos[wid], s_slot[wid]);
         for (int v = lane; v < p.V; v += 32)
-            st_v4(p.out + (size_t)t * p.V + v, reduce_vector<G>(p, s_pos[wid], s_w[wid], n, v));
+            st_v4(p.out + (size_t)t * p.V + v,
+                  reduce_vector<G>(p, s_pos[wid], s_slot[wid], t, n, v));
         __syncwarp();
     }
     pdl_launch_dependents();
