@@ -34,6 +34,28 @@ bool layout_ok(const ep_layout_t *L)
 
 ep_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
 
+// peers[0..R) into device form; false if an entry is malformed
+bool peers_in(const ep_peer_rows_t *peers, int R, int64_t row_align, PeerRows *out,
+                     bool meta)
+{
+    for (int r = 0; r < R; ++r) {
+        const ep_peer_rows_t &e = peers[r];
+        if (e.cap < 0 || e.row0 < 0 || e.first < 0 || e.count < 0) return false;
+        if (e.cap > 0 && !e.rows) return false;
+        if (!aligned(e.rows, (size_t)row_align)) return false;
+        if (meta && ((e.meta_idx && !aligned(e.meta_idx, 4)) || (e.meta_w && !aligned(e.meta_w, 4))))
+            return false;
+        out[r].rows = static_cast<uint4 *>(e.rows);
+        out[r].meta_idx = meta ? e.meta_idx : nullptr;
+        out[r].meta_w = meta ? e.meta_w : nullptr;
+        out[r].row0 = e.row0;
+        out[r].cap = e.cap;
+        out[r].first = e.first;
+        out[r].count = e.count;
+    }
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -314,6 +336,110 @@ ep_status_t ep_route_meta(const void *topk_idx, const float *topk_weights, const
     p.rows = rows;
     p.err = L->totals + 3;
     return from_cuda(launch_route_meta(p, L->idx_bits, as_stream(stream)));
+}
+
+ep_status_t ep_dispatch_p2p(const void *x, int32_t H, const ep_layout_t *L, const void *topk_idx,
+                            const float *topk_weights, const ep_peer_rows_t *peers, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!x || !topk_idx || !topk_weights || !peers) return EP_ERR_INVALID_ARG;
+    if (!aligned(x, 16)) return EP_ERR_MISALIGNED;
+    if (!aligned(topk_idx, (size_t)L->idx_bits / 8) || !aligned(topk_weights, 4))
+        return EP_ERR_MISALIGNED;
+    P2PDispatchParams p;
+    memset(&p, 0, sizeof p);
+    if (!peers_in(peers, L->R, 16, p.peer, true)) return EP_ERR_INVALID_ARG;
+    p.x = static_cast<const uint4 *>(x);
+    p.recv_pos = L->recv_pos;
+    p.off_r = L->off_r;
+    p.idx = topk_idx;
+    p.w = topk_weights;
+    p.idx_bits = L->idx_bits;
+    p.T = L->T;
+    p.k = L->k;
+    p.E = L->E;
+    p.R = L->R;
+    p.V = H / 8;
+    p.inv_epr = 1.0f / (float)(L->E / L->R);
+    p.err = L->totals + 3;
+    return from_cuda(launch_dispatch_p2p(p, as_stream(stream)));
+}
+
+ep_status_t ep_combine_local_reduce_p2p(const void *expert_out, const float *topk_weights,
+                                        int32_t H, const ep_layout_t *L, int32_t partial_bits,
+                                        int64_t y_rows, const ep_peer_rows_t *peers, void *stream)
+{
+    if (!layout_ok(L)) return EP_ERR_INVALID_ARG;
+    if (H <= 0 || H % 8 != 0 || y_rows < 0) return EP_ERR_INVALID_ARG;
+    if (partial_bits != 32 && partial_bits != 16) return EP_ERR_INVALID_ARG;
+    if (L->T == 0) return EP_OK;
+    if (!expert_out || !topk_weights || !peers) return EP_ERR_INVALID_ARG;
+    if (!aligned(expert_out, 16) || !aligned(topk_weights, 4)) return EP_ERR_MISALIGNED;
+    LocalP2PParams p;
+    memset(&p, 0, sizeof p);
+    if (!peers_in(peers, L->R, 16, p.peer, false)) return EP_ERR_INVALID_ARG;
+    p.n_peer = L->R;
+    p.y = static_cast<const uint4 *>(expert_out);
+    p.w = topk_weights;
+    p.pos = L->pos;
+    p.recv_pos = L->recv_pos;
+    p.off_e = L->off_e;
+    p.T = L->T;
+    p.k = L->k;
+    p.R = L->R;
+    p.epr = L->E / L->R;
+    p.V = H / 8;
+    p.y_rows = y_rows;
+    p.partial = nullptr;
+    p.part_cap = INT64_MAX;  // the peers' caps are checked per row
+    p.part_bits = partial_bits;
+    p.err = L->totals + 3;
+    return from_cuda(launch_local_reduce_p2p(p, as_stream(stream)));
+}
+
+ep_status_t ep_ipc_malloc(size_t bytes, void **dev_ptr, void *handle)
+{
+    if (!dev_ptr || !handle || bytes == 0) return EP_ERR_INVALID_ARG;
+    *dev_ptr = nullptr;
+    void *ptr = nullptr;
+    if (cudaMalloc(&ptr, bytes) != cudaSuccess) return EP_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, ptr) != cudaSuccess) {
+        cudaFree(ptr);
+        return EP_ERR_CUDA;
+    }
+    static_assert(sizeof(cudaIpcMemHandle_t) <= EPX_IPC_HANDLE_BYTES, "IPC handle size");
+    memset(handle, 0, EPX_IPC_HANDLE_BYTES);
+    memcpy(handle, &h, sizeof h);
+    *dev_ptr = ptr;
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_free(void *dev_ptr)
+{
+    if (!dev_ptr) return EP_ERR_INVALID_ARG;
+    return from_cuda(cudaFree(dev_ptr));
+}
+
+ep_status_t ep_ipc_open(const void *handle, void **dev_ptr)
+{
+    if (!handle || !dev_ptr) return EP_ERR_INVALID_ARG;
+    *dev_ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof h);
+    void *ptr = nullptr;
+    if (cudaIpcOpenMemHandle(&ptr, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return EP_ERR_CUDA;
+    *dev_ptr = ptr;
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_close(void *dev_ptr)
+{
+    if (!dev_ptr) return EP_ERR_INVALID_ARG;
+    return from_cuda(cudaIpcCloseMemHandle(dev_ptr));
 }
 
 ep_status_t ep_expand_index(const ep_layout_t *L, int32_t *src_row, int64_t rows, void *stream)

@@ -17,6 +17,8 @@
 // combine: CTA (hidden chunk, token), all loads of a vector in flight.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "epx_internal.cuh"
 
 namespace epx {
@@ -55,17 +57,40 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&acc)[8])
     return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-// store 8 partial values of vector v of row d
-__device__ __forceinline__ void store_partial(const LocalParams &p, int64_t d, int v,
+// store 8 partial values of vector v of the partial row starting at `row`
+__device__ __forceinline__ void store_partial(int part_bits, char *row, int v,
                                               const float (&acc)[8])
 {
-    if (p.part_bits == 32) {
-        float4 *dst = reinterpret_cast<float4 *>(p.partial) + ((size_t)d * p.V + v) * 2;
+    if (part_bits == 32) {
+        float4 *dst = reinterpret_cast<float4 *>(row) + (size_t)v * 2;
         dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     } else {
-        reinterpret_cast<uint4 *>(p.partial)[(size_t)d * p.V + v] = pack_bf16x8(acc);
+        reinterpret_cast<uint4 *>(row)[v] = pack_bf16x8(acc);
     }
+}
+
+// Where partial row d goes: this rank's partial buffer, or (peer-memory
+// form) the entry whose range holds d; nullptr (flagged) when nowhere.
+__device__ __forceinline__ char *partial_row(const LocalParams &p, int64_t d)
+{
+    const size_t row_bytes = (size_t)p.V * 16 * (p.part_bits == 32 ? 2 : 1);
+    return static_cast<char *>(p.partial) + (size_t)d * row_bytes;
+}
+
+__device__ __forceinline__ char *partial_row(const LocalP2PParams &p, int64_t d)
+{
+    const size_t row_bytes = (size_t)p.V * 16 * (p.part_bits == 32 ? 2 : 1);
+    for (int s = 0; s < p.n_peer; ++s) {
+        const PeerRows &e = p.peer[s];
+        if (d >= e.first && d < e.first + e.count) {
+            const int64_t q = e.row0 + (d - e.first);
+            if (q < 0 || q >= e.cap) break;
+            return reinterpret_cast<char *>(e.rows) + (size_t)q * row_bytes;
+        }
+    }
+    atomicOr(p.err, (int)EP_DEVERR_RECV_CAP);
+    return nullptr;
 }
 
 // Warp 0: token t's valid routes sorted (stably) by rank into s_pos / s_w,
@@ -129,13 +154,16 @@ __device__ int build_groups(const LocalParams &p, int t, const int32_t *s_bound,
     return __popc(lm);
 }
 
-template <int G>
-__global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
+// P = LocalParams (partial rows in this rank's buffer) or LocalP2PParams
+// (each partial row stored at its source rank); the arithmetic is the same.
+template <int G, typename P>
+__global__ void __launch_bounds__(128) local_reduce_kernel(const __grid_constant__ P p)
 {
     __shared__ int32_t s_bound[EPX_MAX_RANKS + 1];
     __shared__ int s_pos[EPX_MAX_TOPK], s_rank[EPX_MAX_TOPK], s_gend[EPX_MAX_TOPK];
     __shared__ float s_w[EPX_MAX_TOPK];
     __shared__ int64_t s_grow[EPX_MAX_TOPK];
+    __shared__ char *s_gptr[EPX_MAX_TOPK];
     __shared__ int s_n, s_ng;
     if (p.early_pdl) pdl_launch_dependents();
     pdl_wait_previous();
@@ -144,6 +172,8 @@ __global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
     for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
         if (threadIdx.x < 32) {
             const int ng = build_groups(p, t, s_bound, s_pos, s_w, s_rank, s_gend, s_grow, &s_n);
+            for (int g = threadIdx.x; g < ng; g += 32)
+                s_gptr[g] = s_grow[g] >= 0 ? partial_row(p, s_grow[g]) : nullptr;
             if (threadIdx.x == 0) s_ng = ng;
         }
         __syncthreads();
@@ -166,7 +196,7 @@ __global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
                     if (i < n) {
                         fma8(acc, q[u], s_w[i]);
                         if (i + 1 == s_gend[g]) {  // last route of this rank
-                            if (s_grow[g] >= 0) store_partial(p, s_grow[g], v, acc);
+                            if (s_gptr[g]) store_partial(p.part_bits, s_gptr[g], v, acc);
 #pragma unroll
                             for (int a = 0; a < 8; ++a) acc[a] = 0.f;
                             ++g;
@@ -178,6 +208,9 @@ __global__ void __launch_bounds__(128) local_reduce_kernel(LocalParams p)
         }
         __syncthreads();
     }
+    // partial rows stored into other GPUs' memory are ordered before
+    // whatever this GPU writes next (a collective that tells their owners)
+    if constexpr (std::is_same<P, LocalP2PParams>::value) __threadfence_system();
     pdl_launch_dependents();
 }
 
@@ -284,8 +317,25 @@ cudaError_t launch_local_reduce(const LocalParams &p0, cudaStream_t s)
     const int gy = p.T < 65535 ? p.T : 65535;
     p.early_pdl = early_trigger((long long)chunks * gy);
     if (p.k > 8)
-        return launch_pdl(local_reduce_kernel<16>, dim3(chunks, gy), dim3(threads), 0, s, p);
-    return launch_pdl(local_reduce_kernel<8>, dim3(chunks, gy), dim3(threads), 0, s, p);
+        return launch_pdl(local_reduce_kernel<16, LocalParams>, dim3(chunks, gy), dim3(threads),
+                          0, s, p);
+    return launch_pdl(local_reduce_kernel<8, LocalParams>, dim3(chunks, gy), dim3(threads), 0, s,
+                      p);
+}
+
+cudaError_t launch_local_reduce_p2p(const LocalP2PParams &p0, cudaStream_t s)
+{
+    LocalP2PParams p = p0;
+    if (p.T == 0) return cudaSuccess;
+    int chunks, threads;
+    split_rows(p.T, p.V, chunks, p.vpc, threads);
+    const int gy = p.T < 65535 ? p.T : 65535;
+    p.early_pdl = early_trigger((long long)chunks * gy);
+    if (p.k > 8)
+        return launch_pdl(local_reduce_kernel<16, LocalP2PParams>, dim3(chunks, gy),
+                          dim3(threads), 0, s, p);
+    return launch_pdl(local_reduce_kernel<8, LocalP2PParams>, dim3(chunks, gy), dim3(threads), 0,
+                      s, p);
 }
 
 cudaError_t launch_epilogue(const EpilogueParams &p0, cudaStream_t s)

@@ -148,6 +148,36 @@ struct LocalParams {
     int early_pdl;  // trigger dependents at start (grid fits in one wave)
 };
 
+// A peer's buffers as the kernels see them (ep_peer_rows_t, in device form).
+struct PeerRows {
+    uint4 *rows;
+    int32_t *meta_idx;
+    float *meta_w;
+    int64_t row0, cap, first, count;
+};
+
+// local reduce whose partial rows go to other ranks' buffers
+struct LocalP2PParams : LocalParams {
+    int n_peer;
+    PeerRows peer[EPX_MAX_RANKS];
+};
+
+// dispatch whose rows go straight into the receiving ranks' buffers
+struct P2PDispatchParams {
+    const uint4 *x;
+    const int32_t *recv_pos;
+    const int32_t *off_r;
+    const void *idx;  // topk_idx [T, k], idx_bits wide
+    const float *w;   // topk_weights [T, k]
+    int idx_bits;
+    int T, k, E, R;
+    int V, vpc;
+    float inv_epr;
+    int32_t *err;
+    int early_pdl;
+    PeerRows peer[EPX_MAX_RANKS];
+};
+
 struct EpilogueParams {
     const void *partial;
     int part_bits;
@@ -206,6 +236,8 @@ cudaError_t launch_layout_dispatch(const FusedParams &p, int idx_bits, cudaStrea
 cudaError_t launch_combine(const CombineParams &p, int variant, cudaStream_t s);
 cudaError_t launch_route_meta(const MetaParams &p, int idx_bits, cudaStream_t s);
 cudaError_t launch_local_reduce(const LocalParams &p, cudaStream_t s);
+cudaError_t launch_local_reduce_p2p(const LocalP2PParams &p, cudaStream_t s);
+cudaError_t launch_dispatch_p2p(const P2PDispatchParams &p, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueParams &p, cudaStream_t s);
 cudaError_t launch_expand_index(const IndexParams &p, cudaStream_t s);
 cudaError_t launch_standin_gather(const GatherParams &p, cudaStream_t s);

@@ -30,10 +30,19 @@ order; the partials come back in each source's send order, which is the
 receive layout of its own layout, so the epilogue of the two-stage combine
 applies unchanged.
 
-The exchanges use NCCL's all-to-all (the plain transport; a kernel that
-stores rows straight into the owner's memory over NVLink, overlapped with
-the copies, is the next step and is not built here).  With no process
-group (one GPU) the exchanges are the identity and the path reduces to the
+Two transports for the rows (`transport=`):
+  "nccl" -- ep_dispatch into a send buffer, then NCCL's all-to-all (rows and
+            their routing), and the same back for the partials;
+  "p2p"  -- ep_dispatch_p2p stores every row and its routing straight into
+            the receiving GPU's buffer (device pointers to the other ranks'
+            buffers, mapped once through CUDA IPC by PeerBuffers), and
+            ep_combine_local_reduce_p2p stores every partial row straight
+            into its source's buffer; a one-word all-reduce on the stream
+            after each kernel orders the ranks (no kernel waits on another
+            GPU).  Placement and transfer are one kernel; there is no send
+            buffer and no all-to-all.
+Both give the same rows in the same places.  With no process group (one
+GPU) the exchanges are the identity and the path reduces to the
 single-GPU two-stage combine.
 """
 from __future__ import annotations
@@ -73,6 +82,108 @@ def send_plan(counts: torch.Tensor, rank: int) -> dict:
         run += v
     return dict(send_splits=send, recv_splits=recv, recv_offsets=offs,
                 n_send=sum(send), n_recv=run)
+
+
+def p2p_plan(counts: torch.Tensor, rank: int) -> dict:
+    """Where this rank's rows go under the peer-memory transport, from
+    counts[src, dst] (rows src sends to dst).
+
+    dispatch_row0[r]: first row of rank r's receive buffer that this rank
+    writes (the rows r receives from lower ranks come first); back_first[s] /
+    back_count[s]: the rows this rank received from source s ([first, first
+    + count) of its receive order), whose partials go back to s at
+    back_row0[s] = the first row of s's send block for this rank (s's blocks
+    are in destination order).  n_recv / n_send: rows this rank receives /
+    sends."""
+    c = counts.to(torch.int64).cpu()
+    if c.dim() != 2 or c.shape[0] != c.shape[1] or not (0 <= rank < c.shape[0]):
+        raise ValueError("counts must be [world, world] and rank inside it")
+    if bool((c < 0).any()):
+        raise ValueError("negative counts")
+    world = c.shape[0]
+    dispatch_row0 = [int(c[:rank, r].sum()) for r in range(world)]
+    back_first = [int(c[:s, rank].sum()) for s in range(world)]
+    back_count = [int(c[s, rank]) for s in range(world)]
+    back_row0 = [int(c[s, :rank].sum()) for s in range(world)]
+    return dict(dispatch_row0=dispatch_row0, back_first=back_first, back_count=back_count,
+                back_row0=back_row0, n_recv=int(c[:, rank].sum()), n_send=int(c[rank].sum()))
+
+
+class PeerBuffers:
+    """This rank's receive buffers (rows, routing) and partial-return buffer,
+    and every other rank's, mapped into this process: the destinations of
+    ep_dispatch_p2p and ep_combine_local_reduce_p2p.  Sized for batches of up
+    to t_max tokens per rank: a rank receives at most one row per token of
+    every rank (world * t_max rows) and gets back at most one partial per
+    (token, rank) pair it sent (t_max * min(k, world) rows).  With one rank
+    the buffers are plain local allocations."""
+
+    def __init__(self, t_max: int, H: int, k: int, pg=None, partial_dtype=torch.float32,
+                 device=None):
+        world, rank = _world(pg)
+        self.world, self.rank, self.pg = world, rank, pg
+        self.H, self.k, self.partial_dtype = H, k, partial_dtype
+        self.device = device if device is not None else torch.device(
+            "cuda", torch.cuda.current_device())
+        self.recv_cap = world * t_max
+        self.back_cap = t_max * min(k, world)
+        pbytes = 4 if partial_dtype == torch.float32 else 2
+        shapes = [("rows", (self.recv_cap, H), torch.bfloat16, 2 * H),
+                  ("meta_idx", (self.recv_cap, k), torch.int32, 4 * k),
+                  ("meta_w", (self.recv_cap, k), torch.float32, 4 * k),
+                  ("back", (self.back_cap, H), partial_dtype, pbytes * H)]
+        self._own, self._opened = [], []
+        self.local, self.peer = {}, {}
+        handles = {}
+        for name, shape, dtype, row_bytes in shapes:
+            nbytes = max(16, shape[0] * row_bytes)
+            if world == 1:
+                t = torch.empty(shape, dtype=dtype, device=self.device)
+                self.local[name] = t
+                self.peer[name] = [t]
+                continue
+            ptr, h = epx.ipc_malloc(nbytes)
+            self._own.append(ptr)
+            self.local[name] = epx.tensor_at(ptr, shape, dtype, self.device)
+            handles[name] = (ptr, h)
+        if world > 1:
+            import torch.distributed as dist
+            mine = {n: h for n, (_, h) in handles.items()}
+            gathered = [None] * world
+            dist.all_gather_object(gathered, mine, group=pg)
+            for name, _, _, _ in shapes:
+                ptrs = []
+                for r in range(world):
+                    if r == rank:
+                        ptrs.append(handles[name][0])
+                    else:
+                        p = epx.ipc_open(gathered[r][name])
+                        self._opened.append(p)
+                        ptrs.append(p)
+                self.peer[name] = ptrs
+
+    def close(self):
+        """Unmap the other ranks' buffers and free this rank's (collective:
+        every rank calls it, so no peer still writes into freed memory)."""
+        if self.world > 1:
+            import torch.distributed as dist
+            torch.cuda.synchronize(self.device)
+            dist.barrier(group=self.pg)
+        for p in self._opened:
+            epx.ipc_close(p)
+        for p in self._own:
+            epx.ipc_free(p)
+        self._opened, self._own = [], []
+
+
+def _order_ranks(pg, device):
+    """A one-word all-reduce on the current stream: every rank's kernels
+    before it (its stores into other GPUs' buffers) have completed before any
+    rank's work after it starts."""
+    if pg is None:
+        return
+    import torch.distributed as dist
+    dist.all_reduce(torch.zeros(1, dtype=torch.int32, device=device), group=pg)
 
 
 def exchange_counts(cnt_r: torch.Tensor, pg=None) -> torch.Tensor:
@@ -128,36 +239,77 @@ class Dispatched:
     layout_in: epx.Layout       # layout of the received rows (all on this rank)
     expanded: torch.Tensor      # [n_recv*k, H] received rows once per local expert
     pg: object = None
+    buffers: "PeerBuffers" = None   # peer-memory transport: where the partials go
 
 
 def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-             num_experts: int, pg=None) -> Dispatched:
+             num_experts: int, pg=None, transport: str = "nccl",
+             buffers: PeerBuffers = None) -> Dispatched:
     """Multi-GPU dispatch of this rank's tokens (x [T, H] bf16, topk_idx
     [T, k], topk_weights [T, k] fp32, all on this rank's GPU), on the current
-    stream (the one the collectives are ordered with)."""
+    stream (the one the collectives are ordered with).  transport "p2p"
+    needs `buffers` (PeerBuffers of this process group); the received rows
+    are then views of buffers.local, valid until the next dispatch."""
     world, rank = _world(pg)
     E = num_experts
     lay = epx.layout(topk_idx, E, world)
-    send = epx.dispatch(x, lay)
-    meta_idx, meta_w = epx.route_meta(topk_idx, topk_weights, lay)
-    counts = exchange_counts(lay.cnt_r, pg)          # synchronises the stream
-    plan = send_plan(counts, rank)
-    n = plan["n_send"]
-    recv_x = exchange_rows(send[:n], plan, pg)
-    recv_idx = exchange_rows(meta_idx[:n], plan, pg)
-    recv_w = exchange_rows(meta_w[:n], plan, pg)
+    if transport == "p2p":
+        if buffers is None:
+            raise ValueError("transport 'p2p' needs PeerBuffers")
+        if x.shape[0] * world > buffers.recv_cap or x.shape[1] != buffers.H:
+            raise ValueError("batch larger than the PeerBuffers were sized for")
+        counts = exchange_counts(lay.cnt_r, pg)      # synchronises the stream
+        plan = p2p_plan(counts, rank)
+        plan.update(send_plan(counts, rank))
+        if max(int(counts[:, r].sum()) for r in range(world)) > buffers.recv_cap:
+            raise ValueError("a rank receives more rows than its PeerBuffers hold")
+        peers = [epx.PeerRows(buffers.peer["rows"][r], buffers.recv_cap,
+                              row0=plan["dispatch_row0"][r],
+                              meta_idx=buffers.peer["meta_idx"][r],
+                              meta_w=buffers.peer["meta_w"][r]) for r in range(world)]
+        epx.dispatch_p2p(x, topk_idx, topk_weights, lay, peers)
+        _order_ranks(pg, x.device)
+        n = plan["n_recv"]
+        recv_x = buffers.local["rows"][:n]
+        recv_idx = buffers.local["meta_idx"][:n]
+        recv_w = buffers.local["meta_w"][:n]
+    elif transport == "nccl":
+        send = epx.dispatch(x, lay)
+        meta_idx, meta_w = epx.route_meta(topk_idx, topk_weights, lay)
+        counts = exchange_counts(lay.cnt_r, pg)      # synchronises the stream
+        plan = send_plan(counts, rank)
+        n = plan["n_send"]
+        recv_x = exchange_rows(send[:n], plan, pg)
+        recv_idx = exchange_rows(meta_idx[:n], plan, pg)
+        recv_w = exchange_rows(meta_w[:n], plan, pg)
+    else:
+        raise ValueError(f"unknown transport {transport!r}")
     lay_in = epx.layout(recv_idx, E, world)
     _, expanded = epx.dispatch_expand(recv_x, lay_in, expand_only=True)
-    return Dispatched(lay, plan, recv_x, recv_idx, recv_w, lay_in, expanded, pg)
+    return Dispatched(lay, plan, recv_x, recv_idx, recv_w, lay_in, expanded, pg,
+                      buffers if transport == "p2p" else None)
 
 
 def combine(h: Dispatched, expert_out: torch.Tensor, residual: torch.Tensor = None,
             partial_dtype=torch.float32) -> torch.Tensor:
     """Multi-GPU combine: expert_out holds the expert outputs of h.expanded's
     rows.  The local reduce leaves one partial row per received row, in
-    receive order; those travel back by the reversed plan and land in the
-    source's receive layout, where the epilogue sums each token's partials
-    (plus `residual`, if given) and rounds once to bf16."""
+    receive order; those travel back (by the reversed plan, or stored
+    straight into the sources' buffers) and land in the source's receive
+    layout, where the epilogue sums each token's partials (plus `residual`,
+    if given) and rounds once to bf16."""
+    if h.buffers is not None:
+        b = h.buffers
+        if partial_dtype != b.partial_dtype:
+            raise ValueError("partial_dtype differs from the PeerBuffers' one")
+        world = b.world
+        peers = [epx.PeerRows(b.peer["back"][s], b.back_cap, row0=h.plan["back_row0"][s],
+                              first=h.plan["back_first"][s], count=h.plan["back_count"][s])
+                 for s in range(world)]
+        epx.combine_local_reduce_p2p(expert_out, h.recv_w, h.layout_in, peers,
+                                     partial_dtype=partial_dtype)
+        _order_ranks(h.pg, expert_out.device)
+        return epx.combine_epilogue(b.local["back"], h.layout, residual=residual)
     part = epx.combine_local_reduce(expert_out, h.recv_w, h.layout_in,
                                     partial_dtype=partial_dtype)
     back = exchange_rows(part[:h.plan["n_recv"]], h.plan, h.pg, reverse=True)

@@ -23,7 +23,8 @@ __all__ = [
     "EpxError", "Layout", "lib", "layout", "dispatch_expand", "standin_expert",
     "combine_reduce", "combine_local_reduce", "combine_epilogue", "read_totals",
     "dispatch", "expand_index", "standin_expert_gather", "layout_dispatch_expand",
-    "latency_floor", "route_meta",
+    "latency_floor", "route_meta", "PeerRows", "dispatch_p2p", "combine_local_reduce_p2p",
+    "ipc_malloc", "ipc_free", "ipc_open", "ipc_close", "tensor_at", "IPC_HANDLE_BYTES",
     "roundtrip_host", "roundtrip_device_bytes",
     "roundtrip_host_noalloc", "NOALLOC_SCRATCH_BYTES", "debug_dispatch_first_wait_limit",
     "LIB_PATH", "MAX_TOPK", "MAX_RANKS", "MAX_EXPERTS",
@@ -56,6 +57,15 @@ class _LayoutC(ctypes.Structure):
                 ("pos", ctypes.c_void_p), ("recv_pos", ctypes.c_void_p),
                 ("totals", ctypes.c_void_p), ("work", ctypes.c_void_p)]
 
+
+class _PeerRowsC(ctypes.Structure):
+    """ep_peer_rows_t."""
+    _fields_ = [("rows", ctypes.c_void_p), ("meta_idx", ctypes.c_void_p),
+                ("meta_w", ctypes.c_void_p), ("row0", ctypes.c_int64), ("cap", ctypes.c_int64),
+                ("first", ctypes.c_int64), ("count", ctypes.c_int64)]
+
+
+IPC_HANDLE_BYTES = 64             # EPX_IPC_HANDLE_BYTES
 
 _lib = None
 
@@ -100,6 +110,13 @@ def lib():
         "ep_layout_dispatch_expand_variant": ([P, LP, P, I32, P, I64, P, I64, I32, P], I32),
         "ep_latency_floor": ([P, I64, I32, P], I32),
         "ep_route_meta": ([P, P, LP, P, P, I64, P], I32),
+        "ep_dispatch_p2p": ([P, I32, LP, P, P, ctypes.POINTER(_PeerRowsC), P], I32),
+        "ep_combine_local_reduce_p2p": ([P, P, I32, LP, I32, I64, ctypes.POINTER(_PeerRowsC),
+                                         P], I32),
+        "ep_ipc_malloc": ([SZ, ctypes.POINTER(P), P], I32),
+        "ep_ipc_free": ([P], I32),
+        "ep_ipc_open": ([P, ctypes.POINTER(P)], I32),
+        "ep_ipc_close": ([P], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -271,6 +288,115 @@ def route_meta(topk_idx: torch.Tensor, topk_weights: torch.Tensor, lay: Layout,
                                _dev(meta_w, "meta_w", torch.float32), meta_idx.shape[0],
                                _stream(stream)), "ep_route_meta")
     return meta_idx, meta_w
+
+
+class PeerRows:
+    """One peer's buffers for ep_dispatch_p2p / ep_combine_local_reduce_p2p:
+    `rows` (and, for the dispatch, `meta_idx` / `meta_w`) as CUDA tensors or
+    raw device pointers (ints, e.g. from ipc_open), the first row this rank
+    writes there (`row0`), the rows the buffers hold (`cap`) and, for the
+    combine, the local partial rows [first, first + count) that go there."""
+
+    def __init__(self, rows, cap: int, row0: int = 0, meta_idx=None, meta_w=None,
+                 first: int = 0, count: int = 0):
+        self.rows, self.cap, self.row0 = rows, int(cap), int(row0)
+        self.meta_idx, self.meta_w = meta_idx, meta_w
+        self.first, self.count = int(first), int(count)
+
+
+def _ptr(v, name):
+    if v is None:
+        return None
+    if isinstance(v, torch.Tensor):
+        return _dev(v, name)
+    return int(v)
+
+
+def _peers_c(peers, R: int):
+    if len(peers) != R:
+        raise ValueError(f"{len(peers)} peer entries for {R} ranks")
+    arr = (_PeerRowsC * R)()
+    for r, e in enumerate(peers):
+        arr[r].rows = _ptr(e.rows, f"peers[{r}].rows")
+        arr[r].meta_idx = _ptr(e.meta_idx, f"peers[{r}].meta_idx")
+        arr[r].meta_w = _ptr(e.meta_w, f"peers[{r}].meta_w")
+        arr[r].row0, arr[r].cap = e.row0, e.cap
+        arr[r].first, arr[r].count = e.first, e.count
+    return arr
+
+
+def dispatch_p2p(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                 lay: Layout, peers, stream=None) -> None:
+    """ep_dispatch_p2p: every (token, rank) row of this rank's layout stored,
+    with its routing kept on that rank, at peers[r].row0 + (recv_pos[t, r] -
+    off_r[r]) of rank r's buffers."""
+    if x.dim() != 2 or x.shape[0] != lay.T:
+        raise ValueError("x must be [T, H]")
+    if topk_idx.shape != (lay.T, lay.k) or topk_weights.shape != (lay.T, lay.k):
+        raise ValueError("topk_idx and topk_weights must be [T, k]")
+    arr = _peers_c(peers, lay.R)
+    _check(lib().ep_dispatch_p2p(_dev(x, "x", torch.bfloat16), x.shape[1], lay.ref,
+                                 _dev(topk_idx, "topk_idx", (torch.int32, torch.int64)),
+                                 _dev(topk_weights, "topk_weights", torch.float32), arr,
+                                 _stream(stream)), "ep_dispatch_p2p")
+
+
+def combine_local_reduce_p2p(expert_out: torch.Tensor, topk_weights: torch.Tensor, lay: Layout,
+                             peers, partial_dtype=torch.float32, stream=None) -> None:
+    """ep_combine_local_reduce_p2p: the local reduce of ep_combine_local_reduce
+    with partial row d stored at row peers[s].row0 + (d - peers[s].first) of
+    peers[s].rows for the entry whose [first, first + count) holds d."""
+    if topk_weights.shape != (lay.T, lay.k):
+        raise ValueError("topk_weights must be [T, k]")
+    bits = {torch.float32: 32, torch.bfloat16: 16}[partial_dtype]
+    arr = _peers_c(peers, lay.R)
+    _check(lib().ep_combine_local_reduce_p2p(
+        _dev(expert_out, "expert_out", torch.bfloat16),
+        _dev(topk_weights, "topk_weights", torch.float32), expert_out.shape[1], lay.ref, bits,
+        expert_out.shape[0], arr, _stream(stream)), "ep_combine_local_reduce_p2p")
+
+
+def ipc_malloc(nbytes: int):
+    """ep_ipc_malloc: (device pointer, handle bytes) of a new allocation."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().ep_ipc_malloc(nbytes, ctypes.byref(ptr), handle), "ep_ipc_malloc")
+    return ptr.value, handle.raw
+
+
+def ipc_free(ptr: int) -> None:
+    _check(lib().ep_ipc_free(ptr), "ep_ipc_free")
+
+
+def ipc_open(handle: bytes) -> int:
+    """ep_ipc_open: another process's allocation mapped into this one."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be IPC_HANDLE_BYTES long")
+    ptr = ctypes.c_void_p()
+    _check(lib().ep_ipc_open(handle, ctypes.byref(ptr)), "ep_ipc_open")
+    return ptr.value
+
+
+def ipc_close(ptr: int) -> None:
+    _check(lib().ep_ipc_close(ptr), "ep_ipc_close")
+
+
+class _DevArray:
+    """A raw device pointer with shape and dtype, for torch.as_tensor (bf16
+    travels as int16 and is viewed back)."""
+
+    _TYPESTR = {torch.bfloat16: "<i2", torch.float32: "<f4", torch.int32: "<i4"}
+
+    def __init__(self, ptr: int, shape, dtype):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": self._TYPESTR[dtype],
+                                         "data": (int(ptr), False), "version": 3}
+
+
+def tensor_at(ptr: int, shape, dtype, device) -> torch.Tensor:
+    """A tensor view of device memory at `ptr` (not owned: the caller keeps
+    the allocation alive)."""
+    raw = torch.as_tensor(_DevArray(ptr, shape, dtype), device=device)
+    return raw.view(torch.bfloat16) if dtype == torch.bfloat16 else raw
 
 
 def latency_floor(buf: torch.Tensor, n_kernels: int = 3, stream=None) -> None:

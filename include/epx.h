@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define EPX_ABI_VERSION 2
+#define EPX_ABI_VERSION 3
 
 #define EPX_MAX_TOPK 32      /* k <= 32: one warp holds a token's routes      */
 #define EPX_MAX_RANKS 64     /* R <= 64: a token's rank set fits in 64 bits   */
@@ -391,6 +391,94 @@ ep_status_t ep_roundtrip_host_noalloc(const void *x_host, const void *topk_idx_h
                                       int32_t H, int32_t k, int32_t E, int32_t R,
                                       int32_t idx_bits, void *out_host,
                                       int32_t *dev_err_host, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Multi-GPU expert parallelism over peer memory (one process per GPU, rank r
+ * owning experts [r*E/R, (r+1)*E/R)): a token crosses to every rank that owns
+ * one of its experts exactly once, with its routing (DeepEP issue #48,
+ * question: token A on rank 0 "dispatched only once" to rank 1 for experts M
+ * and N), and the per-rank partial sums travel back (issue #48, answer on the
+ * reduction before the combine all2all).  The kernels below store those rows
+ * straight into the other GPUs' buffers (plain 16-byte stores through device
+ * pointers that map a peer's memory into this process, e.g. from
+ * ep_ipc_open; never a TMA copy): the placement of each row and the
+ * transfer are one kernel, in place of a dispatch kernel followed by an
+ * all-to-all.  The caller orders the ranks around them: all ranks' stores
+ * must have completed before a receiver reads its buffers (e.g. a one-word
+ * collective on every rank's stream after the kernel).  Nothing here waits
+ * on another GPU, so a rank that fails cannot leave a kernel spinning.
+ *
+ * One entry per peer (index = rank), host array of L->R entries:
+ */
+typedef struct {
+    void *rows;         /* device pointer (mapped peer memory or local): bf16
+                           [cap, H] rows for the dispatch, fp32 or bf16
+                           [cap, H] partial rows for the combine; 16-byte
+                           aligned */
+    int32_t *meta_idx;  /* dispatch: int32 [cap, k] routes kept on that rank
+                           (NULL: not written); combine: unused */
+    float *meta_w;      /* dispatch: fp32 [cap, k] their weights (NULL: not
+                           written); combine: unused */
+    int64_t row0;       /* first row this rank writes there */
+    int64_t cap;        /* rows the buffers hold; a row >= cap is skipped and
+                           flagged EP_DEVERR_RECV_CAP */
+    int64_t first;      /* combine: first local partial row that goes there */
+    int64_t count;      /* combine: partial rows that go there */
+} ep_peer_rows_t;
+
+/*
+ * Dispatch to peers: for every token t with a route on rank r (recv_pos[t,
+ * r] >= 0 in the layout *L of this rank's batch over R ranks), the row
+ *   q = peers[r].row0 + (recv_pos[t, r] - off_r[r])
+ * of rank r's buffers gets
+ *   rows[q]        = x[t]                           (bf16 [H]),
+ *   meta_idx[q, j] = topk_idx[t, j] if expert topk_idx[t, j] is on rank r,
+ *                    else -1,          meta_w[q, j] = its weight, else 0,
+ * i.e. what ep_dispatch + ep_route_meta would write into this rank's send
+ * buffer, stored instead at this source's place in the receiver's buffer
+ * (peers[r].row0 = the rows rank r receives from lower ranks).  Per rank r
+ * the received rows are then ordered by source rank, then by the source's
+ * token order.  x: device bf16 [T, H]; topk_idx / topk_weights as in
+ * ep_route_meta; the layout must come from ep_layout (or
+ * ep_layout_dispatch_expand) of the same topk_idx with R = the number of
+ * ranks.  The kernel ends with a system-scope fence.
+ */
+ep_status_t ep_dispatch_p2p(const void *x, int32_t H, const ep_layout_t *L,
+                            const void *topk_idx, const float *topk_weights,
+                            const ep_peer_rows_t *peers, void *stream);
+
+/*
+ * Local reduce to peers: ep_combine_local_reduce of the receiving rank, with
+ * each partial row stored at its source instead of locally: partial row d
+ * (in the receive layout of *L) with peers[s].first <= d < peers[s].first +
+ * peers[s].count goes to row peers[s].row0 + (d - peers[s].first) of
+ * peers[s].rows.  Arithmetic identical to ep_combine_local_reduce (fp32
+ * sums in k order, stored fp32 or bf16); a row that falls in no entry's
+ * range, or beyond its cap, is skipped and flagged EP_DEVERR_RECV_CAP.
+ * For the source, its partial rows then sit in its own receive layout, so
+ * ep_combine_epilogue applies unchanged.  The kernel ends with a
+ * system-scope fence.
+ */
+ep_status_t ep_combine_local_reduce_p2p(const void *expert_out, const float *topk_weights,
+                                        int32_t H, const ep_layout_t *L,
+                                        int32_t partial_bits, int64_t y_rows,
+                                        const ep_peer_rows_t *peers, void *stream);
+
+/*
+ * Device memory other processes can map (cudaIpcGetMemHandle /
+ * cudaIpcOpenMemHandle on an allocation of this library's own, so the
+ * handle covers exactly the buffer).  ep_ipc_malloc: bytes of device memory
+ * on the current device, its pointer in *dev_ptr and its handle in
+ * handle[0..EPX_IPC_HANDLE_BYTES).  ep_ipc_open: maps another process's
+ * handle into this one (peer access must be possible; the same process
+ * cannot open its own handle), pointer in *dev_ptr.  ep_ipc_close /
+ * ep_ipc_free undo them.  Errors: EP_ERR_INVALID_ARG, EP_ERR_CUDA.
+ */
+#define EPX_IPC_HANDLE_BYTES 64
+ep_status_t ep_ipc_malloc(size_t bytes, void **dev_ptr, void *handle);
+ep_status_t ep_ipc_free(void *dev_ptr);
+ep_status_t ep_ipc_open(const void *handle, void **dev_ptr);
+ep_status_t ep_ipc_close(void *dev_ptr);
 
 /*
  * Measurement helper: the latency floor of a step of this path.  Launches

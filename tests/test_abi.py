@@ -38,7 +38,7 @@ def test_header_declares_the_path():
 def test_every_declared_symbol_is_exported(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.ep_abi_version() == 2
+    assert lib.ep_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -162,6 +162,45 @@ def test_one_launch_call_validates_on_host(lib):
     assert lib.ep_latency_floor(None, 0, 3, None) == 1
     assert lib.ep_latency_floor(fake, 64, 3, None) == 1                            # too small
     assert lib.ep_latency_floor(fake + 4, 64 * 8, 3, None) == 2
+
+
+def test_peer_memory_calls_validate_on_host(lib):
+    """ep_dispatch_p2p / ep_combine_local_reduce_p2p / ep_ipc_* reject bad
+    arguments before touching the GPU."""
+    c = epx._LayoutC()
+    fake = 0x10000
+    n = lib.ep_layout_bytes(4, 2, 4, 2)
+    assert lib.ep_layout_init(ctypes.byref(c), 4, 2, 4, 2, 64, fake, n) == 0
+    peers = (epx._PeerRowsC * 2)()
+    for r in range(2):
+        peers[r].rows, peers[r].cap = fake, 8
+    d = lib.ep_dispatch_p2p
+    assert d(fake, 16, ctypes.byref(c), fake, fake, None, None) == 1          # no peers
+    assert d(fake, 12, ctypes.byref(c), fake, fake, peers, None) == 1         # H % 8
+    assert d(fake + 2, 16, ctypes.byref(c), fake, fake, peers, None) == 2     # x alignment
+    assert d(fake, 16, ctypes.byref(c), fake + 4, fake, peers, None) == 2     # idx alignment
+    peers[1].cap = -1
+    assert d(fake, 16, ctypes.byref(c), fake, fake, peers, None) == 1         # bad entry
+    peers[1].cap, peers[1].rows = 8, fake + 8
+    assert d(fake, 16, ctypes.byref(c), fake, fake, peers, None) == 1         # rows alignment
+    peers[1].rows = None
+    assert d(fake, 16, ctypes.byref(c), fake, fake, peers, None) == 1         # rows missing
+    peers[1].rows = fake
+    cl = lib.ep_combine_local_reduce_p2p
+    assert cl(fake, fake, 16, ctypes.byref(c), 8, 16, peers, None) == 1       # partial bits
+    assert cl(fake, fake, 16, ctypes.byref(c), 32, 16, None, None) == 1       # no peers
+    assert cl(fake + 2, fake, 16, ctypes.byref(c), 32, 16, peers, None) == 2
+    ptr = ctypes.c_void_p()
+    h = ctypes.create_string_buffer(epx.IPC_HANDLE_BYTES)
+    assert lib.ep_ipc_malloc(0, ctypes.byref(ptr), h) == 1
+    assert lib.ep_ipc_malloc(16, None, h) == 1
+    assert lib.ep_ipc_free(None) == 1
+    assert lib.ep_ipc_open(None, ctypes.byref(ptr)) == 1
+    assert lib.ep_ipc_close(None) == 1
+    src = open(HEADER).read()
+    assert int(re.search(r"#define EPX_IPC_HANDLE_BYTES (\d+)", src).group(1)) == \
+        epx.IPC_HANDLE_BYTES
+    assert ctypes.sizeof(epx._PeerRowsC) == 56
 
 
 def test_layout_block_holds_the_grid_workspace(lib):

@@ -170,3 +170,29 @@ def test_two_ranks_match_the_single_gpu_layout_split_by_rank():
         p.join(timeout=60)
     for r in range(world):
         assert res[r] == "ok", res[r]
+
+
+def test_p2p_plan_places_rows_where_the_all_to_all_does():
+    """The peer-memory transport's placements (ep_dist.p2p_plan) against
+    the all-to-all plan (send_plan): source s's rows for rank r start, in
+    r's buffer, where the all-to-all puts them (recv_offsets of r, entry s),
+    and r's partials for s go back to the start of s's send block for r."""
+    from combine_ep_layout_07_b200 import ep_dist
+    rng = np.random.default_rng(7)
+    for world in (1, 2, 3, 5):
+        counts = torch.from_numpy(rng.integers(0, 9, size=(world, world)))
+        counts[0, world - 1] = 0                     # an empty block
+        plans = [ep_dist.p2p_plan(counts, g) for g in range(world)]
+        sends = [ep_dist.send_plan(counts, g) for g in range(world)]
+        for s in range(world):
+            for r in range(world):
+                assert plans[s]["dispatch_row0"][r] == sends[r]["recv_offsets"][s]
+                assert plans[r]["back_first"][s] == sends[r]["recv_offsets"][s]
+                assert plans[r]["back_count"][s] == int(counts[s, r])
+                assert plans[r]["back_row0"][s] == sum(sends[s]["send_splits"][:r])
+            assert plans[s]["n_recv"] == sends[s]["n_recv"]
+            assert plans[s]["n_send"] == sends[s]["n_send"]
+    with pytest.raises(ValueError):
+        ep_dist.p2p_plan(torch.zeros(2, 3), 0)
+    with pytest.raises(ValueError):
+        ep_dist.p2p_plan(-torch.ones(2, 2), 0)
