@@ -2,7 +2,8 @@
  * epx -- MoE token dispatch and combine on one B200 (sm_100a).
  *
  * C ABI of libepx.so.  Every pointer documented as "device" is caller-owned
- * device memory; the library never allocates or frees memory.  Every call is
+ * device memory; the library allocates and frees memory only in
+ * ep_ipc_malloc / ep_ipc_free (memory other processes map).  Every call is
  * asynchronous on the given CUDA stream (`stream` is a cudaStream_t passed as
  * void*, NULL = the legacy default stream) except ep_layout_read_totals,
  * which synchronises that stream.
@@ -23,7 +24,10 @@
  *
  * Logical ranks: experts live on ranks in contiguous blocks of E/R
  * (expert e on rank e / (E/R)), as in the issue #760 reproduction's
- * local_experts.  All ranks are partitions of buffers on this one GPU.
+ * local_experts.  On one GPU all ranks are partitions of buffers on that
+ * GPU; with one process per GPU, ep_dispatch_p2p and
+ * ep_combine_local_reduce_p2p (below) store rows into the other ranks'
+ * buffers directly.
  *
  * Ordering: inside an expert's segment of `expanded` and inside a rank's
  * segment of `recv`, rows are ordered by token, then by top-k slot.  The
