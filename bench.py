@@ -823,7 +823,9 @@ def run_epx(args):
         sep_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_sep]
                   for i, (n, _) in enumerate(sep_calls)}
         sep_bytes = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
-                              args.idx_bits // 8, fused="separate")
+                              args.idx_bits // 8,
+                              None if step.part is None else step.part.element_size(),
+                              args.no_expand, fused="separate")
     names = step.names
     k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)
