@@ -66,6 +66,7 @@ CASES = [
     dict(R=2, E=16, k=4, H=64, T_of=[37, 50]),
     dict(R=4, E=32, k=6, H=136, T_of=[1, 0, 64, 9]),     # a rank with no tokens, k not 2^n
     dict(R=8, E=256, k=8, H=7168, T_of=[16] * 8),        # the decode shape, 16 tokens per rank
+    dict(R=64, E=128, k=32, H=8, T_of=[3] * 63 + [0]),   # R and k at their maxima
 ]
 
 
