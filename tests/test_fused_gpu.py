@@ -114,21 +114,21 @@ def test_fused_empty_batch():
     assert lay.off_e.cpu().sum().item() == 0 and lay.cnt_r.cpu().sum().item() == 0
 
 
-@pytest.mark.parametrize("T,variant", [(64, 1), (64, 2), (1536, 2)],
-                         ids=["one_launch", "paired_vec", "paired_bulk"])
+@pytest.mark.parametrize("T,variant,H", [(64, 1, 64), (64, 1, 4096), (64, 2, 64), (1536, 2, 64)],
+                         ids=["one_launch", "one_launch_bulk", "paired_vec", "paired_bulk"])
 @pytest.mark.parametrize("which", ["recv", "expanded", "both"])
-def test_fused_capacity_overflow_flagged_not_written(T, variant, which):
+def test_fused_capacity_overflow_flagged_not_written(T, variant, H, which):
     # "both": tokens whose every row lies beyond the capacities have their
     # chunk of x loaded before the dispatch's wait (paired path) and nothing
     # to write
-    wl = _random_wl(T=T, H=64, E=16, R=4, k=4, seed=10)
+    wl = _random_wl(T=T, H=H, E=16, R=4, k=4, seed=10)
     o = oracle.run_all(wl)
     x, idx, _ = gpu_inputs(wl)
     cap = 10
-    canary = {n: torch.full((cap + 4, 64), 7, dtype=torch.int16, device="cuda")
+    canary = {n: torch.full((cap + 4, H), 7, dtype=torch.int16, device="cuda")
               for n in ("recv", "expanded")}
     bufs = {n: (canary[n][:cap].view(torch.bfloat16) if which in (n, "both") else
-                torch.empty((T * 4, 64), dtype=torch.bfloat16, device="cuda"))
+                torch.empty((T * 4, H), dtype=torch.bfloat16, device="cuda"))
             for n in ("recv", "expanded")}
     lay, _, _ = epx.layout_dispatch_expand(idx, x, 16, 4, recv=bufs["recv"],
                                            expanded=bufs["expanded"], variant=variant)
@@ -145,10 +145,11 @@ def test_fused_capacity_overflow_flagged_not_written(T, variant, which):
     assert_layout_equal(lay, o["layout"])
 
 
-def test_fused_guard_bands_untouched():
-    wl = _random_wl(T=200, H=136, E=32, R=8, k=6, seed=11, p_pad=0.3)
+@pytest.mark.parametrize("H", [136, 4096], ids=["spread_stores", "bulk_stores"])
+def test_fused_guard_bands_untouched(H):
+    wl = _random_wl(T=200, H=H, E=32, R=8, k=6, seed=11, p_pad=0.3)
     o = oracle.run_all(wl)
-    T, H, k, R = 200, 136, 6, 8
+    T, k, R = 200, 6, 8
     x, idx, _ = gpu_inputs(wl)
     G = 3
     big_r = torch.full((T * min(k, R) + 2 * G, H), -3, dtype=torch.int16, device="cuda")
