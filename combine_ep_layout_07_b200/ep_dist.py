@@ -134,6 +134,9 @@ class PeerBuffers:
                   ("back", (self.back_cap, H), partial_dtype, pbytes * H)]
         self._own, self._opened = [], []
         self.local, self.peer = {}, {}
+        # every rank's capacities (a peer's buffers are written up to its own)
+        self.peer_recv_cap = [self.recv_cap] * world
+        self.peer_back_cap = [self.back_cap] * world
         handles = {}
         for name, shape, dtype, row_bytes in shapes:
             nbytes = max(16, shape[0] * row_bytes)
@@ -148,26 +151,40 @@ class PeerBuffers:
             handles[name] = (ptr, h)
         if world > 1:
             import torch.distributed as dist
-            mine = {n: h for n, (_, h) in handles.items()}
+            mine = dict(handles={n: h for n, (_, h) in handles.items()},
+                        recv_cap=self.recv_cap, back_cap=self.back_cap, H=H, k=k,
+                        partial=str(partial_dtype))
             gathered = [None] * world
             dist.all_gather_object(gathered, mine, group=pg)
+            if any((g["H"], g["k"], g["partial"]) != (H, k, str(partial_dtype)) for g in gathered):
+                self.close_local()
+                raise ValueError("PeerBuffers: H, k and partial_dtype must agree on every rank")
+            self.peer_recv_cap = [int(g["recv_cap"]) for g in gathered]
+            self.peer_back_cap = [int(g["back_cap"]) for g in gathered]
             for name, _, _, _ in shapes:
                 ptrs = []
                 for r in range(world):
                     if r == rank:
                         ptrs.append(handles[name][0])
                     else:
-                        p = epx.ipc_open(gathered[r][name])
+                        p = epx.ipc_open(gathered[r]["handles"][name])
                         self._opened.append(p)
                         ptrs.append(p)
                 self.peer[name] = ptrs
+
+    def close_local(self):
+        """Free this rank's own allocations (before any peer has mapped them)."""
+        for p in self._own:
+            epx.ipc_free(p)
+        self._own = []
 
     def close(self):
         """Unmap the other ranks' buffers and free this rank's (collective:
         every rank calls it, so no peer still writes into freed memory)."""
         if self.world > 1:
             import torch.distributed as dist
-            torch.cuda.synchronize(self.device)
+            if self.device.type == "cuda":
+                torch.cuda.synchronize(self.device)
             dist.barrier(group=self.pg)
         for p in self._opened:
             epx.ipc_close(p)
@@ -261,9 +278,9 @@ def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor
         counts = exchange_counts(lay.cnt_r, pg)      # synchronises the stream
         plan = p2p_plan(counts, rank)
         plan.update(send_plan(counts, rank))
-        if max(int(counts[:, r].sum()) for r in range(world)) > buffers.recv_cap:
+        if any(int(counts[:, r].sum()) > buffers.peer_recv_cap[r] for r in range(world)):
             raise ValueError("a rank receives more rows than its PeerBuffers hold")
-        peers = [epx.PeerRows(buffers.peer["rows"][r], buffers.recv_cap,
+        peers = [epx.PeerRows(buffers.peer["rows"][r], buffers.peer_recv_cap[r],
                               row0=plan["dispatch_row0"][r],
                               meta_idx=buffers.peer["meta_idx"][r],
                               meta_w=buffers.peer["meta_w"][r]) for r in range(world)]
@@ -303,7 +320,7 @@ def combine(h: Dispatched, expert_out: torch.Tensor, residual: torch.Tensor = No
         if partial_dtype != b.partial_dtype:
             raise ValueError("partial_dtype differs from the PeerBuffers' one")
         world = b.world
-        peers = [epx.PeerRows(b.peer["back"][s], b.back_cap, row0=h.plan["back_row0"][s],
+        peers = [epx.PeerRows(b.peer["back"][s], b.peer_back_cap[s], row0=h.plan["back_row0"][s],
                               first=h.plan["back_first"][s], count=h.plan["back_count"][s])
                  for s in range(world)]
         epx.combine_local_reduce_p2p(expert_out, h.recv_w, h.layout_in, peers,

@@ -196,3 +196,74 @@ def test_p2p_plan_places_rows_where_the_all_to_all_does():
         ep_dist.p2p_plan(torch.zeros(2, 3), 0)
     with pytest.raises(ValueError):
         ep_dist.p2p_plan(-torch.ones(2, 2), 0)
+
+
+def _peer_buffers_worker(rank, world, port, out_q, H_of):
+    """PeerBuffers' exchange on a gloo group, with the CUDA IPC calls of the
+    binding replaced by fakes that record what they were given: every rank
+    must map every other rank's handle, learn every rank's capacities, and
+    refuse a group whose ranks disagree on the row width."""
+    try:
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        sys.path.insert(0, ROOT)
+        from combine_ep_layout_07_b200 import ep_dist, epx
+        calls = dict(malloc=[], open=[], close=[], free=[])
+
+        def fake_malloc(nbytes):
+            ptr = 0x1000 * (rank + 1) + len(calls["malloc"])
+            calls["malloc"].append((nbytes, ptr))
+            return ptr, bytes([rank, len(calls["malloc"]) - 1]) + bytes(62)
+
+        epx.ipc_malloc = fake_malloc
+        epx.ipc_open = lambda h: calls["open"].append(h) or 0x900000 + h[0] * 16 + h[1]
+        epx.ipc_close = lambda p: calls["close"].append(p)
+        epx.ipc_free = lambda p: calls["free"].append(p)
+        epx.tensor_at = lambda ptr, shape, dtype, device: torch.zeros(shape, dtype=dtype)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        pg = dist.group.WORLD
+        t_max = [5, 7][rank]
+        H = H_of[rank]
+        if len(set(H_of)) > 1:
+            try:
+                ep_dist.PeerBuffers(t_max, H, 4, pg, device=torch.device("cpu"))
+                raise AssertionError("mismatched H accepted")
+            except ValueError:
+                pass
+            assert len(calls["free"]) == 4 and not calls["open"]   # own buffers freed, none mapped
+            out_q.put((rank, "ok"))
+            return
+        b = ep_dist.PeerBuffers(t_max, H, 4, pg, device=torch.device("cpu"))
+        assert b.peer_recv_cap == [2 * 5, 2 * 7] and b.peer_back_cap == [5 * 2, 7 * 2]
+        assert b.recv_cap == 2 * t_max and b.local["rows"].shape == (2 * t_max, H)
+        other = 1 - rank
+        for i, name in enumerate(("rows", "meta_idx", "meta_w", "back")):
+            assert b.peer[name][rank] == calls["malloc"][i][1]             # own allocation
+            assert b.peer[name][other] == 0x900000 + other * 16 + i        # the other's, mapped
+        assert calls["malloc"][0][0] == 2 * t_max * H * 2                  # bf16 rows
+        assert calls["malloc"][3][0] == t_max * 2 * H * 4                  # fp32 partials
+        b.close()
+        assert sorted(calls["close"]) == sorted(0x900000 + other * 16 + i for i in range(4))
+        assert sorted(calls["free"]) == sorted(p for _, p in calls["malloc"])
+        out_q.put((rank, "ok"))
+    except Exception:
+        out_q.put((rank, traceback.format_exc()))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("H_of", [(64, 64), (64, 128)], ids=["agree", "mismatch"])
+def test_peer_buffers_exchange_on_two_ranks(H_of):
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_buffers_worker, args=(r, world, port, q, H_of))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+    for r in range(world):
+        assert res[r] == "ok", res[r]
