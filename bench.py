@@ -167,6 +167,14 @@ def alg_bytes(T, T_real, N_recv, N_route, H, k, R, idx_bytes, part_bytes=None,
     return out
 
 
+def step_alg_bytes(T, tot, H, k, R, args, part_bytes, mode):
+    """alg_bytes of one step of the bench's own workload: the same options
+    (index width, two-stage partials, no-expand) in whichever form the calls
+    take (`mode`: one_launch, paired or separate)."""
+    return alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
+                     args.idx_bits // 8, part_bytes, args.no_expand, fused=mode)
+
+
 def sources_hash(kernel):
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[kernel]:
@@ -784,10 +792,8 @@ def run_epx(args):
         consumer = time_consumers(torch, epx, lay, recv, expanded, y, stream, dev, tot, H,
                                   max(10, min(args.steps, 200)))
 
-    bytes_ = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
-                       args.idx_bits // 8,
-                       None if step.part is None else step.part.element_size(), args.no_expand,
-                       fused=mode)
+    part_bytes = None if step.part is None else step.part.element_size()
+    bytes_ = step_alg_bytes(T, tot, H, k, R, args, part_bytes, mode)
     working = bytes_["total"]
     do_flush = args.flush == "always" or (args.flush == "auto" and working < 2 * L2_BYTES)
     l2flush = L2Flush(torch, dev)
@@ -822,10 +828,7 @@ def run_epx(args):
             pg=pg)
         sep_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_sep]
                   for i, (n, _) in enumerate(sep_calls)}
-        sep_bytes = alg_bytes(T, tot["T_real"], tot["N_recv"], tot["N_route"], H, k, R,
-                              args.idx_bits // 8,
-                              None if step.part is None else step.part.element_size(),
-                              args.no_expand, fused="separate")
+        sep_bytes = step_alg_bytes(T, tot, H, k, R, args, part_bytes, "separate")
     names = step.names
     k_ms = {n: [r[i] - (r[i - 1] if i else 0.0) for r in rec_k] for i, n in enumerate(names)}
     total_ms = reduce_max(pg, sum(step_ms), dev)

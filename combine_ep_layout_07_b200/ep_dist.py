@@ -273,6 +273,8 @@ def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor
     if transport == "p2p":
         if buffers is None:
             raise ValueError("transport 'p2p' needs PeerBuffers")
+        if buffers.world != world or buffers.rank != rank:
+            raise ValueError("PeerBuffers belong to another process group")
         if x.shape[0] * world > buffers.recv_cap or x.shape[1] != buffers.H:
             raise ValueError("batch larger than the PeerBuffers were sized for")
         counts = exchange_counts(lay.cnt_r, pg)      # synchronises the stream

@@ -117,3 +117,21 @@ def test_pinned_to_one_core_restores_affinity():
     with bench.PinnedToOneCore() as pin:
         assert os.sched_getaffinity(0) == {pin.core}
     assert os.sched_getaffinity(0) == before
+
+
+def test_split_pass_bytes_follow_the_step_options():
+    """The split pass of separate calls (paired steps) is charged the same
+    options as the step: two-stage partials, no-expand, index width."""
+    tot = dict(T_real=4096, N_recv=25936, N_route=32768)
+    for argv, part, keys in [([], None, {"layout", "dispatch_expand", "combine_reduce"}),
+                             (["--two-stage", "fp32"], 4,
+                              {"layout", "dispatch_expand", "combine_local", "combine_epilogue"}),
+                             (["--no-expand"], None, {"layout", "dispatch", "expand_index",
+                                                      "combine_reduce"})]:
+        a = bench.parse_args(argv)
+        sep = bench.step_alg_bytes(4096, tot, 7168, 8, 16, a, part, "separate")
+        assert set(sep) - {"total"} == keys
+        if not a.no_expand:
+            pair = bench.step_alg_bytes(4096, tot, 7168, 8, 16, a, part, "paired")
+            assert pair["total"] == sep["total"]
+            assert pair["layout_dispatch_expand"] == sep["layout"] + sep["dispatch_expand"]
