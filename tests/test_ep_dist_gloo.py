@@ -267,3 +267,60 @@ def test_peer_buffers_exchange_on_two_ranks(H_of):
         p.join(timeout=60)
     for r in range(world):
         assert res[r] == "ok", res[r]
+
+
+def test_p2p_placement_is_the_single_gpu_layout_split_by_rank():
+    """The peer-memory dispatch's placement rule -- source s writes its row
+    for (t, r) at p2p_plan(counts, s).dispatch_row0[r] + (recv_pos_s[t, r] -
+    off_r_s[r]) of rank r's buffer, with the routing kept on r -- computed
+    here with the oracle's layouts of each source's batch, must fill rank
+    r's buffer exactly as the single-GPU layout of all batches concatenated
+    in rank order fills rank r's block of recv (rows and routing), with no
+    row written twice or left empty; and the partials' return rule must put
+    every partial back at the source's own recv_pos row."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    from combine_ep_layout_07_b200 import ep_dist
+    for world in (2, 4):                 # E = 16 experts split evenly
+        parts = [_batch(g % 2) for g in range(world)]
+        lays = [oracle.layout(p[1], E, world) for p in parts]
+        counts = torch.tensor(np.stack([l["cnt_r"] for l in lays]))
+        gidx = np.concatenate([p[1] for p in parts])
+        gw = np.concatenate([p[2] for p in parts])
+        gx = np.concatenate([p[0] for p in parts])
+        glay = oracle.layout(gidx, E, world)
+        grecv, _ = oracle.dispatch_expand(gx, glay)
+        gmi, gmw = _meta(gidx, gw, glay, world)
+        for r in range(world):
+            n = int(counts[:, r].sum())
+            rows = np.full((n, H), 0xFFFF, np.uint16)
+            mi = np.full((n, K), -7, np.int32)
+            mw = np.full((n, K), -7.0, np.float32)
+            written = np.zeros(n, np.int64)
+            for s, (x, idx, w) in enumerate(parts):
+                plan = ep_dist.p2p_plan(counts, s)
+                lay = lays[s]
+                smi, smw = _meta(idx, w, lay, world)
+                for t in range(lay["T"]):
+                    q = lay["recv_pos"][t, r]
+                    if q < 0:
+                        continue
+                    row = plan["dispatch_row0"][r] + (q - lay["off_r"][r])
+                    rows[row], mi[row], mw[row] = x[t], smi[q], smw[q]
+                    written[row] += 1
+            assert np.all(written == 1)
+            lo, hi = glay["off_r"][r], glay["off_r"][r + 1]
+            np.testing.assert_array_equal(rows, grecv[lo:hi])
+            np.testing.assert_array_equal(mi, gmi[lo:hi])
+            np.testing.assert_array_equal(mw, gmw[lo:hi])
+            # the return trip: received row d from source s goes to the
+            # source's row back_row0[s] + (d - back_first[s]), which must be
+            # that source's own recv_pos row for (t, r)
+            plan_r = ep_dist.p2p_plan(counts, r)
+            for s in range(world):
+                lay = lays[s]
+                mine = [t for t in range(lay["T"]) if lay["recv_pos"][t, r] >= 0]
+                for i, t in enumerate(mine):
+                    d = plan_r["back_first"][s] + i
+                    assert plan_r["back_row0"][s] + (d - plan_r["back_first"][s]) == \
+                        lay["recv_pos"][t, r]
