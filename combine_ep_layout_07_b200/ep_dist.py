@@ -269,7 +269,8 @@ def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor
     are then views of buffers.local, valid until the next dispatch."""
     world, rank = _world(pg)
     E = num_experts
-    lay = epx.layout(topk_idx, E, world)
+    if transport not in ("p2p", "nccl"):
+        raise ValueError(f"unknown transport {transport!r}")
     if transport == "p2p":
         if buffers is None:
             raise ValueError("transport 'p2p' needs PeerBuffers")
@@ -277,6 +278,8 @@ def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor
             raise ValueError("PeerBuffers belong to another process group")
         if x.shape[0] * world > buffers.recv_cap or x.shape[1] != buffers.H:
             raise ValueError("batch larger than the PeerBuffers were sized for")
+    lay = epx.layout(topk_idx, E, world)
+    if transport == "p2p":
         counts = exchange_counts(lay.cnt_r, pg)      # synchronises the stream
         plan = p2p_plan(counts, rank)
         plan.update(send_plan(counts, rank))
@@ -301,8 +304,6 @@ def dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor
         recv_x = exchange_rows(send[:n], plan, pg)
         recv_idx = exchange_rows(meta_idx[:n], plan, pg)
         recv_w = exchange_rows(meta_w[:n], plan, pg)
-    else:
-        raise ValueError(f"unknown transport {transport!r}")
     lay_in = epx.layout(recv_idx, E, world)
     _, expanded = epx.dispatch_expand(recv_x, lay_in, expand_only=True)
     return Dispatched(lay, plan, recv_x, recv_idx, recv_w, lay_in, expanded, pg,

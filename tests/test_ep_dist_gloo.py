@@ -324,3 +324,24 @@ def test_p2p_placement_is_the_single_gpu_layout_split_by_rank():
                     d = plan_r["back_first"][s] + i
                     assert plan_r["back_row0"][s] + (d - plan_r["back_first"][s]) == \
                         lay["recv_pos"][t, r]
+
+
+def test_dispatch_arguments_are_checked_before_any_device_work():
+    """Bad transport arguments fail on the host, before a layout is launched
+    (the inputs here are CPU tensors a kernel could not take)."""
+    from combine_ep_layout_07_b200 import ep_dist
+    x = torch.zeros((4, 8), dtype=torch.bfloat16)
+    idx = torch.zeros((4, 2), dtype=torch.int64)
+    w = torch.zeros((4, 2), dtype=torch.float32)
+    with pytest.raises(ValueError, match="unknown transport"):
+        ep_dist.dispatch(x, idx, w, 4, transport="rdma")
+    with pytest.raises(ValueError, match="needs PeerBuffers"):
+        ep_dist.dispatch(x, idx, w, 4, transport="p2p")
+
+    class Fake:
+        world, rank, recv_cap, H = 2, 0, 8, 8
+    with pytest.raises(ValueError, match="another process group"):
+        ep_dist.dispatch(x, idx, w, 4, transport="p2p", buffers=Fake())
+    Fake.world, Fake.recv_cap = 1, 2
+    with pytest.raises(ValueError, match="larger than"):
+        ep_dist.dispatch(x, idx, w, 4, transport="p2p", buffers=Fake())
