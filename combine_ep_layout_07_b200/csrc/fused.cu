@@ -26,10 +26,11 @@
 //    token t) and a subset of the tokens, so the count has no cross-lane
 //    dependency until one shuffle sum at the end;
 //  * warp 0 adds the warps' counts and lists the destination rows; the CTA
-//    stores its chunk (staged in shared memory) to every destination row,
-//    the (row, vector) pairs spread over all threads so that a chunk of a
-//    few vectors still uses the whole CTA; chunk 0 of token t writes
-//    pos[t, :] and recv_pos[t, :];
+//    stores its chunk (staged in shared memory) to every destination row --
+//    a long chunk as one TMA bulk store per row, a short one with the (row,
+//    vector) pairs spread over all threads so that a chunk of a few vectors
+//    still uses the whole CTA; chunk 0 of token t writes pos[t, :] and
+//    recv_pos[t, :];
 //  * one extra CTA writes what no token CTA owns: the per-expert and per-rank
 //    counts and exclusive scans, the totals and the error word.
 //
